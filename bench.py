@@ -1,0 +1,373 @@
+"""Throughput benchmark of the fused Hyena forward (B*D*L elements/s).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one hyena_forward over the whole batch of the workload (all N
+orders, every row), inputs resident in HBM. The default workload is the
+order-2 bf16 B=8 D=768 L=2048 case. With N>1 (torchrun) every rank runs the
+same workload on its own GPU with its own seed, with no collective on the data
+path (weak scaling); the reported value is all ranks' elements divided by the
+slowest rank's time.
+
+Prints one JSON line on rank 0. See the design doc for the roofline arithmetic.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "order2_bf16_b8_d768_l2048"
+FP32_LANES_PER_SM = 128          # FP32 FMA lanes per SM (4 sub-partitions x 32)
+SM_MAX_MHZ_FALLBACK = 1965.0
+HBM_NOMINAL_GBS = 8000.0         # the operator's roofline convention (8 TB/s)
+L2_FLUSH_BYTES = 512 << 20       # > 126 MB L2, written between timed steps
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- cost model
+def cost_model(w):
+    """Algorithmic flops and bytes of one step (whole batch), per the operator's
+    roofline convention: 5 M log2 M flops per transform, two transforms per row
+    per order; bytes = v, N gates and y once each, plus every spectrum row once."""
+    io = 4 if w.dtype == "f32" else 2
+    N = w.order
+    if w.ndim == 1:
+        L = w.shape[0]
+        M = 1 << max(5, (2 * L - 1).bit_length())
+        transforms = 2 * N * w.B * w.D
+        flops = transforms * 5.0 * M * math.log2(M)
+        spec_bytes = N * w.D * (M // 2 + 1) * 8
+    else:
+        H, W = w.shape
+        M = (2 * H) * (2 * W)
+        transforms = 2 * N * w.B * w.D
+        flops = transforms * 5.0 * M * math.log2(M)
+        spec_bytes = N * w.D * (2 * H) * (W + 1) * 8
+    act_bytes = (N + 2) * w.elements * io
+    return {"flops": flops, "bytes": act_bytes + spec_bytes + N * w.D * 4, "M": M}
+
+
+def device_fp32_peak_tflops(sm_mhz):
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return sms * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12, sms
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": SM_MAX_MHZ_FALLBACK}, "fallback"
+
+
+# ------------------------------------------------------------- clock sampler
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 6:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        sm, smax = [], []
+        for s in self.samples:
+            try:
+                sm.append(float(s[0]))
+                smax.append(float(s[1]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, s[2:]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w, rank, world, dist):
+    import torch
+    from long_convolution_sequence_hyena_b200 import capi
+    from long_convolution_sequence_hyena_b200.api import Plan
+    from long_convolution_sequence_hyena_b200.workloads import make_inputs
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = make_inputs(w, seed=w.seed + 1000 * rank)
+    adt = inp["v"].dtype
+    v = inp["v"].to(dev)
+    gates = [g.to(dev) for g in inp["gates"]]
+    dskip = inp["dskip"].to(dev)
+    plan = Plan(w.shape, w.D, w.order, adt)
+    if "h" in inp:
+        H = plan.filter_spectrum(h=inp["h"].to(dev))
+    else:
+        imp = {k: (x.to(dev) if torch.is_tensor(x) else x) for k, x in inp["implicit"].items()}
+        H = plan.filter_spectrum(implicit=imp)
+    y = torch.empty_like(v)
+    ws_bytes = plan.workspace_bytes(w.B)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    gptrs = [g.data_ptr() for g in gates]
+
+    def step():
+        st = capi.hyena_forward(plan.handle, w.B, v.data_ptr(), gptrs, H.data_ptr(), dskip.data_ptr(),
+                                y.data_ptr(), ws.data_ptr() if ws_bytes else None, ws_bytes, sptr)
+        if st != capi.HYENA_OK:
+            raise RuntimeError("hyena_forward: " + capi.hyena_status_string(st))
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()                      # L2 flush, outside the timed events
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+
+    # end to end through the C ABI: pinned host inputs -> device, forward, result -> host
+    hv = inp["v"].pin_memory()
+    hg = [g.pin_memory() for g in inp["gates"]]
+    hy = torch.empty_like(hv).pin_memory()
+
+    def e2e_step():
+        v.copy_(hv, non_blocking=True)
+        for dst, src in zip(gates, hg):
+            dst.copy_(src, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    if dist is not None:
+        t = torch.tensor([ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    io = 4 if w.dtype == "f32" else 2
+    h2d = (w.order + 1) * w.elements * io
+    d2h = w.elements * io
+    plan.close()
+    return ms, step_ms, e2e_ms, h2d, d2h, clk
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def oracle_sample(w, seconds):
+    """Time the fp64 oracle on a bounded sample of the workload's rows (planes).
+    Returns (elements/s, sample description, threads)."""
+    import numpy as np
+
+    import oracle
+    from long_convolution_sequence_hyena_b200.workloads import make_inputs
+
+    small = w.scaled(B=1, D=min(w.D, 64), name=w.name + "_sample")
+    inp = make_inputs(small)
+    threads = oracle.num_threads()
+    N = w.order
+    if w.ndim == 1:
+        L = w.shape[0]
+        if "h" in inp:
+            h64 = inp["h"].double().numpy()
+        else:
+            p = inp["implicit"]
+            h64 = oracle.implicit_filter_1d(L, N, small.D, *(p[k].double().numpy() for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
+                                            p["alpha"].double().numpy(), p["num_freqs"], p["omega0"], p["omega_hidden"])
+        v = inp["v"].double().reshape(small.D, L).numpy()
+        g = inp["gates"].double().reshape(N, small.D, L).numpy()
+        d = inp["dskip"].double().numpy()
+
+        def run(rows):
+            idx = np.arange(rows) % small.D
+            oracle.hyena_1d(v[idx], g[:, idx], h64, d, fidx=idx)
+        unit = L
+    else:
+        H, W = w.shape
+        p = inp["implicit"]
+        k64 = oracle.implicit_filter_2d(H, W, N, small.D, *(p[k].double().numpy() for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
+                                        p["sigma"].double().numpy(), p["omega0"], p["omega_hidden"])
+        v = inp["v"].double().reshape(small.D, H, W).numpy()
+        g = inp["gates"].double().reshape(N, small.D, H, W).numpy()
+        d = inp["dskip"].double().numpy()
+
+        def run(rows):
+            idx = np.arange(rows) % small.D
+            oracle.hyena_2d(v[idx], g[:, idx], k64, d, fidx=idx)
+        unit = H * W
+    rows = threads
+    t0 = time.perf_counter()
+    run(rows)
+    dt = time.perf_counter() - t0
+    while dt < seconds / 4 and rows < 64 * threads:
+        rows *= 2
+        t0 = time.perf_counter()
+        run(rows)
+        dt = time.perf_counter() - t0
+    target = max(threads, int(rows * seconds / max(dt, 1e-9)) // threads * threads)
+    if target > rows:
+        rows = target
+        t0 = time.perf_counter()
+        run(rows)
+        dt = time.perf_counter() - t0
+    return rows * unit / dt, "%d rows of the workload (%d elements each), direct fp64 sum" % (rows, unit), threads, dt
+
+
+def main():
+    args = parse()
+    from long_convolution_sequence_hyena_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    metric = "Hyena op throughput (B·D·L elems/s)"
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    cfg = {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L, "channels": w.D, "order": w.order,
+           "shape": list(w.shape), "parallelism": "independent replicas x%d (no data-path collective)" % world,
+           "l2": "flushed between timed steps (512 MiB write)", "filters": w.filt}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        value, sample, threads, secs = oracle_sample(w, args.cpu_seconds)
+        line = {"metric": metric, "value": value, "unit": "elems/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": w.elements * world / value * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+                "impl": "reference",
+                "cpu_baseline": {"value": value, "unit": "elems/s", "cores": threads, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    ms, step_ms, e2e_ms, h2d, d2h, clk = run_ours(args, w, rank, world, dist)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    cost = cost_model(w)
+    peaks, peak_src = measured_peaks()
+    sm_max = peaks.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)
+    fp32_peak, sms = device_fp32_peak_tflops(sm_max)
+    sec = ms * 1e-3
+    achieved_tflops = cost["flops"] / sec / 1e12
+    achieved_gbs = cost["bytes"] / sec / 1e9
+    t_roof = max(cost["bytes"] / (HBM_NOMINAL_GBS * 1e9), cost["flops"] / (fp32_peak * 1e12))
+    value = w.elements * world / sec
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic_%s.json" % w.name)
+    try:
+        with open(prof) as f:
+            pj = json.load(f)
+        from long_convolution_sequence_hyena_b200.build import source_hash
+        if pj.get("source_hash") == source_hash():
+            traffic = pj.get("dram_bytes_per_launch")
+    except Exception:
+        traffic = None
+    line = {
+        "metric": metric, "value": value, "unit": "elems/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": achieved_tflops / fp32_peak, "traffic": traffic,
+                     "peak_source": "FP32 FMA lanes x2 x max SM clock (%d SMs, %.0f MHz)" % (sms, sm_max),
+                     "flops_convention": "5 M log2 M per transform, 2 transforms per row per order (M=%d)" % cost["M"],
+                     "hbm_achieved_gbs": achieved_gbs, "hbm_peak_gbs": peaks.get("hbm_gbs"),
+                     "hbm_frac": achieved_gbs / peaks.get("hbm_gbs", 6650.0), "hbm_peak_source": peak_src,
+                     "operator_roofline_frac": t_roof / sec},
+        "e2e": {"value": w.elements * world / (e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cv, sample, threads, _ = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": cv, "unit": "elems/s", "cores": threads, "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

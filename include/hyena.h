@@ -1,0 +1,176 @@
+/*
+ * hyena.h -- C ABI of the B200 (sm_100a) Hyena operator library (libhyena.so).
+ *
+ * The operator ("Hyena — Long Convolutions Math", "The Toeplitz picture";
+ * "Hyena, Long Convolution, and Linear Attention", "The Hyena operator" and
+ * "FFTConv: the O(L log L) primitive"):
+ *
+ *     z^0 = v
+ *     z^n = x^n ⊙ ( h^n ∗ z^{n-1}  +  Dskip^n ⊙ z^{n-1} )      n = 1..N
+ *     y   = z^N
+ *
+ * with ∗ a depthwise causal convolution along the sequence (1D) or a depthwise
+ * linear, non-causal convolution over a grid ("How HyenaND works", "2. The
+ * convolution theorem (FFT)"). Every convolution is computed by FFT on inputs
+ * zero-padded to M = next_pow2(2L) (per grid axis in 2D), so the cyclic
+ * product never wraps ("Hyena — Long Convolutions Math", "Linear vs circular").
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *    and 16-byte aligned, unless a comment says "host".
+ *  - Activation layout: 1D [B, D, L] (one channel row per (b, d));
+ *    2D [B, C, H, W]. io dtype is the plan's (fp32 or bf16); filters, spectra
+ *    and Dskip are always fp32 / complex64 (interleaved re, im).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only
+ *    enqueue work; none synchronises the host except plan create / destroy.
+ *  - Arguments are validated on the host before anything is launched; a call
+ *    that returns an error has launched nothing (HYENA_ERR_CUDA excepted: the
+ *    launch itself failed). Nothing aborts the process.
+ *  - Calls on one plan from several host threads are safe: a plan is read-only
+ *    after creation.
+ */
+#ifndef HYENA_H
+#define HYENA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HYENA_MAX_ORDER 8
+
+#if defined(__GNUC__)
+#define HYENA_API __attribute__((visibility("default")))
+#else
+#define HYENA_API
+#endif
+
+typedef struct hyena_plan_s *hyena_plan_t;
+
+typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype_t;
+
+typedef enum {
+    HYENA_OK = 0,
+    HYENA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+    HYENA_ERR_UNSUPPORTED = 2,   /* valid but outside what this build implements */
+    HYENA_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
+    HYENA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than hyena_workspace_bytes */
+    HYENA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+    HYENA_ERR_NOMEM = 6          /* host or device allocation failed (plan create only) */
+} hyena_status_t;
+
+/* Which kernel family a plan runs (hyena_plan_info). */
+typedef enum {
+    HYENA_PATH_CTA = 0,          /* 1D, M <= 32768: one CTA per row, all orders fused */
+    HYENA_PATH_CLUSTER = 1,      /* 1D, 32768 < M <= 262144: a thread-block cluster per row */
+    HYENA_PATH_2D = 2            /* 2D grid */
+} hyena_path_t;
+
+/*
+ * Parameters of the implicit filter network, all DEVICE pointers to fp32.
+ *
+ * 1D ("Hyena — Long Convolutions Math", "Implicit filters: an MLP over
+ * positions" and "The decay window"): positional features
+ *   g(t) = [t/L, cos(2π·1·t/L), sin(2π·1·t/L), ..., cos(2π·K·t/L), sin(2π·K·t/L)]
+ * (in = 1 + 2K, K = num_freqs), then
+ *   a1 = sin(omega0 (W1 g + b1)), a2 = sin(omega_hidden (W2 a1 + b2)), o = W3 a2 + b3,
+ *   h[n, d, t] = exp(-window[n*D + d] * t) * o[n*D + d]        (window = decay rates α ≥ 0)
+ * 2D ("How HyenaND works", "1. An implicit filter"): coordinates
+ *   p = (oy / H, ox / W), oy in [-H, H), ox in [-W, W)  (in = 2, num_freqs ignored),
+ *   same two sine layers and head, K[n, c, oy + H, ox + W] =
+ *   exp(-|p|^2 / (2 window[n*C + c]^2)) * o[n*C + c]           (window = Gaussian σ > 0)
+ * Shapes: W1 [width, in], b1 [width], W2 [width, width], b2 [width],
+ * W3 [N*D, width], b3 [N*D], window [N*D]; row-major. width <= 128 and a
+ * multiple of 4; num_freqs <= 32. W3 must be 16-byte aligned.
+ */
+typedef struct {
+    const float *W1, *b1, *W2, *b2, *W3, *b3;
+    const float *window;
+    int32_t width;
+    int32_t num_freqs;
+    float omega0;
+    float omega_hidden;
+} hyena_implicit_params_t;
+
+/*
+ * Create a plan.
+ *   ndim      1 (sequence) or 2 (grid)
+ *   shape     host array of ndim sizes: {L} or {H, W}; each >= 1.
+ *             1D: L <= 131072. 2D: H, W powers of two with 2H, 2W <= 1024.
+ *   channels  D (1D) or C (2D), >= 1
+ *   order     N, 1..HYENA_MAX_ORDER
+ *   io_dtype  storage type of v, the gates and y
+ *   causal    must be 1 for ndim 1 and 0 for ndim 2
+ * Allocates the plan's device twiddle tables on the current device (the plan
+ * may only be used on that device) and synchronises. *out is NULL on error.
+ */
+HYENA_API hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *shape, int64_t channels,
+                                 int order, hyena_dtype_t io_dtype, int causal);
+
+/* Free the plan's device tables (synchronises the device). NULL is accepted. */
+HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);
+
+/*
+ * Geometry of a plan (any out-pointer may be NULL):
+ *   fft_len        M (1D) or 2H * 2W (2D): the padded transform size
+ *   spectrum_elems complex64 elements of one (order, channel) spectrum:
+ *                  M/2 + 1 (1D) or 2H * (W + 1) (2D)
+ *   path           a hyena_path_t
+ */
+HYENA_API hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path);
+
+/* Bytes of device workspace hyena_forward needs for `batch` (0 for on-chip paths). */
+HYENA_API size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch);
+
+/*
+ * Evaluate the implicit filter network (see hyena_implicit_params_t) into
+ * h_out: [N, D, L] (1D) or [N, C, 2H, 2W] (2D) fp32, device.
+ */
+HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_implicit_params_t *params,
+                                     float *h_out, void *stream);
+
+/*
+ * Filter spectra ("Hyena — Long Convolutions Math", "The convolution theorem":
+ * FFT(h) is the filter's transfer function, one gain per frequency).
+ *   h       1D: [N, D, L] causal taps 0..L-1 (zero-extended to M);
+ *           2D: [N, C, 2H, 2W] kernel on the offset grid, element (oy, ox) at
+ *           [oy + H, ox + W], oy in [-H, H), ox in [-W, W).
+ *           May be NULL when params is given: the filters are then generated by
+ *           the implicit network, inside H_out, with no other memory.
+ *   params  implicit network, or NULL (then h must not be NULL)
+ *   H_out   1D: [N, D, M/2 + 1] complex64, bin k = sum_t h[t] e^{-2πi k t / M};
+ *           2D: [N, C, 2H, W + 1] complex64, the 2D DFT of the kernel placed
+ *           cyclically (offset o at index o mod 2H, o mod 2W), bins over the
+ *           full row axis and the non-negative half of the column axis.
+ *           Unnormalised. Must not overlap h.
+ */
+HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
+                                     void *H_out, void *stream);
+
+/*
+ * The fused forward pass: all N orders in one launch per row, each row read
+ * once from and written once to device memory.
+ *   batch      B >= 0 (B = 0 launches nothing)
+ *   v          [B, D, L] or [B, C, H, W], io dtype
+ *   gates      HOST array of N device pointers x^1..x^N, each shaped like v
+ *   H          spectra from hyena_filter_spectrum
+ *   Dskip      [N, D] fp32 feedthrough, or NULL for none
+ *   y          output, shaped like v, io dtype; may alias v or a gate
+ *              (each row is read completely before it is written)
+ *   workspace  device scratch of at least hyena_workspace_bytes(plan, batch)
+ *              bytes, or NULL when that is 0
+ */
+HYENA_API hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, const void *const *gates,
+                             const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* Static, human-readable name of a status code. */
+HYENA_API const char *hyena_status_string(hyena_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_H */

@@ -1,0 +1,235 @@
+// Register-resident FFT building blocks for sm_100a.
+//
+// A CTA-level complex FFT of length Mc is run as Stockham passes: each thread
+// keeps E complex values in registers, performs radix-16 (or a final radix-2/4/8)
+// butterflies on them, and the threads exchange data through shared memory
+// between passes. Thread t holds element t + q*T in register q (T = Mc / E)
+// both before the first pass and after the last one (natural order), so
+// element-wise work (loads, gating, the spectral product) happens in registers.
+//
+// Shared memory holds the exchange buffer as two float planes (re, im). The
+// write pattern of a pass with stride Ns = 16^p is made bank-conflict-free with
+// an XOR swizzle of the low five index bits; reads of the next pass are
+// consecutive per warp and stay conflict-free under the same swizzle.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <utility>
+
+namespace hyena {
+
+// Compile-time loop: f(std::integral_constant<int, i>) for i = 0..N-1.
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F &&f, std::integer_sequence<int, I...>) {
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F &&f) {
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+struct c32 {
+    float x, y;
+};
+
+__device__ __forceinline__ c32 mk(float x, float y) { return c32{x, y}; }
+__device__ __forceinline__ c32 add(c32 a, c32 b) { return c32{a.x + b.x, a.y + b.y}; }
+__device__ __forceinline__ c32 sub(c32 a, c32 b) { return c32{a.x - b.x, a.y - b.y}; }
+__device__ __forceinline__ c32 mul(c32 a, c32 b) {
+    return c32{fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x)};
+}
+__device__ __forceinline__ c32 conj(c32 a) { return c32{a.x, -a.y}; }
+__device__ __forceinline__ c32 scale(c32 a, float s) { return c32{a.x * s, a.y * s}; }
+// a * (DIR * i): multiply by +i (DIR = +1) or -i (DIR = -1)
+template <int DIR>
+__device__ __forceinline__ c32 rot90(c32 a) {
+    return DIR > 0 ? c32{-a.y, a.x} : c32{a.y, -a.x};
+}
+
+// cos / sin of k*pi/8 for the radix-16 internal twiddles (exact math constants)
+#define HY_C1 0.92387953251128675613f  // cos(pi/8)
+#define HY_S1 0.38268343236508977173f  // sin(pi/8)
+#define HY_R2 0.70710678118654752440f  // sqrt(1/2)
+
+// W_16^m = exp(DIR * 2 pi i m / 16) for the m that a 4x4 split needs.
+template <int DIR, int m>
+__device__ __forceinline__ c32 tw16(c32 a) {
+    constexpr float s = (float)DIR;
+    if constexpr (m == 0) return a;
+    else if constexpr (m == 1) return mul(a, c32{HY_C1, s * HY_S1});
+    else if constexpr (m == 2) return mul(a, c32{HY_R2, s * HY_R2});
+    else if constexpr (m == 3) return mul(a, c32{HY_S1, s * HY_C1});
+    else if constexpr (m == 4) return rot90<DIR>(a);
+    else if constexpr (m == 6) return mul(a, c32{-HY_R2, s * HY_R2});
+    else if constexpr (m == 9) return mul(a, c32{-HY_C1, -s * HY_S1});
+    else return a;  // not reached
+}
+
+template <int DIR, int m>
+__device__ __forceinline__ c32 tw8(c32 a) {
+    constexpr float s = (float)DIR;
+    if constexpr (m == 0) return a;
+    else if constexpr (m == 1) return mul(a, c32{HY_R2, s * HY_R2});
+    else if constexpr (m == 2) return rot90<DIR>(a);
+    else return mul(a, c32{-HY_R2, s * HY_R2});  // m == 3
+}
+
+// In-place 4-point DFT, X[k] = sum_n a[n] W_4^{nk}, W_4 = exp(DIR 2 pi i / 4).
+template <int DIR>
+__device__ __forceinline__ void dft4(c32 &a0, c32 &a1, c32 &a2, c32 &a3) {
+    c32 s02 = add(a0, a2), d02 = sub(a0, a2);
+    c32 s13 = add(a1, a3), d13 = rot90<DIR>(sub(a1, a3));
+    a0 = add(s02, s13);
+    a2 = sub(s02, s13);
+    a1 = add(d02, d13);
+    a3 = sub(d02, d13);
+}
+
+// 4-point DFT of (a0, a1, 0, 0).
+template <int DIR>
+__device__ __forceinline__ void dft4_half(c32 &a0, c32 &a1, c32 &a2, c32 &a3) {
+    c32 j1 = rot90<DIR>(a1);
+    a2 = sub(a0, a1);
+    a3 = sub(a0, j1);
+    c32 t = a0;
+    a0 = add(t, a1);
+    a1 = add(t, j1);
+}
+
+__device__ __forceinline__ void dft2(c32 &a0, c32 &a1) {
+    c32 t = a0;
+    a0 = add(t, a1);
+    a1 = sub(t, a1);
+}
+
+// 16-point DFT on x[o + st*n], n = 0..15, result in natural order at the same
+// positions. Split n = 4 n1 + n2, k = k1 + 4 k2. HALF: inputs n >= 8 are zero.
+template <int DIR, bool HALF, int st, int o, int NR>
+__device__ __forceinline__ void dft16(c32 (&x)[NR]) {
+#define X(i) x[o + st * (i)]
+    // DFT4 over n1 for each n2; result A[n2][k1] kept at position 4*k1 + n2
+    if constexpr (HALF) {
+        dft4_half<DIR>(X(0), X(4), X(8), X(12));
+        dft4_half<DIR>(X(1), X(5), X(9), X(13));
+        dft4_half<DIR>(X(2), X(6), X(10), X(14));
+        dft4_half<DIR>(X(3), X(7), X(11), X(15));
+    } else {
+        dft4<DIR>(X(0), X(4), X(8), X(12));
+        dft4<DIR>(X(1), X(5), X(9), X(13));
+        dft4<DIR>(X(2), X(6), X(10), X(14));
+        dft4<DIR>(X(3), X(7), X(11), X(15));
+    }
+    // twiddles W_16^{n2 k1}
+    X(5) = tw16<DIR, 1>(X(5));
+    X(6) = tw16<DIR, 2>(X(6));
+    X(7) = tw16<DIR, 3>(X(7));
+    X(9) = tw16<DIR, 2>(X(9));
+    X(10) = tw16<DIR, 4>(X(10));
+    X(11) = tw16<DIR, 6>(X(11));
+    X(13) = tw16<DIR, 3>(X(13));
+    X(14) = tw16<DIR, 6>(X(14));
+    X(15) = tw16<DIR, 9>(X(15));
+    // DFT4 over n2 for each k1: X[k1 + 4 k2] lands at position 4*k1 + k2
+    dft4<DIR>(X(0), X(1), X(2), X(3));
+    dft4<DIR>(X(4), X(5), X(6), X(7));
+    dft4<DIR>(X(8), X(9), X(10), X(11));
+    dft4<DIR>(X(12), X(13), X(14), X(15));
+    // transpose 4x4 back to natural order
+    c32 t;
+    t = X(1); X(1) = X(4); X(4) = t;
+    t = X(2); X(2) = X(8); X(8) = t;
+    t = X(3); X(3) = X(12); X(12) = t;
+    t = X(6); X(6) = X(9); X(9) = t;
+    t = X(7); X(7) = X(13); X(13) = t;
+    t = X(11); X(11) = X(14); X(14) = t;
+#undef X
+}
+
+// 8-point DFT on x[o + st*n], n = 0..7 (split n = 2 n1 + n2, k = k1 + 4 k2).
+template <int DIR, int st, int o, int NR>
+__device__ __forceinline__ void dft8(c32 (&x)[NR]) {
+#define X(i) x[o + st * (i)]
+    dft4<DIR>(X(0), X(2), X(4), X(6));   // n2 = 0 -> A[0][k1] at 2*k1
+    dft4<DIR>(X(1), X(3), X(5), X(7));   // n2 = 1 -> A[1][k1] at 2*k1 + 1
+    X(3) = tw8<DIR, 1>(X(3));
+    X(5) = tw8<DIR, 2>(X(5));
+    X(7) = tw8<DIR, 3>(X(7));
+    dft2(X(0), X(1));                    // X[k1 + 4 k2] at 2*k1 + k2
+    dft2(X(2), X(3));
+    dft2(X(4), X(5));
+    dft2(X(6), X(7));
+    c32 t;                               // positions 2k1+k2 -> k1+4k2
+    t = X(1); X(1) = X(2); X(2) = X(4); X(4) = t;
+    t = X(3); X(3) = X(6); X(6) = X(5); X(5) = t;
+#undef X
+}
+
+template <int DIR, int st, int o, int NR>
+__device__ __forceinline__ void dft4r(c32 (&x)[NR]) {
+    dft4<DIR>(x[o], x[o + st], x[o + 2 * st], x[o + 3 * st]);
+}
+
+template <int DIR, int st, int o, int NR>
+__device__ __forceinline__ void dft2r(c32 (&x)[NR]) {
+    dft2(x[o], x[o + st]);
+}
+
+template <int R, int DIR, bool HALF, int st, int o, int NR>
+__device__ __forceinline__ void dftR(c32 (&x)[NR]) {
+    if constexpr (R == 16) dft16<DIR, HALF, st, o>(x);
+    else if constexpr (R == 8) dft8<DIR, st, o>(x);
+    else if constexpr (R == 4) dft4r<DIR, st, o>(x);
+    else dft2r<DIR, st, o>(x);
+}
+
+// Powers w^1..w^(R-1) of a twiddle applied to x[o + st*r], built by a product
+// tree of depth <= 4 from one table value.
+template <int R, int st, int o, int NR>
+__device__ __forceinline__ void twiddle_powers(c32 (&x)[NR], c32 w1) {
+    if constexpr (R >= 2) x[o + st] = mul(x[o + st], w1);
+    if constexpr (R >= 4) {
+        c32 w2 = mul(w1, w1);
+        c32 w3 = mul(w2, w1);
+        x[o + 2 * st] = mul(x[o + 2 * st], w2);
+        x[o + 3 * st] = mul(x[o + 3 * st], w3);
+        if constexpr (R >= 8) {
+            c32 w4 = mul(w2, w2);
+            c32 w5 = mul(w4, w1), w6 = mul(w4, w2), w7 = mul(w4, w3);
+            x[o + 4 * st] = mul(x[o + 4 * st], w4);
+            x[o + 5 * st] = mul(x[o + 5 * st], w5);
+            x[o + 6 * st] = mul(x[o + 6 * st], w6);
+            x[o + 7 * st] = mul(x[o + 7 * st], w7);
+            if constexpr (R >= 16) {
+                c32 w8 = mul(w4, w4);
+                x[o + 8 * st] = mul(x[o + 8 * st], w8);
+                x[o + 9 * st] = mul(x[o + 9 * st], mul(w8, w1));
+                x[o + 10 * st] = mul(x[o + 10 * st], mul(w8, w2));
+                x[o + 11 * st] = mul(x[o + 11 * st], mul(w8, w3));
+                x[o + 12 * st] = mul(x[o + 12 * st], mul(w8, w4));
+                x[o + 13 * st] = mul(x[o + 13 * st], mul(w8, w5));
+                x[o + 14 * st] = mul(x[o + 14 * st], mul(w8, w6));
+                x[o + 15 * st] = mul(x[o + 15 * st], mul(w8, w7));
+            }
+        }
+    }
+}
+
+// Swizzle of an exchange-buffer index written by a pass of stride Ns.
+template <int NS>
+__device__ __forceinline__ int swz(int i) {
+    if constexpr (NS == 1) return i ^ ((i >> 5) & 15);
+    else if constexpr (NS == 16) return i ^ (((i >> 8) & 1) << 4);
+    else return i;
+}
+
+// Radix of pass p for an FFT of length Mc: radix-16 passes, then one radix
+// 2/4/8 pass for the remaining factor.
+constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
+constexpr int num_passes(int Mc) { return (ilog2(Mc) + 3) / 4; }
+constexpr int pass_radix(int Mc, int p) {
+    return (p < ilog2(Mc) / 4) ? 16 : (1 << (ilog2(Mc) % 4));
+}
+constexpr int pass_stride(int Mc, int p) { return 1 << (4 * p); }  // Ns = 16^p
+
+}  // namespace hyena

@@ -1,0 +1,235 @@
+// 1D kernels: the fused order-N forward (one CTA group per channel row) and the
+// filter spectrum. Launch wrappers are declared in launch.h.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "cta_fft.cuh"
+#include "hyena.h"
+
+namespace hyena {
+
+struct Fwd1dArgs {
+    const void *v;
+    const void *gates[HYENA_MAX_ORDER];
+    const c32 *H;         // [N, D, MC + 1]
+    const float *dskip;   // [N, D] or nullptr
+    void *y;
+    const c32 *tw;        // W_M^m, m in [0, M)
+    int64_t rows;         // B * D
+    int64_t L;
+    int64_t D;
+    int64_t B;
+    int order;
+};
+
+constexpr int rows_per_cta(int MC, int E) { return (MC / E) >= 128 ? 1 : 128 / (MC / E); }
+
+// ---- activation I/O: element pairs (x[2k], x[2k+1]) as one complex value ----
+template <typename IO>
+struct io;
+
+template <>
+struct io<float> {
+    using pair_t = float2;
+    __device__ __forceinline__ static c32 unpack(pair_t p) { return mk(p.x, p.y); }
+    __device__ __forceinline__ static pair_t pack(c32 a) { return make_float2(a.x, a.y); }
+    __device__ __forceinline__ static float to_f(float a) { return a; }
+    __device__ __forceinline__ static float from_f(float a) { return a; }
+    __device__ __forceinline__ static pair_t zero() { return make_float2(0.f, 0.f); }
+};
+
+template <>
+struct io<__nv_bfloat16> {
+    using pair_t = __nv_bfloat162;
+    __device__ __forceinline__ static c32 unpack(pair_t p) {
+        const float2 f = __bfloat1622float2(p);
+        return mk(f.x, f.y);
+    }
+    __device__ __forceinline__ static pair_t pack(c32 a) { return __floats2bfloat162_rn(a.x, a.y); }
+    __device__ __forceinline__ static float to_f(__nv_bfloat16 a) { return __bfloat162float(a); }
+    __device__ __forceinline__ static __nv_bfloat16 from_f(float a) { return __float2bfloat16_rn(a); }
+    __device__ __forceinline__ static pair_t zero() { return __floats2bfloat162_rn(0.f, 0.f); }
+};
+
+// Load positions (pos, pos+1) of a row of length L, zero beyond L.
+// EVEN: L is even, so the pair is either fully inside or fully outside and the
+// pair load is aligned.
+template <typename IO, bool EVEN>
+__device__ __forceinline__ c32 load_pair(const IO *__restrict__ row, int64_t pos, int64_t L) {
+    if constexpr (EVEN) {
+        if (pos < L) return io<IO>::unpack(__ldg(reinterpret_cast<const typename io<IO>::pair_t *>(row + pos)));
+        return mk(0.f, 0.f);
+    } else {
+        const float a = pos < L ? io<IO>::to_f(row[pos]) : 0.f;
+        const float b = pos + 1 < L ? io<IO>::to_f(row[pos + 1]) : 0.f;
+        return mk(a, b);
+    }
+}
+
+template <typename IO, bool EVEN>
+__device__ __forceinline__ void store_pair(IO *__restrict__ row, int64_t pos, int64_t L, c32 val) {
+    if constexpr (EVEN) {
+        if (pos < L) *reinterpret_cast<typename io<IO>::pair_t *>(row + pos) = io<IO>::pack(val);
+    } else {
+        if (pos < L) row[pos] = io<IO>::from_f(val.x);
+        if (pos + 1 < L) row[pos + 1] = io<IO>::from_f(val.y);
+    }
+}
+
+__device__ __forceinline__ c32 ldg_c(const c32 *p) {
+    const float2 f = __ldg(reinterpret_cast<const float2 *>(p));
+    return mk(f.x, f.y);
+}
+
+// Spectral step of one order for a row held as packed complex spectrum Z
+// (natural order in registers): unpack the real-row spectrum X, multiply by
+// the filter gain plus the feedthrough (the feedthrough is the delta tap, whose
+// spectrum is the constant Dskip), repack for the half-length inverse, and fold
+// in the 1/2 of the repacking and the 1/MC of the inverse transform.
+template <int MC, int E>
+__device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim,
+                                                 int t, const c32 *__restrict__ Hrow, float dsk,
+                                                 const c32 *__restrict__ tw) {
+    constexpr int T = MC / E;
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        sre[t + q * T] = v[q].x;
+        sim[t + q * T] = v[q].y;
+    }
+    __syncthreads();
+    constexpr float s = 0.5f / (float)MC;
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int k = t + q * T;
+        const int km = (MC - k) & (MC - 1);
+        const c32 Zk = v[q];
+        const c32 Zm = mk(sre[km], sim[km]);
+        const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
+        const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
+        const c32 w = ldg_c(tw + k);
+        const c32 wO = mul(w, Ok);
+        const c32 Xk = add(Ek, wO);
+        const c32 Xm = conj(sub(Ek, wO));
+        c32 Hk = ldg_c(Hrow + k);
+        c32 Hm = ldg_c(Hrow + (MC - k));
+        Hk.x += dsk;
+        Hm.x += dsk;
+        const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
+        const c32 Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
+        const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
+        const c32 Yo = mul(Yd, conj(w));
+        v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+    }
+    __syncthreads();
+}
+
+// Fused order-N forward, one group of MC/E threads per channel row.
+// Grid: ceil(B*D / rows_per_cta) CTAs, rows visited d-major / b-minor so the B
+// rows that read the same filter spectrum run at the same time (L2 reuse).
+template <int MC, int E, typename IO, bool EVEN>
+__global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
+    hyena_fwd_1d_cta(const Fwd1dArgs a) {
+    constexpr int T = MC / E;
+    constexpr int RPC = rows_per_cta(MC, E);
+    extern __shared__ float smem[];
+    const int lrow = threadIdx.x / T;
+    const int t = threadIdx.x - lrow * T;
+    const int64_t ord = (int64_t)blockIdx.x * RPC + lrow;
+    const bool active = ord < a.rows;
+    const int64_t d = active ? ord / a.B : 0;
+    const int64_t b = active ? ord - d * a.B : 0;
+    const int64_t row = b * a.D + d;
+    float *sre = smem + lrow * 2 * MC;
+    float *sim = sre + MC;
+    const int64_t L = a.L;
+
+    c32 v[E];
+    {
+        const IO *vrow = reinterpret_cast<const IO *>(a.v) + row * L;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q)
+            v[q] = active ? load_pair<IO, EVEN>(vrow, 2 * (int64_t)(t + q * T), L) : mk(0.f, 0.f);
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+    }
+
+    for (int n = 0; n < a.order; ++n) {
+        const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + row * L;
+        c32 g[E / 2];
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q)
+            g[q] = active ? load_pair<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L) : mk(0.f, 0.f);
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
+
+        fft_cta<MC, E, -1, true>(v, sre, sim, t, a.tw);
+        spectral_product<MC, E>(v, sre, sim, t, a.H + ((int64_t)n * a.D + d) * (MC + 1), dsk, a.tw);
+        fft_cta<MC, E, +1, false>(v, sre, sim, t, a.tw);
+
+        // gate; positions >= L are cleared so the next order sees a zero-padded row
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = 2 * (int64_t)(t + q * T);
+            v[q] = mk(pos < L ? g[q].x * v[q].x : 0.f, pos + 1 < L ? g[q].y * v[q].y : 0.f);
+        }
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+    }
+
+    if (active) {
+        IO *yrow = reinterpret_cast<IO *>(a.y) + row * L;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) store_pair<IO, EVEN>(yrow, 2 * (int64_t)(t + q * T), L, v[q]);
+    }
+}
+
+// Spectrum of causal real filters: Hout[o, k] = sum_t h[o, t] e^{-2 pi i k t / M},
+// k in [0, MC]. Input row o starts at h + o * h_stride (floats) and has L taps.
+// May run in place (h_stride = 2 (MC + 1), h == Hout): a row is read completely
+// before the first barrier, and only its own slot is written.
+template <int MC, int E>
+__global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
+    hyena_spectrum_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows,
+                      const c32 *__restrict__ tw) {
+    constexpr int T = MC / E;
+    constexpr int RPC = rows_per_cta(MC, E);
+    extern __shared__ float smem[];
+    const int lrow = threadIdx.x / T;
+    const int t = threadIdx.x - lrow * T;
+    const int64_t o = (int64_t)blockIdx.x * RPC + lrow;
+    const bool active = o < nrows;
+    float *sre = smem + lrow * 2 * MC;
+    float *sim = sre + MC;
+    c32 v[E];
+    const float *hrow = h + (active ? o : 0) * h_stride;
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        const int64_t pos = 2 * (int64_t)(t + q * T);
+        v[q] = mk(active && pos < L ? hrow[pos] : 0.f, active && pos + 1 < L ? hrow[pos + 1] : 0.f);
+    }
+#pragma unroll
+    for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+    fft_cta<MC, E, -1, true>(v, sre, sim, t, tw);
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        sre[t + q * T] = v[q].x;
+        sim[t + q * T] = v[q].y;
+    }
+    __syncthreads();
+    c32 *Hrow = Hout + (active ? o : 0) * (MC + 1);
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int k = t + q * T;
+        const int km = (MC - k) & (MC - 1);
+        const c32 Zk = v[q];
+        const c32 Zm = mk(sre[km], sim[km]);
+        const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
+        const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
+        const c32 wO = mul(ldg_c(tw + k), Ok);
+        if (active) {
+            Hrow[k] = add(Ek, wO);
+            if (k == 0) Hrow[MC] = mk(Ek.x - Ok.x, 0.f);  // Nyquist bin: E_0 - O_0, real
+        }
+    }
+}
+
+}  // namespace hyena

@@ -1,0 +1,27 @@
+// Plan object behind the opaque hyena_plan_t handle.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hyena.h"
+
+#define HYENA_MAX_L_1D 131072    // longest 1D sequence (M = 262144)
+#define HYENA_MAX_M_CTA 32768    // longest padded length the single-CTA path runs
+
+struct hyena_plan_s {
+    int ndim = 1;
+    int64_t D = 0;               // channels
+    int order = 0;
+    hyena_dtype_t dtype = HYENA_F32;
+    int path = HYENA_PATH_CTA;
+    int device = 0;
+    // 1D geometry
+    int64_t L = 0;               // sequence length
+    int64_t M = 0;               // padded real FFT length, next_pow2(2L) (at least 32)
+    int64_t MC = 0;              // M / 2: length of the packed complex FFT
+    // 2D geometry
+    int64_t Hh = 0, Ww = 0;      // grid extents (the transform is 2H x 2W)
+    int64_t spectrum_elems = 0;  // complex bins per (order, channel)
+    // device tables (owned)
+    float2 *tw = nullptr;        // W_M^m, m in [0, M)
+};

@@ -1,0 +1,87 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the C ABI
+and the fp64 oracle on the same seeded inputs, then compare with the stated
+tolerances.
+
+Tolerances (from the operator's accuracy target):
+  fp32 I/O: relative L2 error <= 1e-5, and per element
+            |y - y_ref| <= 1e-4 * S_row,
+            S_row = |v_row|_inf * prod_n (|h^n_d|_1 + |Dskip^n_d|) * |x^n_row|_inf
+            (the a-priori bound on |y| for that row);
+  bf16 I/O: relative L2 error <= 2e-2 (fp32 accumulation, bf16 output rounding).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from long_convolution_sequence_hyena_b200.workloads import Workload, make_inputs
+
+REL_L2 = {"f32": 1e-5, "bf16": 2e-2}
+MAXABS_FACTOR = 1e-4
+
+
+def explicit_case(B, D, L, N, dtype="f32", seed=0, alpha=(1e-3, 1e-1)):
+    return Workload("case_b%d_d%d_l%d_n%d_%s" % (B, D, L, N, dtype), 1, B, D, (L,), N, dtype, "explicit",
+                    alpha_lo=alpha[0], alpha_hi=alpha[1], seed=seed)
+
+
+def to_gpu(inp):
+    g = {"v": inp["v"].cuda(), "gates": [x.cuda() for x in inp["gates"]], "dskip": inp["dskip"].cuda()}
+    if "h" in inp:
+        g["h"] = inp["h"].cuda()
+    if "implicit" in inp:
+        g["implicit"] = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp["implicit"].items()}
+    return g
+
+
+def oracle_filters_1d(w: Workload, inp):
+    """fp64 filters [N, D, L] the oracle uses: the given taps, or the implicit network in fp64."""
+    if "h" in inp:
+        return inp["h"].double().numpy()
+    p = inp["implicit"]
+    return oracle.implicit_filter_1d(w.shape[0], w.order, w.D, p["W1"].double().numpy(), p["b1"].double().numpy(),
+                                     p["W2"].double().numpy(), p["b2"].double().numpy(), p["W3"].double().numpy(),
+                                     p["b3"].double().numpy(), p["alpha"].double().numpy(), p["num_freqs"],
+                                     p["omega0"], p["omega_hidden"])
+
+
+def oracle_1d(w: Workload, inp, h64, rows=None):
+    """Oracle output for the selected flat rows (b * D + d), fp64 [len(rows), L]."""
+    N, B, D, L = w.order, w.B, w.D, w.shape[0]
+    R = B * D
+    rows = np.arange(R) if rows is None else np.asarray(rows)
+    v = inp["v"].double().reshape(R, L).numpy()[rows]
+    gates = inp["gates"].double().reshape(N, R, L).numpy()[:, rows]
+    return oracle.hyena_1d(v, gates, h64, inp["dskip"].double().numpy(), fidx=rows % D)
+
+
+def row_bound(w: Workload, inp, h64, rows):
+    """S_row for each selected row (see module docstring)."""
+    N, B, D, L = w.order, w.B, w.D, w.shape[0]
+    R = B * D
+    v = inp["v"].double().reshape(R, L).numpy()[rows]
+    gates = inp["gates"].double().reshape(N, R, L).numpy()[:, rows]
+    dsk = inp["dskip"].double().numpy()
+    d = rows % D
+    s = np.abs(v).max(axis=1)
+    for n in range(N):
+        s = s * (np.abs(h64[n, d]).sum(axis=1) + np.abs(dsk[n, d])) * np.abs(gates[n]).max(axis=1)
+    return s
+
+
+def compare(w: Workload, inp, h64, y_gpu, rows=None, context=""):
+    """Check the GPU output (torch tensor [B, D, L]) on the given rows against the oracle."""
+    N, B, D, L = w.order, w.B, w.D, w.shape[0]
+    R = B * D
+    rows = np.arange(R) if rows is None else np.asarray(rows)
+    ref = oracle_1d(w, inp, h64, rows)
+    got = y_gpu.detach().double().cpu().reshape(R, L).numpy()[rows]
+    assert np.all(np.isfinite(got)), context + ": non-finite output"
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err <= REL_L2[w.dtype], "%s: relative L2 error %.3e > %.1e" % (context, err, REL_L2[w.dtype])
+    if w.dtype == "f32":
+        bound = MAXABS_FACTOR * row_bound(w, inp, h64, rows)
+        worst = (np.abs(got - ref) / np.maximum(bound, 1e-300)[:, None]).max()
+        assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
+    return err

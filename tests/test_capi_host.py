@@ -1,0 +1,65 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from long_convolution_sequence_hyena_b200 import build
+    build.build()
+    from long_convolution_sequence_hyena_b200 import capi as c
+    return c
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"HYENA_API\s+[\w\s\*]+?\b(hyena_\w+)\s*\(", src)
+    return names
+
+
+def test_every_declared_symbol_is_exported(capi):
+    declared = _declared_symbols()
+    assert set(capi.EXPORTED) <= set(declared) and len(declared) >= len(capi.EXPORTED)
+    lib = ctypes.CDLL(capi.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(capi):
+    for code in range(7):
+        assert capi.hyena_status_string(code) not in ("", "unknown status")
+    assert capi.hyena_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((1, [256], 0, 2, 1, 1), "HYENA_ERR_INVALID_ARG"),        # no channels
+    ((1, [256], 4, 0, 1, 1), "HYENA_ERR_INVALID_ARG"),        # order 0
+    ((1, [256], 4, 9, 1, 1), "HYENA_ERR_INVALID_ARG"),        # order above HYENA_MAX_ORDER
+    ((1, [0], 4, 2, 1, 1), "HYENA_ERR_INVALID_ARG"),          # empty sequence
+    ((1, [256], 4, 2, 7, 1), "HYENA_ERR_INVALID_ARG"),        # bad dtype
+    ((3, [4, 4, 4], 4, 1, 1, 0), "HYENA_ERR_INVALID_ARG"),    # 3D
+    ((1, [256], 4, 2, 1, 0), "HYENA_ERR_UNSUPPORTED"),        # non-causal 1D
+    ((2, [64, 64], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # causal 2D
+    ((1, [262145], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # longer than the longest path
+])
+def test_plan_create_rejects(capi, args, expect):
+    st, h = capi.hyena_plan_create(*args)
+    assert capi.STATUS_NAMES[st] == expect and h is None
+
+
+def test_null_plan_rejected(capi):
+    assert capi.hyena_plan_destroy(None) == capi.HYENA_OK
+    assert capi.hyena_plan_info(None)[0] == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_workspace_bytes(None, 4) == 0
+    assert capi.hyena_forward(None, 1, 16, [16], 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_filter_spectrum(None, 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_implicit_filter(None, None, 16) == capi.HYENA_ERR_INVALID_ARG
