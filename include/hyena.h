@@ -152,7 +152,7 @@ HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h
 /*
  * The fused forward pass: all N orders in one launch per row, each row read
  * once from and written once to device memory.
- *   batch      B >= 0 (B = 0 launches nothing)
+ *   batch      B >= 0 (B = 0 launches nothing; the pointers are then not read)
  *   v          [B, D, L] or [B, C, H, W], io dtype
  *   gates      HOST array of N device pointers x^1..x^N, each shaped like v
  *   H          spectra from hyena_filter_spectrum

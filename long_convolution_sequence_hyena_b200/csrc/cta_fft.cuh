@@ -1,9 +1,21 @@
-// CTA-level complex FFT of length MC over registers + a shared-memory exchange
-// buffer, and the real-input packing used by the 1D kernels.
+// Block-level complex FFT of length LEN over registers + a shared-memory
+// exchange buffer, used by every kernel of the library.
 //
-// Real-input packing (standard "two reals in one complex" identity): a real
-// row x of length M = 2*MC is carried as z[n] = x[2n] + i x[2n+1], n < MC.
-// With Z = DFT_MC(z):
+// Two shared-memory layouts:
+//  * NSEQ == 0: one sequence per buffer, contiguous; the Stockham write
+//    pattern is made bank-conflict-free by swz<NS>() (see fft_regs.cuh).
+//  * NSEQ  > 0: NSEQ sequences interleaved, element i of sequence s at
+//    i * NSEQ + (s ^ (i & (NSEQ - 1))). Warps span the sequence index, and
+//    the XOR keeps both "same i, all s" and "same s, consecutive i" accesses
+//    on distinct banks (NSEQ = 32).
+//
+// Twiddles come from one table of W_TWM^m = exp(-2 pi i m / TWM), m < TWM,
+// with TWM a multiple of LEN.
+//
+// Real-input packing used by the 1D kernels (the standard identity that
+// carries a real sequence as a complex one of half the length): a real row x
+// of length M = 2*MC is carried as z[n] = x[2n] + i x[2n+1], n < MC. With
+// Z = DFT_MC(z):
 //   E[k] = (Z[k] + conj Z[MC-k]) / 2,  O[k] = (Z[k] - conj Z[MC-k]) / (2i)
 //   X[k] = E[k] + W_M^k O[k],  X[MC-k] = conj(E[k] - W_M^k O[k])          (X = DFT_M(x))
 // and back, for a spectrum Y of a real row y:
@@ -14,23 +26,29 @@
 
 namespace hyena {
 
-// One Stockham pass p of a length-MC FFT (see fft_regs.cuh for the layout).
-// tw: W_M^m = exp(-2 pi i m / M), m in [0, M), M = 2*MC (forward sign).
-template <int MC, int E, int DIR, bool HALF_IN, int p>
+template <int NS, int NSEQ>
+__device__ __forceinline__ int saddr(int i, int seq) {
+    if constexpr (NSEQ == 0) return swz<NS>(i);
+    else return i * NSEQ + (seq ^ (i & (NSEQ - 1)));
+}
+
+// One Stockham pass p of a length-LEN FFT (register layout in fft_regs.cuh).
+template <int LEN, int E, int DIR, bool HALF_IN, int p, int TWM, int NSEQ>
 __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim, int t,
-                                         const c32 *__restrict__ tw) {
-    constexpr int T = MC / E;
-    constexpr int P = num_passes(MC);
-    constexpr int R = pass_radix(MC, p);
-    constexpr int NS = pass_stride(MC, p);
+                                         int seq, const c32 *__restrict__ tw) {
+    constexpr int T = LEN / E;
+    constexpr int P = num_passes(LEN);
+    constexpr int R = pass_radix(LEN, p);
+    constexpr int NS = pass_stride(LEN, p);
     constexpr int S = E / R;
     constexpr bool LAST = (p == P - 1);
+    static_assert(TWM % LEN == 0, "twiddle table must cover the transform");
     if constexpr (p > 0) {
-        constexpr int NSP = pass_stride(MC, p - 1);
+        constexpr int NSP = pass_stride(LEN, p - 1);
         __syncthreads();  // writes of pass p-1 visible
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int i = swz<NSP>(t + q * T);
+            const int i = saddr<NSP, NSEQ>(t + q * T, seq);
             v[q] = mk(sre[i], sim[i]);
         }
         __syncthreads();  // every read done before pass p writes
@@ -41,7 +59,7 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
         const int k = j & (NS - 1);
         (void)k;
         if constexpr (NS > 1) {
-            const float2 wf = __ldg(reinterpret_cast<const float2 *>(tw) + (size_t)k * (2 * MC / (NS * R)));
+            const float2 wf = __ldg(reinterpret_cast<const float2 *>(tw) + (size_t)k * (TWM / (NS * R)));
             twiddle_powers<R, S, s>(v, DIR > 0 ? mk(wf.x, -wf.y) : mk(wf.x, wf.y));
         }
         dftR<R, DIR, HALF_IN && p == 0, S, s>(v);
@@ -49,22 +67,24 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
             const int base = (j / NS) * NS * R + k;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const int i = swz<NS>(base + r * NS);
+                const int i = saddr<NS, NSEQ>(base + r * NS, seq);
                 sre[i] = v[s + r * S].x;
                 sim[i] = v[s + r * S].y;
             }
         }
     });
-    if constexpr (!LAST) fft_pass<MC, E, DIR, false, p + 1>(v, sre, sim, t, tw);
+    if constexpr (!LAST) fft_pass<LEN, E, DIR, false, p + 1, TWM, NSEQ>(v, sre, sim, t, seq, tw);
 }
 
-// Full length-MC FFT in place on v (natural order in and out).
+// Full length-LEN FFT in place on v (natural order in and out).
 // HALF_IN: registers q >= E/2 hold zeros on entry (zero-padded input).
-// On return every smem read of this FFT is complete in all threads of the CTA
-// (the last exchange ends with a barrier), unless the FFT has a single pass.
-template <int MC, int E, int DIR, bool HALF_IN>
-__device__ __forceinline__ void fft_cta(c32 (&v)[E], float *sre, float *sim, int t, const c32 *__restrict__ tw) {
-    fft_pass<MC, E, DIR, HALF_IN, 0>(v, sre, sim, t, tw);
+// When the FFT has more than one pass, every shared-memory read it makes is
+// complete in all threads of the block on return (the last exchange ends with
+// a barrier).
+template <int LEN, int E, int DIR, bool HALF_IN, int TWM = 2 * LEN, int NSEQ = 0>
+__device__ __forceinline__ void fft_cta(c32 (&v)[E], float *sre, float *sim, int t, const c32 *__restrict__ tw,
+                                        int seq = 0) {
+    fft_pass<LEN, E, DIR, HALF_IN, 0, TWM, NSEQ>(v, sre, sim, t, seq, tw);
 }
 
 }  // namespace hyena

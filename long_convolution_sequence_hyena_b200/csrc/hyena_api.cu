@@ -279,7 +279,9 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
                              const float *Dskip, void *y, void *workspace, size_t ws_bytes, void *stream) {
     (void)workspace;
     (void)ws_bytes;
-    if (!plan || batch < 0 || !v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
+    if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
+    if (batch == 0) return HYENA_OK;  // nothing to read or write; pointers may be NULL
+    if (!v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
     for (int n = 0; n < plan->order; ++n)
         if (!gates[n]) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(v) || !aligned16(H) || !aligned16(y) || (Dskip && !aligned4(Dskip))) return HYENA_ERR_ALIGNMENT;
@@ -287,7 +289,6 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
         if (!aligned16(gates[n])) return HYENA_ERR_ALIGNMENT;
     hyena_status_t s = check_device(plan);
     if (s != HYENA_OK) return s;
-    if (batch == 0) return HYENA_OK;
 
     Fwd1dArgs a;
     std::memset(&a, 0, sizeof(a));
