@@ -98,7 +98,7 @@ typedef struct {
  * Create a plan.
  *   ndim      1 (sequence) or 2 (grid)
  *   shape     host array of ndim sizes: {L} or {H, W}; each >= 1.
- *             1D: L <= 131072. 2D: H, W powers of two with 2H, 2W <= 1024.
+ *             1D: L <= 131072. 2D: H == W, one of 32, 64, 128, 256.
  *   channels  D (1D) or C (2D), >= 1
  *   order     N, 1..HYENA_MAX_ORDER
  *   io_dtype  storage type of v, the gates and y

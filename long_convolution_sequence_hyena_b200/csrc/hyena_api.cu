@@ -11,6 +11,8 @@
 
 #include "hyena.h"
 #include "kernels_1d.cuh"
+#include "kernels_1d_cluster.cuh"
+#include "kernels_2d.cuh"
 #include "kernels_implicit.cuh"
 #include "plan.h"
 
@@ -112,6 +114,92 @@ cudaError_t launch_implicit(const ImplicitArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------- cluster paths
+using G1_32K = ClusterGeom<32768, 4, 128, 16>;    // 1D, 32768 < M <= 65536
+using G1_64K = ClusterGeom<65536, 8, 256, 16>;    // 1D, M = 131072
+using G1_128K = ClusterGeom<131072, 8, 512, 32>;  // 1D, M = 262144
+using G2_32 = ClusterGeom<2048, 1, 64, 16>;       // 2D, 32 x 32 grid (64 x 64 padded)
+using G2_64 = ClusterGeom<8192, 2, 128, 16>;      // 2D, 64 x 64
+using G2_128 = ClusterGeom<32768, 4, 256, 16>;    // 2D, 128 x 128
+using G2_256 = ClusterGeom<131072, 8, 512, 32>;   // 2D, 256 x 256
+
+template <typename G, typename Kern, typename... Args>
+cudaError_t launch_cluster(Kern kern, int64_t units, cudaStream_t st, Args... args) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * G::C), 1, 1);
+    cfg.blockDim = dim3(G::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = G::C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename G>
+cudaError_t launch_fwd_1d_cluster_g(const Fwd1dArgs &a, hyena_dtype_t dt, bool even, cudaStream_t st) {
+    if (dt == HYENA_F32)
+        return even ? launch_cluster<G>(hyena_fwd_1d_cluster<G, float, true>, a.rows, st, a)
+                    : launch_cluster<G>(hyena_fwd_1d_cluster<G, float, false>, a.rows, st, a);
+    return even ? launch_cluster<G>(hyena_fwd_1d_cluster<G, __nv_bfloat16, true>, a.rows, st, a)
+                : launch_cluster<G>(hyena_fwd_1d_cluster<G, __nv_bfloat16, false>, a.rows, st, a);
+}
+
+cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
+    switch (MC) {
+        case 32768: return launch_fwd_1d_cluster_g<G1_32K>(a, dt, even, st);
+        case 65536: return launch_fwd_1d_cluster_g<G1_64K>(a, dt, even, st);
+        case 131072: return launch_fwd_1d_cluster_g<G1_128K>(a, dt, even, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
+                                   const c32 *tw, cudaStream_t st) {
+    switch (MC) {
+        case 32768: return launch_cluster<G1_32K>(hyena_spectrum_1d_cluster<G1_32K>, nrows, st, h, h_stride, L, Hout, tw);
+        case 65536: return launch_cluster<G1_64K>(hyena_spectrum_1d_cluster<G1_64K>, nrows, st, h, h_stride, L, Hout, tw);
+        case 131072:
+            return launch_cluster<G1_128K>(hyena_spectrum_1d_cluster<G1_128K>, nrows, st, h, h_stride, L, Hout, tw);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename G>
+cudaError_t launch_fwd_2d_g(const Fwd2dArgs &a, hyena_dtype_t dt, cudaStream_t st) {
+    if (dt == HYENA_F32) return launch_cluster<G>(hyena_fwd_2d_cluster<G, float>, a.planes, st, a);
+    return launch_cluster<G>(hyena_fwd_2d_cluster<G, __nv_bfloat16>, a.planes, st, a);
+}
+
+cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st) {
+    switch (W) {
+        case 32: return launch_fwd_2d_g<G2_32>(a, dt, st);
+        case 64: return launch_fwd_2d_g<G2_64>(a, dt, st);
+        case 128: return launch_fwd_2d_g<G2_128>(a, dt, st);
+        case 256: return launch_fwd_2d_g<G2_256>(a, dt, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W, const c32 *tw,
+                           cudaStream_t st) {
+    switch (W) {
+        case 32: return launch_cluster<G2_32>(hyena_spectrum_2d_cluster<G2_32>, n, st, K, rs, cs, Kout, tw);
+        case 64: return launch_cluster<G2_64>(hyena_spectrum_2d_cluster<G2_64>, n, st, K, rs, cs, Kout, tw);
+        case 128: return launch_cluster<G2_128>(hyena_spectrum_2d_cluster<G2_128>, n, st, K, rs, cs, Kout, tw);
+        case 256: return launch_cluster<G2_256>(hyena_spectrum_2d_cluster<G2_256>, n, st, K, rs, cs, Kout, tw);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 // W_M^m = exp(-2 pi i m / M), m in [0, M), computed in double and rounded once.
 std::vector<float2> twiddle_table(int64_t M) {
     std::vector<float2> t((size_t)M);
@@ -193,14 +281,20 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         if (p.M < 32) p.M = 32;  // smallest FFT the kernels run (extra zero padding is exact)
         p.MC = p.M / 2;
         p.path = p.M <= HYENA_MAX_M_CTA ? HYENA_PATH_CTA : HYENA_PATH_CLUSTER;
-        if (p.path == HYENA_PATH_CLUSTER) return HYENA_ERR_UNSUPPORTED;
         p.spectrum_elems = p.MC + 1;
+        p.tw_len = p.M;
     } else {
-        return HYENA_ERR_UNSUPPORTED;
+        p.Hh = shape[0];
+        p.Ww = shape[1];
+        const bool ok = p.Hh == p.Ww && (p.Ww == 32 || p.Ww == 64 || p.Ww == 128 || p.Ww == 256);
+        if (!ok) return HYENA_ERR_UNSUPPORTED;
+        p.path = HYENA_PATH_2D;
+        p.spectrum_elems = 2 * p.Hh * (p.Ww + 1);
+        p.tw_len = 2 * p.Ww;
     }
     if (cudaGetDevice(&p.device) != cudaSuccess) return HYENA_ERR_CUDA;
 
-    std::vector<float2> tw = twiddle_table(p.M);
+    std::vector<float2> tw = twiddle_table(p.tw_len);
     if (cudaMalloc(&p.tw, sizeof(float2) * tw.size()) != cudaSuccess) {
         cudaGetLastError();
         return HYENA_ERR_NOMEM;
@@ -261,17 +355,32 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t nrows = (int64_t)plan->order * plan->D;
     c32 *Hc = reinterpret_cast<c32 *>(H_out);
+    const c32 *tw = reinterpret_cast<const c32 *>(plan->tw);
     const float *src = h;
-    int64_t src_stride = plan->L;
-    if (!h) {
-        // generate the taps inside each row's own output slot, then transform in place
-        src_stride = 2 * (plan->MC + 1);
-        ImplicitArgs a = implicit_args(plan, params, reinterpret_cast<float *>(H_out), src_stride, 0);
-        if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
-        src = reinterpret_cast<const float *>(H_out);
+    cudaError_t e;
+    if (plan->ndim == 1) {
+        int64_t src_stride = plan->L;
+        if (!h) {
+            // generate the taps inside each row's own output slot, then transform in place
+            src_stride = 2 * (plan->MC + 1);
+            ImplicitArgs a = implicit_args(plan, params, reinterpret_cast<float *>(H_out), src_stride, 0);
+            if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
+            src = reinterpret_cast<const float *>(H_out);
+        }
+        e = plan->path == HYENA_PATH_CTA ? launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st)
+                                         : launch_spec_1d_cluster(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st);
+    } else {
+        int64_t rs = 2 * plan->Ww, cs = 4 * plan->Hh * plan->Ww;
+        if (!h) {
+            // kernel rows written at the spectrum's row pitch inside each channel's slot
+            rs = 2 * (plan->Ww + 1);
+            cs = 2 * plan->Hh * rs;
+            ImplicitArgs a = implicit_args(plan, params, reinterpret_cast<float *>(H_out), cs, rs);
+            if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
+            src = reinterpret_cast<const float *>(H_out);
+        }
+        e = launch_spec_2d(src, rs, cs, Hc, nrows, plan->Ww, tw, st);
     }
-    cudaError_t e = launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC,
-                                   reinterpret_cast<const c32 *>(plan->tw), st);
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
@@ -290,6 +399,21 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     hyena_status_t s = check_device(plan);
     if (s != HYENA_OK) return s;
 
+    if (plan->ndim == 2) {
+        Fwd2dArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.v = v;
+        for (int n = 0; n < plan->order; ++n) a.gates[n] = gates[n];
+        a.K = reinterpret_cast<const c32 *>(H);
+        a.dskip = Dskip;
+        a.y = y;
+        a.tw = reinterpret_cast<const c32 *>(plan->tw);
+        a.planes = batch * plan->D;
+        a.C = plan->D;
+        a.B = batch;
+        a.order = plan->order;
+        return launch_fwd_2d(a, plan->Ww, plan->dtype, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+    }
     Fwd1dArgs a;
     std::memset(&a, 0, sizeof(a));
     a.v = v;
@@ -303,7 +427,10 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     a.D = plan->D;
     a.B = batch;
     a.order = plan->order;
-    cudaError_t e = launch_fwd_1d(a, plan->MC, plan->dtype, (plan->L % 2) == 0, (cudaStream_t)stream);
+    const bool even = (plan->L % 2) == 0;
+    cudaError_t e = plan->path == HYENA_PATH_CTA
+                        ? launch_fwd_1d(a, plan->MC, plan->dtype, even, (cudaStream_t)stream)
+                        : launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 

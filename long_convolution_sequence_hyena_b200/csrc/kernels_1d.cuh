@@ -66,6 +66,19 @@ __device__ __forceinline__ c32 load_pair(const IO *__restrict__ row, int64_t pos
     }
 }
 
+// Raw (still packed) pair for prefetching: one register per pair in bf16.
+template <typename IO, bool EVEN>
+__device__ __forceinline__ typename io<IO>::pair_t load_pair_raw(const IO *__restrict__ row, int64_t pos, int64_t L) {
+    using P = typename io<IO>::pair_t;
+    if constexpr (EVEN) {
+        if (pos < L) return __ldg(reinterpret_cast<const P *>(row + pos));
+        return io<IO>::zero();
+    } else {
+        const c32 c = load_pair<IO, false>(row, pos, L);
+        return io<IO>::pack(c);
+    }
+}
+
 template <typename IO, bool EVEN>
 __device__ __forceinline__ void store_pair(IO *__restrict__ row, int64_t pos, int64_t L, c32 val) {
     if constexpr (EVEN) {
@@ -155,10 +168,10 @@ __global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
 
     for (int n = 0; n < a.order; ++n) {
         const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + row * L;
-        c32 g[E / 2];
+        typename io<IO>::pair_t g[E / 2];
 #pragma unroll
         for (int q = 0; q < E / 2; ++q)
-            g[q] = active ? load_pair<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L) : mk(0.f, 0.f);
+            g[q] = active ? load_pair_raw<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L) : io<IO>::zero();
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
 
         fft_cta<MC, E, -1, true>(v, sre, sim, t, a.tw);
@@ -169,7 +182,8 @@ __global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
             const int64_t pos = 2 * (int64_t)(t + q * T);
-            v[q] = mk(pos < L ? g[q].x * v[q].x : 0.f, pos + 1 < L ? g[q].y * v[q].y : 0.f);
+            const c32 gq = io<IO>::unpack(g[q]);
+            v[q] = mk(pos < L ? gq.x * v[q].x : 0.f, pos + 1 < L ? gq.y * v[q].y : 0.f);
         }
 #pragma unroll
         for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);

@@ -1,0 +1,167 @@
+// 2D (HyenaND-style) fused forward and kernel spectrum: one thread-block
+// cluster per (batch, channel) plane.
+//
+// A real plane v[y][x] of H x W is zero-padded to 2H x 2W and packed along x,
+// z[y][x'] = v[y][2x'] + i v[y][2x'+1], giving a complex [M1 = 2H][M2 = W]
+// array. Its 2D DFT is the cluster four-step transform without the
+// inter-stage twiddle (columns = y, rows = x'). Only y < H and x' < W/2 carry
+// data, so both stages start from half-zero input and the inverse keeps only
+// that quarter. The real-packing identity along x unpacks the spectrum with
+// the 2D mirror bin Z[-ky][-kx'] and the twiddle W_{2W}^{kx'}.
+//
+// Convolution ("How HyenaND works", "2. The convolution theorem (FFT)"): the
+// kernel on offsets o in [-H, H) x [-W, W) is placed cyclically (offset o at
+// index o mod 2H, o mod 2W), so the cyclic product of the padded plane with it
+// is the linear, non-causal convolution, read out on [0, H) x [0, W).
+#pragma once
+#include "kernels_1d_cluster.cuh"
+
+namespace hyena {
+
+struct Fwd2dArgs {
+    const void *v;
+    const void *gates[HYENA_MAX_ORDER];
+    const c32 *K;         // [N, C, 2H, W + 1]
+    const float *dskip;   // [N, C] or nullptr
+    void *y;
+    const c32 *tw;        // W_TWM^m
+    int64_t planes;       // B * C
+    int64_t C;
+    int64_t B;
+    int order;
+};
+
+// Fused order-N 2D forward (planes visited c-major, b-minor).
+template <typename G, typename IO>
+__global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2dArgs a) {
+    using Ctx = ClusterCtx<G, false>;
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
+    constexpr int Hh = M1 / 2, Ww = M2;                 // plane extents
+    constexpr int TWM = Ctx::TWM;
+    extern __shared__ float smem[];
+    Ctx cx(smem);
+    const int64_t ord = (int64_t)blockIdx.x / G::C;
+    const int64_t c = ord / a.B;
+    const int64_t b = ord - c * a.B;
+    const int64_t plane = b * a.C + c;
+    const bool xin = 2 * cx.n2 < Ww;                    // this column carries data
+
+    // column-layout register q holds (y = t1 + q T1, x' = n2)
+    auto pos_of = [&](int q) -> int64_t { return (int64_t)(cx.t1 + q * G::T1) * Ww + 2 * cx.n2; };
+
+    c32 v[E];
+    {
+        const IO *vp = reinterpret_cast<const IO *>(a.v) + plane * Hh * Ww;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) v[q] = xin ? load_pair<IO, true>(vp, pos_of(q), (int64_t)Hh * Ww) : mk(0.f, 0.f);
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+    }
+
+    for (int n = 0; n < a.order; ++n) {
+        const IO *gp = reinterpret_cast<const IO *>(a.gates[n]) + plane * Hh * Ww;
+        typename io<IO>::pair_t g[E / 2];
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q)
+            g[q] = xin ? load_pair_raw<IO, true>(gp, pos_of(q), (int64_t)Hh * Ww) : io<IO>::zero();
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.C + c) : 0.f;
+        const c32 *Kp = a.K + ((int64_t)n * a.C + c) * (M1 * (M2 + 1));
+
+        cx.template forward<true, true>(v, a.tw);
+        cx.publish(v);
+        constexpr float s = 0.5f / (float)(M1 * M2);
+        const int ky = cx.k1;
+        const int kym = (M1 - ky) & (M1 - 1);
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const int kx = cx.t2 + q * G::T2;
+            const int kxm = (M2 - kx) & (M2 - 1);
+            const c32 Zm = cx.bin(kym + M1 * kxm);
+            const c32 Zk = v[q];
+            const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
+            const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
+            const c32 w = ldg_c(a.tw + kx * (TWM / (2 * M2)));
+            const c32 wO = mul(w, Ok);
+            const c32 Xk = add(Ek, wO);                  // bin (ky, kx)
+            const c32 Xm = conj(sub(Ek, wO));            // bin (-ky, M2 - kx)
+            c32 Hk = ldg_c(Kp + (int64_t)ky * (M2 + 1) + kx);
+            c32 Hm = ldg_c(Kp + (int64_t)kym * (M2 + 1) + (M2 - kx));
+            Hk.x += dsk;
+            Hm.x += dsk;
+            const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
+            const c32 Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
+            const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
+            const c32 Yo = mul(Yd, conj(w));
+            v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+            if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
+        }
+        cx.cluster.sync();
+        cx.inverse(v, a.tw);
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const c32 gq = io<IO>::unpack(g[q]);
+            v[q] = xin ? mk(gq.x * v[q].x, gq.y * v[q].y) : mk(0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+    }
+
+    if (xin) {
+        IO *yp = reinterpret_cast<IO *>(a.y) + plane * Hh * Ww;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) store_pair<IO, true>(yp, pos_of(q), (int64_t)Hh * Ww, v[q]);
+    }
+}
+
+// 2D kernel spectra. Kernel (n, c) starts at K + o * cs (o = n * C + c); row iy
+// of its offset grid (offset oy = iy - H) starts at + iy * rs and holds 2W
+// floats (ox = ix - W). In place (K == Kout, rs = 2W + 2, cs = 2H (2W + 2)) is
+// allowed: every read precedes the first cluster barrier.
+template <typename G>
+__global__ void __launch_bounds__(G::THREADS, 1)
+    hyena_spectrum_2d_cluster(const float *K, int64_t rs, int64_t cs, c32 *Kout, const c32 *__restrict__ tw) {
+    using Ctx = ClusterCtx<G, false>;
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
+    constexpr int Hh = M1 / 2, Ww = M2;
+    constexpr int TWM = Ctx::TWM;
+    extern __shared__ float smem[];
+    Ctx cx(smem);
+    const int64_t o = (int64_t)blockIdx.x / G::C;
+    const float *Kp = K + o * cs;
+    c32 v[E];
+    const int ix = (2 * cx.n2 + Ww) & (2 * Ww - 1);    // cyclic column 2 n2 -> offset-grid column
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int iy = (cx.t1 + q * G::T1 + Hh) & (M1 - 1);
+        const float *rowp = Kp + iy * rs;
+        v[q] = mk(rowp[ix], rowp[ix + 1]);
+    }
+    cx.cluster.sync();                                  // every read done before anything is written
+    cx.template forward<false, false>(v, tw);
+    cx.publish(v);
+    const int ky = cx.k1;
+    const int kym = (M1 - ky) & (M1 - 1);
+    c32 outv[E];
+    c32 nyq = mk(0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int kx = cx.t2 + q * G::T2;
+        const c32 Zm = cx.bin(kym + M1 * ((M2 - kx) & (M2 - 1)));
+        const c32 Zk = v[q];
+        const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
+        const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
+        const c32 wO = mul(ldg_c(tw + kx * (TWM / (2 * M2))), Ok);
+        outv[q] = add(Ek, wO);
+        if (kx == 0) nyq = conj(sub(Ek, wO));            // bin (-ky, M2)
+    }
+    cx.cluster.sync();
+    c32 *Ko = Kout + o * (M1 * (M2 + 1));
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int kx = cx.t2 + q * G::T2;
+        Ko[(int64_t)ky * (M2 + 1) + kx] = outv[q];
+        if (kx == 0) Ko[(int64_t)kym * (M2 + 1) + M2] = nyq;
+    }
+}
+
+}  // namespace hyena

@@ -23,5 +23,6 @@ struct hyena_plan_s {
     int64_t Hh = 0, Ww = 0;      // grid extents (the transform is 2H x 2W)
     int64_t spectrum_elems = 0;  // complex bins per (order, channel)
     // device tables (owned)
-    float2 *tw = nullptr;        // W_M^m, m in [0, M)
+    int64_t tw_len = 0;          // 1D: M; 2D: 2W
+    float2 *tw = nullptr;        // W_tw_len^m, m in [0, tw_len)
 };

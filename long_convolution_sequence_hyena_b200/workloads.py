@@ -108,7 +108,8 @@ def make_inputs(w: Workload, seed=None) -> dict:
       v      [B, D, *shape]      activation dtype
       gates  [N, B, D, *shape]   activation dtype
       dskip  [N, D]              float32
-      h      [N, D, L]           float32 (explicit filters only)
+      h      [N, D, L]           float32 (explicit filters only; 2D: [N, C, 2H, 2W] on
+                                 the offset grid, N(0,1) under exp(-|p|^2 / (2 sigma^2)))
       implicit: dict of float32 weights W1 b1 W2 b2 W3 b3 and the window
                parameter (alpha [N, D] in 1D, sigma [N, D] in 2D), plus the
                scalars width, num_freqs, omega0, omega_hidden (implicit only)
@@ -120,7 +121,15 @@ def make_inputs(w: Workload, seed=None) -> dict:
     out["v"] = torch.randn((B, D) + w.shape, generator=g, dtype=torch.float64).to(adt)
     out["gates"] = torch.randn((N, B, D) + w.shape, generator=g, dtype=torch.float64).to(adt)
     out["dskip"] = torch.randn((N, D), generator=g, dtype=torch.float64).to(torch.float32)
-    if w.filt == "explicit":
+    if w.filt == "explicit" and w.ndim == 2:
+        H, W = w.shape
+        oy = torch.arange(-H, H, dtype=torch.float64) / H
+        ox = torch.arange(-W, W, dtype=torch.float64) / W
+        r2 = oy[:, None] ** 2 + ox[None, :] ** 2
+        # explicit 2D kernels on the offset grid: Gaussian taps under a Gaussian envelope
+        out["h"] = (torch.randn((N, D, 2 * H, 2 * W), generator=g, dtype=torch.float64)
+                    * torch.exp(-r2 / (2 * w.sigma ** 2))).to(torch.float32)
+    elif w.filt == "explicit":
         L = w.shape[0]
         alpha = _alphas(w, N * D, g).reshape(N, D, 1)
         t = torch.arange(L, dtype=torch.float64)

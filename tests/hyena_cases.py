@@ -85,3 +85,46 @@ def compare(w: Workload, inp, h64, y_gpu, rows=None, context=""):
         worst = (np.abs(got - ref) / np.maximum(bound, 1e-300)[:, None]).max()
         assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
     return err
+
+
+# ------------------------------------------------------------------------ 2D --
+
+def explicit_case_2d(B, C, Hw, N, dtype="f32", seed=0, sigma=0.5):
+    return Workload("case2d_b%d_c%d_%d_n%d_%s" % (B, C, Hw, N, dtype), 2, B, C, (Hw, Hw), N, dtype, "explicit",
+                    sigma=sigma, seed=seed)
+
+
+def oracle_kernels_2d(w: Workload, inp):
+    """fp64 kernels [N, C, 2H, 2W] on the offset grid."""
+    if "h" in inp:
+        return inp["h"].double().numpy()
+    p = inp["implicit"]
+    H, W = w.shape
+    return oracle.implicit_filter_2d(H, W, w.order, w.D, p["W1"].double().numpy(), p["b1"].double().numpy(),
+                                     p["W2"].double().numpy(), p["b2"].double().numpy(), p["W3"].double().numpy(),
+                                     p["b3"].double().numpy(), p["sigma"].double().numpy(), p["omega0"],
+                                     p["omega_hidden"])
+
+
+def compare_2d(w: Workload, inp, k64, y_gpu, planes=None, context=""):
+    N, B, C = w.order, w.B, w.D
+    H, W = w.shape
+    P = B * C
+    planes = np.arange(P) if planes is None else np.asarray(planes)
+    v = inp["v"].double().reshape(P, H, W).numpy()[planes]
+    gates = inp["gates"].double().reshape(N, P, H, W).numpy()[:, planes]
+    dsk = inp["dskip"].double().numpy()
+    ref = oracle.hyena_2d(v, gates, k64, dsk, fidx=planes % C)
+    got = y_gpu.detach().double().cpu().reshape(P, H, W).numpy()[planes]
+    assert np.all(np.isfinite(got)), context + ": non-finite output"
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err <= REL_L2[w.dtype], "%s: relative L2 error %.3e > %.1e" % (context, err, REL_L2[w.dtype])
+    if w.dtype == "f32":
+        c = planes % C
+        bound = np.abs(v).reshape(len(planes), -1).max(axis=1)
+        for n in range(N):
+            bound = bound * (np.abs(k64[n, c]).reshape(len(planes), -1).sum(axis=1) + np.abs(dsk[n, c])) \
+                * np.abs(gates[n]).reshape(len(planes), -1).max(axis=1)
+        worst = (np.abs(got - ref) / (MAXABS_FACTOR * np.maximum(bound, 1e-300))[:, None, None]).max()
+        assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
+    return err
