@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--channels", type=int, default=None,
+                    help="override the workload's channel count (small cases for profiling)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
     return ap.parse_args()
 
 
@@ -294,10 +297,12 @@ def main():
     args = parse()
     from long_convolution_sequence_hyena_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.channels is not None or args.batch is not None:
+        w = w.scaled(B=args.batch, D=args.channels, name=w.name)
     metric = "Hyena op throughput (B·D·L elems/s)"
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    cfg = {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L, "channels": w.D, "order": w.order,
+    cfg = {"workload": w.name, "batch": w.B, "global_batch": w.B * world, "seq_len": w.L, "channels": w.D, "order": w.order,
            "shape": list(w.shape), "parallelism": "independent replicas x%d (no data-path collective)" % world,
            "l2": "flushed between timed steps (512 MiB write)", "filters": w.filt}
 

@@ -47,6 +47,81 @@ __device__ __forceinline__ c32 rot90(c32 a) {
     return DIR > 0 ? c32{-a.y, a.x} : c32{a.y, -a.x};
 }
 
+// W_64^m = exp(-2 pi i m / 64), m = 0..63 (cos and sin of m pi / 32, rounded to
+// float). Indexed with compile-time offsets, they become constant-bank operands.
+__constant__ float2 c_w64[64] = {
+    {1.000000000e+00f, -0.000000000e+00f},
+    {9.951847267e-01f, -9.801714033e-02f},
+    {9.807852804e-01f, -1.950903220e-01f},
+    {9.569403357e-01f, -2.902846773e-01f},
+    {9.238795325e-01f, -3.826834324e-01f},
+    {8.819212643e-01f, -4.713967368e-01f},
+    {8.314696123e-01f, -5.555702330e-01f},
+    {7.730104534e-01f, -6.343932842e-01f},
+    {7.071067812e-01f, -7.071067812e-01f},
+    {6.343932842e-01f, -7.730104534e-01f},
+    {5.555702330e-01f, -8.314696123e-01f},
+    {4.713967368e-01f, -8.819212643e-01f},
+    {3.826834324e-01f, -9.238795325e-01f},
+    {2.902846773e-01f, -9.569403357e-01f},
+    {1.950903220e-01f, -9.807852804e-01f},
+    {9.801714033e-02f, -9.951847267e-01f},
+    {6.123233996e-17f, -1.000000000e+00f},
+    {-9.801714033e-02f, -9.951847267e-01f},
+    {-1.950903220e-01f, -9.807852804e-01f},
+    {-2.902846773e-01f, -9.569403357e-01f},
+    {-3.826834324e-01f, -9.238795325e-01f},
+    {-4.713967368e-01f, -8.819212643e-01f},
+    {-5.555702330e-01f, -8.314696123e-01f},
+    {-6.343932842e-01f, -7.730104534e-01f},
+    {-7.071067812e-01f, -7.071067812e-01f},
+    {-7.730104534e-01f, -6.343932842e-01f},
+    {-8.314696123e-01f, -5.555702330e-01f},
+    {-8.819212643e-01f, -4.713967368e-01f},
+    {-9.238795325e-01f, -3.826834324e-01f},
+    {-9.569403357e-01f, -2.902846773e-01f},
+    {-9.807852804e-01f, -1.950903220e-01f},
+    {-9.951847267e-01f, -9.801714033e-02f},
+    {-1.000000000e+00f, -1.224646799e-16f},
+    {-9.951847267e-01f, 9.801714033e-02f},
+    {-9.807852804e-01f, 1.950903220e-01f},
+    {-9.569403357e-01f, 2.902846773e-01f},
+    {-9.238795325e-01f, 3.826834324e-01f},
+    {-8.819212643e-01f, 4.713967368e-01f},
+    {-8.314696123e-01f, 5.555702330e-01f},
+    {-7.730104534e-01f, 6.343932842e-01f},
+    {-7.071067812e-01f, 7.071067812e-01f},
+    {-6.343932842e-01f, 7.730104534e-01f},
+    {-5.555702330e-01f, 8.314696123e-01f},
+    {-4.713967368e-01f, 8.819212643e-01f},
+    {-3.826834324e-01f, 9.238795325e-01f},
+    {-2.902846773e-01f, 9.569403357e-01f},
+    {-1.950903220e-01f, 9.807852804e-01f},
+    {-9.801714033e-02f, 9.951847267e-01f},
+    {-1.836970199e-16f, 1.000000000e+00f},
+    {9.801714033e-02f, 9.951847267e-01f},
+    {1.950903220e-01f, 9.807852804e-01f},
+    {2.902846773e-01f, 9.569403357e-01f},
+    {3.826834324e-01f, 9.238795325e-01f},
+    {4.713967368e-01f, 8.819212643e-01f},
+    {5.555702330e-01f, 8.314696123e-01f},
+    {6.343932842e-01f, 7.730104534e-01f},
+    {7.071067812e-01f, 7.071067812e-01f},
+    {7.730104534e-01f, 6.343932842e-01f},
+    {8.314696123e-01f, 5.555702330e-01f},
+    {8.819212643e-01f, 4.713967368e-01f},
+    {9.238795325e-01f, 3.826834324e-01f},
+    {9.569403357e-01f, 2.902846773e-01f},
+    {9.807852804e-01f, 1.950903220e-01f},
+    {9.951847267e-01f, 9.801714033e-02f}};
+
+// W_{2E}^q for a compile-time q (E <= 32).
+template <int E>
+__device__ __forceinline__ c32 w2e(int q) {
+    const float2 f = c_w64[q * (32 / E)];
+    return c32{f.x, f.y};
+}
+
 // cos / sin of k*pi/8 for the radix-16 internal twiddles (exact math constants)
 #define HY_C1 0.92387953251128675613f  // cos(pi/8)
 #define HY_S1 0.38268343236508977173f  // sin(pi/8)

@@ -10,10 +10,8 @@
 #include <vector>
 
 #include "hyena.h"
-#include "kernels_1d.cuh"
-#include "kernels_1d_cluster.cuh"
 #include "kernels_2d.cuh"
-#include "kernels_implicit.cuh"
+#include "launch.h"
 #include "plan.h"
 
 using namespace hyena;
@@ -27,177 +25,6 @@ int64_t next_pow2(int64_t v) {
     int64_t p = 1;
     while (p < v) p <<= 1;
     return p;
-}
-
-// ---------------------------------------------------------------- 1D dispatch
-// Elements per thread for each half-length MC (threads per row = MC / E).
-constexpr int e_for(int MC) { return MC >= 16384 ? 32 : 16; }
-
-template <int MC>
-size_t smem_1d() {
-    return (size_t)rows_per_cta(MC, e_for(MC)) * 2 * MC * sizeof(float);
-}
-
-template <int MC, typename IO, bool EVEN>
-cudaError_t launch_fwd_1d_t(const Fwd1dArgs &a, cudaStream_t st) {
-    constexpr int E = e_for(MC);
-    constexpr int RPC = rows_per_cta(MC, E);
-    auto kern = hyena_fwd_1d_cta<MC, E, IO, EVEN>;
-    const size_t sm = smem_1d<MC>();
-    if (sm > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t grid = (a.rows + RPC - 1) / RPC;
-    kern<<<(unsigned)grid, RPC * (MC / E), sm, st>>>(a);
-    return cudaGetLastError();
-}
-
-template <int MC>
-cudaError_t launch_fwd_1d_mc(const Fwd1dArgs &a, hyena_dtype_t dt, bool even, cudaStream_t st) {
-    if (dt == HYENA_F32)
-        return even ? launch_fwd_1d_t<MC, float, true>(a, st) : launch_fwd_1d_t<MC, float, false>(a, st);
-    return even ? launch_fwd_1d_t<MC, __nv_bfloat16, true>(a, st) : launch_fwd_1d_t<MC, __nv_bfloat16, false>(a, st);
-}
-
-template <int MC>
-cudaError_t launch_spec_1d_mc(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, const c32 *tw,
-                              cudaStream_t st) {
-    constexpr int E = e_for(MC);
-    constexpr int RPC = rows_per_cta(MC, E);
-    auto kern = hyena_spectrum_1d<MC, E>;
-    const size_t sm = smem_1d<MC>();
-    if (sm > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t grid = (nrows + RPC - 1) / RPC;
-    kern<<<(unsigned)grid, RPC * (MC / E), sm, st>>>(h, h_stride, L, Hout, nrows, tw);
-    return cudaGetLastError();
-}
-
-#define HY_MC_SWITCH(MCV, CALL)     \
-    switch (MCV) {                  \
-        case 16: return CALL(16);   \
-        case 32: return CALL(32);   \
-        case 64: return CALL(64);   \
-        case 128: return CALL(128); \
-        case 256: return CALL(256); \
-        case 512: return CALL(512); \
-        case 1024: return CALL(1024); \
-        case 2048: return CALL(2048); \
-        case 4096: return CALL(4096); \
-        case 8192: return CALL(8192); \
-        case 16384: return CALL(16384); \
-        default: return cudaErrorInvalidValue; \
-    }
-
-cudaError_t launch_fwd_1d(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
-#define HY_CALL(X) launch_fwd_1d_mc<X>(a, dt, even, st)
-    HY_MC_SWITCH(MC, HY_CALL)
-#undef HY_CALL
-}
-
-cudaError_t launch_spec_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
-                           const c32 *tw, cudaStream_t st) {
-#define HY_CALL(X) launch_spec_1d_mc<X>(h, h_stride, L, Hout, nrows, tw, st)
-    HY_MC_SWITCH(MC, HY_CALL)
-#undef HY_CALL
-}
-
-cudaError_t launch_implicit(const ImplicitArgs &a, cudaStream_t st) {
-    const int64_t grid = (a.npos + IMP_TP - 1) / IMP_TP;
-    if (a.p.width <= 64)
-        hyena_implicit_filter_kernel<64><<<(unsigned)grid, IMP_THREADS, 0, st>>>(a);
-    else
-        hyena_implicit_filter_kernel<128><<<(unsigned)grid, IMP_THREADS, 0, st>>>(a);
-    return cudaGetLastError();
-}
-
-// ------------------------------------------------------------- cluster paths
-using G1_32K = ClusterGeom<32768, 4, 128, 16>;    // 1D, 32768 < M <= 65536
-using G1_64K = ClusterGeom<65536, 8, 256, 16>;    // 1D, M = 131072
-using G1_128K = ClusterGeom<131072, 8, 512, 32>;  // 1D, M = 262144
-using G2_32 = ClusterGeom<2048, 1, 64, 16>;       // 2D, 32 x 32 grid (64 x 64 padded)
-using G2_64 = ClusterGeom<8192, 2, 128, 16>;      // 2D, 64 x 64
-using G2_128 = ClusterGeom<32768, 4, 256, 16>;    // 2D, 128 x 128
-using G2_256 = ClusterGeom<131072, 8, 512, 32>;   // 2D, 256 x 256
-
-template <typename G, typename Kern, typename... Args>
-cudaError_t launch_cluster(Kern kern, int64_t units, cudaStream_t st, Args... args) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * G::C), 1, 1);
-    cfg.blockDim = dim3(G::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = G::SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = G::C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, args...);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
-
-template <typename G>
-cudaError_t launch_fwd_1d_cluster_g(const Fwd1dArgs &a, hyena_dtype_t dt, bool even, cudaStream_t st) {
-    if (dt == HYENA_F32)
-        return even ? launch_cluster<G>(hyena_fwd_1d_cluster<G, float, true>, a.rows, st, a)
-                    : launch_cluster<G>(hyena_fwd_1d_cluster<G, float, false>, a.rows, st, a);
-    return even ? launch_cluster<G>(hyena_fwd_1d_cluster<G, __nv_bfloat16, true>, a.rows, st, a)
-                : launch_cluster<G>(hyena_fwd_1d_cluster<G, __nv_bfloat16, false>, a.rows, st, a);
-}
-
-cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
-    switch (MC) {
-        case 32768: return launch_fwd_1d_cluster_g<G1_32K>(a, dt, even, st);
-        case 65536: return launch_fwd_1d_cluster_g<G1_64K>(a, dt, even, st);
-        case 131072: return launch_fwd_1d_cluster_g<G1_128K>(a, dt, even, st);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
-                                   const c32 *tw, cudaStream_t st) {
-    switch (MC) {
-        case 32768: return launch_cluster<G1_32K>(hyena_spectrum_1d_cluster<G1_32K>, nrows, st, h, h_stride, L, Hout, tw);
-        case 65536: return launch_cluster<G1_64K>(hyena_spectrum_1d_cluster<G1_64K>, nrows, st, h, h_stride, L, Hout, tw);
-        case 131072:
-            return launch_cluster<G1_128K>(hyena_spectrum_1d_cluster<G1_128K>, nrows, st, h, h_stride, L, Hout, tw);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-template <typename G>
-cudaError_t launch_fwd_2d_g(const Fwd2dArgs &a, hyena_dtype_t dt, cudaStream_t st) {
-    if (dt == HYENA_F32) return launch_cluster<G>(hyena_fwd_2d_cluster<G, float>, a.planes, st, a);
-    return launch_cluster<G>(hyena_fwd_2d_cluster<G, __nv_bfloat16>, a.planes, st, a);
-}
-
-cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st) {
-    switch (W) {
-        case 32: return launch_fwd_2d_g<G2_32>(a, dt, st);
-        case 64: return launch_fwd_2d_g<G2_64>(a, dt, st);
-        case 128: return launch_fwd_2d_g<G2_128>(a, dt, st);
-        case 256: return launch_fwd_2d_g<G2_256>(a, dt, st);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W, const c32 *tw,
-                           cudaStream_t st) {
-    switch (W) {
-        case 32: return launch_cluster<G2_32>(hyena_spectrum_2d_cluster<G2_32>, n, st, K, rs, cs, Kout, tw);
-        case 64: return launch_cluster<G2_64>(hyena_spectrum_2d_cluster<G2_64>, n, st, K, rs, cs, Kout, tw);
-        case 128: return launch_cluster<G2_128>(hyena_spectrum_2d_cluster<G2_128>, n, st, K, rs, cs, Kout, tw);
-        case 256: return launch_cluster<G2_256>(hyena_spectrum_2d_cluster<G2_256>, n, st, K, rs, cs, Kout, tw);
-        default: return cudaErrorInvalidValue;
-    }
 }
 
 // W_M^m = exp(-2 pi i m / M), m in [0, M), computed in double and rounded once.

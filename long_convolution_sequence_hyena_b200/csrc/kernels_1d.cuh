@@ -94,21 +94,43 @@ __device__ __forceinline__ c32 ldg_c(const c32 *p) {
     return mk(f.x, f.y);
 }
 
+// Asynchronous 8-byte global -> shared copy (bypasses registers).
+__device__ __forceinline__ void cp_async8(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Whether the fused CTA kernel stages each order's spectrum row in shared
+// memory (it must fit next to the exchange buffer).
+constexpr bool stage_spectrum(int MC) { return MC <= 8192; }
+constexpr int fwd_threads(int MC, int E) { return rows_per_cta(MC, E) * (MC / E); }
+constexpr int fwd_min_blocks(int MC, int E) {
+    return fwd_threads(MC, E) >= 512 ? 1 : (fwd_threads(MC, E) >= 256 ? 2 : 4);
+}
+// Shared floats per row: exchange buffer (re, im planes) + staged spectrum row.
+constexpr int fwd_smem_floats_per_row(int MC) { return 2 * MC + (stage_spectrum(MC) ? 2 * (MC + 1) : 0); }
+
 // Spectral step of one order for a row held as packed complex spectrum Z
 // (natural order in registers): unpack the real-row spectrum X, multiply by
 // the filter gain plus the feedthrough (the feedthrough is the delta tap, whose
 // spectrum is the constant Dskip), repack for the half-length inverse, and fold
 // in the 1/2 of the repacking and the 1/MC of the inverse transform.
+// Hs: the spectrum row staged in shared memory (cp.async group pending), or
+// nullptr to read Hrow from global memory. wt = W_M^t.
 template <int MC, int E>
 __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim,
-                                                 int t, const c32 *__restrict__ Hrow, float dsk,
-                                                 const c32 *__restrict__ tw) {
+                                                 int t, const c32 *__restrict__ Hrow, const c32 *Hs, float dsk,
+                                                 c32 wt) {
     constexpr int T = MC / E;
 #pragma unroll
     for (int q = 0; q < E; ++q) {
         sre[t + q * T] = v[q].x;
         sim[t + q * T] = v[q].y;
     }
+    if (Hs) cp_async_wait_all();
     __syncthreads();
     constexpr float s = 0.5f / (float)MC;
 #pragma unroll
@@ -119,12 +141,12 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
         const c32 Zm = mk(sre[km], sim[km]);
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        const c32 w = ldg_c(tw + k);
+        const c32 w = mul(wt, w2e<E>(q));            // W_M^{t + qT} = W_M^t W_{2E}^q
         const c32 wO = mul(w, Ok);
         const c32 Xk = add(Ek, wO);
         const c32 Xm = conj(sub(Ek, wO));
-        c32 Hk = ldg_c(Hrow + k);
-        c32 Hm = ldg_c(Hrow + (MC - k));
+        c32 Hk = Hs ? Hs[k] : ldg_c(Hrow + k);
+        c32 Hm = Hs ? Hs[MC - k] : ldg_c(Hrow + (MC - k));
         Hk.x += dsk;
         Hm.x += dsk;
         const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
@@ -132,6 +154,7 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
         const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
         const c32 Yo = mul(Yd, conj(w));
         v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+        if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
     }
     __syncthreads();
 }
@@ -140,10 +163,11 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
 // Grid: ceil(B*D / rows_per_cta) CTAs, rows visited d-major / b-minor so the B
 // rows that read the same filter spectrum run at the same time (L2 reuse).
 template <int MC, int E, typename IO, bool EVEN>
-__global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
+__global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
     hyena_fwd_1d_cta(const Fwd1dArgs a) {
     constexpr int T = MC / E;
     constexpr int RPC = rows_per_cta(MC, E);
+    constexpr bool HS = stage_spectrum(MC);
     extern __shared__ float smem[];
     const int lrow = threadIdx.x / T;
     const int t = threadIdx.x - lrow * T;
@@ -152,9 +176,11 @@ __global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
     const int64_t d = active ? ord / a.B : 0;
     const int64_t b = active ? ord - d * a.B : 0;
     const int64_t row = b * a.D + d;
-    float *sre = smem + lrow * 2 * MC;
+    float *sre = smem + lrow * fwd_smem_floats_per_row(MC);
     float *sim = sre + MC;
+    c32 *Hs = HS ? reinterpret_cast<c32 *>(sim + MC) : nullptr;
     const int64_t L = a.L;
+    const c32 wt = ldg_c(a.tw + t);                       // W_M^t
 
     c32 v[E];
     {
@@ -173,9 +199,14 @@ __global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
         for (int q = 0; q < E / 2; ++q)
             g[q] = active ? load_pair_raw<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L) : io<IO>::zero();
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        if constexpr (HS) {  // stage the spectrum row while the forward FFT runs
+            for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);
+            cp_async_commit();
+        }
 
         fft_cta<MC, E, -1, true>(v, sre, sim, t, a.tw);
-        spectral_product<MC, E>(v, sre, sim, t, a.H + ((int64_t)n * a.D + d) * (MC + 1), dsk, a.tw);
+        spectral_product<MC, E>(v, sre, sim, t, Hrow, Hs, dsk, wt);
         fft_cta<MC, E, +1, false>(v, sre, sim, t, a.tw);
 
         // gate; positions >= L are cleared so the next order sees a zero-padded row

@@ -1,0 +1,28 @@
+#pragma once
+// Launch wrappers shared by the translation units of the library.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "hyena.h"
+#include "kernels_1d.cuh"
+#include "kernels_implicit.cuh"
+
+namespace hyena {
+
+// 1D, single CTA group per row (MC <= 16384)
+cudaError_t launch_fwd_1d(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
+cudaError_t launch_spec_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
+                           const c32 *tw, cudaStream_t st);
+// 1D, one cluster per row (MC in {32768, 65536, 131072})
+cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
+cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
+                                   const c32 *tw, cudaStream_t st);
+// 2D, one cluster per plane (H == W in {32, 64, 128, 256})
+struct Fwd2dArgs;
+cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);
+cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W, const c32 *tw,
+                           cudaStream_t st);
+// implicit filter network
+cudaError_t launch_implicit(const ImplicitArgs &a, cudaStream_t st);
+
+}  // namespace hyena
