@@ -234,9 +234,9 @@ def run_ours(args, w, rank, world, dist):
 
 
 # ------------------------------------------------------------ oracle (CPU)
-def oracle_sample(w, seconds):
-    """Time the fp64 oracle on a bounded sample of the workload's rows (planes).
-    Returns (elements/s, sample description, threads)."""
+def oracle_runner(w):
+    """Prepare the fp64 oracle on rows (planes) of the workload's recipe.
+    Returns (run(rows) -> None, elements per row, threads)."""
     import numpy as np
 
     import oracle
@@ -246,13 +246,14 @@ def oracle_sample(w, seconds):
     inp = make_inputs(small)
     threads = oracle.num_threads()
     N = w.order
+    names = ("W1", "b1", "W2", "b2", "W3", "b3")
     if w.ndim == 1:
         L = w.shape[0]
         if "h" in inp:
             h64 = inp["h"].double().numpy()
         else:
             p = inp["implicit"]
-            h64 = oracle.implicit_filter_1d(L, N, small.D, *(p[k].double().numpy() for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
+            h64 = oracle.implicit_filter_1d(L, N, small.D, *(p[k].double().numpy() for k in names),
                                             p["alpha"].double().numpy(), p["num_freqs"], p["omega0"], p["omega_hidden"])
         v = inp["v"].double().reshape(small.D, L).numpy()
         g = inp["gates"].double().reshape(N, small.D, L).numpy()
@@ -264,9 +265,12 @@ def oracle_sample(w, seconds):
         unit = L
     else:
         H, W = w.shape
-        p = inp["implicit"]
-        k64 = oracle.implicit_filter_2d(H, W, N, small.D, *(p[k].double().numpy() for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
-                                        p["sigma"].double().numpy(), p["omega0"], p["omega_hidden"])
+        if "h" in inp:
+            k64 = inp["h"].double().numpy()
+        else:
+            p = inp["implicit"]
+            k64 = oracle.implicit_filter_2d(H, W, N, small.D, *(p[k].double().numpy() for k in names),
+                                            p["sigma"].double().numpy(), p["omega0"], p["omega_hidden"])
         v = inp["v"].double().reshape(small.D, H, W).numpy()
         g = inp["gates"].double().reshape(N, small.D, H, W).numpy()
         d = inp["dskip"].double().numpy()
@@ -275,22 +279,51 @@ def oracle_sample(w, seconds):
             idx = np.arange(rows) % small.D
             oracle.hyena_2d(v[idx], g[:, idx], k64, d, fidx=idx)
         unit = H * W
+    return run, unit, threads
+
+
+def calibrate_rows(run, threads, seconds):
+    """Rows (a multiple of the thread count) whose oracle run takes about `seconds`."""
     rows = threads
     t0 = time.perf_counter()
     run(rows)
     dt = time.perf_counter() - t0
-    while dt < seconds / 4 and rows < 64 * threads:
+    while dt < seconds / 4 and rows < 4096 * threads:
         rows *= 2
         t0 = time.perf_counter()
         run(rows)
         dt = time.perf_counter() - t0
-    target = max(threads, int(rows * seconds / max(dt, 1e-9)) // threads * threads)
-    if target > rows:
-        rows = target
+    return max(threads, int(rows * seconds / max(dt, 1e-9)) // threads * threads)
+
+
+def oracle_sample(w, seconds):
+    """Time the fp64 oracle on a bounded sample of the workload's rows (planes).
+    Returns (elements/s, sample description, threads, seconds)."""
+    run, unit, threads = oracle_runner(w)
+    rows = calibrate_rows(run, threads, seconds)
+    t0 = time.perf_counter()
+    run(rows)
+    dt = time.perf_counter() - t0
+    return rows * unit / dt, "%d rows of the workload (%d elements each), direct fp64 sum" % (rows, unit), threads, dt
+
+
+def run_reference(args, w):
+    """The reference arm: the oracle as it stands, W warm-up and K timed steps,
+    each step a bounded sample of the workload's rows (sized so the whole run
+    takes about two minutes)."""
+    run, unit, threads = oracle_runner(w)
+    per_step = max(0.5, 120.0 / (args.steps + args.warmup))
+    rows = calibrate_rows(run, threads, per_step)
+    for _ in range(args.warmup):
+        run(rows)
+    times = []
+    for _ in range(args.steps):
         t0 = time.perf_counter()
         run(rows)
-        dt = time.perf_counter() - t0
-    return rows * unit / dt, "%d rows of the workload (%d elements each), direct fp64 sum" % (rows, unit), threads, dt
+        times.append(time.perf_counter() - t0)
+    value = rows * unit * len(times) / sum(times)
+    sample = "%d rows of the workload (%d elements each) per step, direct fp64 sum" % (rows, unit)
+    return value, sample, threads
 
 
 def main():
@@ -309,7 +342,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        value, sample, threads, secs = oracle_sample(w, args.cpu_seconds)
+        value, sample, threads = run_reference(args, w)
         line = {"metric": metric, "value": value, "unit": "elems/s", "n_gpus": args.gpus, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": w.elements * world / value * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,

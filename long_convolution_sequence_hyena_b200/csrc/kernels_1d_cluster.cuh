@@ -9,13 +9,15 @@
 //   3. transpose through distributed shared memory (each CTA then owns M1/C
 //      rows k1 with all n2);
 //   4. row FFTs of length M2 over n2, giving Z[k1 + M1 k2].
-// The spectral step reads the mirror bin Z[MC - k] from whichever CTA owns it
-// (a DSMEM load), and the inverse runs the same steps backwards, ending in the
-// column layout, so the gate and the next order's input stay in registers.
+// The spectral step reads the mirror bin Z[MC - k] from the same CTA (rows
+// are assigned in mirror pairs), and the inverse runs the same steps
+// backwards, ending in the column layout, so the gate and the next order's
+// input stay in registers.
 //
-// Synchronisation is barrier.cluster only (no flag polling). With two
-// buffers (column, row) a transpose needs one cluster barrier after it; with
-// a single buffer (when two do not fit) also one before it.
+// Synchronisation is barrier.cluster only (no flag polling): one cluster
+// barrier after each transpose, two per order. Rows are paired with their
+// mirror rows inside one CTA, so the spectral step reads only local shared
+// memory.
 #pragma once
 #include <cooperative_groups.h>
 
@@ -29,16 +31,17 @@ template <int MC_, int C_, int M1_, int E_>
 struct ClusterGeom {
     static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_;
     static constexpr int NCOL = M2 / C;          // columns per CTA (column phase)
-    static constexpr int NROW = M1 / C;          // rows per CTA (row phase)
+    static constexpr int NROW = M1 / C;          // rows per CTA (row phase), in mirror pairs
+    static constexpr int HROW = NROW / 2;        // rows k1 < M1/2 per CTA
     static constexpr int T1 = M1 / E;            // threads per column FFT
     static constexpr int T2 = M2 / E;            // threads per row FFT
     static constexpr int THREADS = NCOL * T1;
     static constexpr int PER_CTA = MC / C;       // complex elements per CTA per buffer
-    static constexpr bool TWO_BUF = 2 * PER_CTA * 8 <= 160 * 1024;
-    static constexpr size_t SMEM = (TWO_BUF ? 2 : 1) * (size_t)PER_CTA * 8;
+    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8;   // column buffer + row buffer
     static_assert(THREADS == NROW * T2, "both phases must use the same thread count");
-    static_assert(NCOL >= 32 && NROW >= 32, "interleaved layouts need at least 32 sequences");
+    static_assert(NCOL >= 16 && NROW >= 16, "interleaved layouts need at least 16 sequences");
     static_assert(THREADS <= 1024, "too many threads");
+    static_assert(SMEM <= 200 * 1024, "two buffers must fit in shared memory");
 };
 
 // Distributed shared memory through 32-bit shared::cluster addresses.
@@ -48,13 +51,12 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t local, int rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
     return remote;
 }
-__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
 __device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// Cluster barrier that also orders shared::cluster memory (release / acquire).
+__device__ __forceinline__ void cluster_sync_mem() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Interleaved address of element i of sequence s (NSEQ sequences), matching saddr<.., NSEQ>.
@@ -63,25 +65,53 @@ __device__ __forceinline__ int iaddr(int i, int s) {
     return i * NSEQ + (s ^ (i & (NSEQ - 1)));
 }
 
+// Rows of the row phase are held in mirror pairs: CTA c owns rows k1 in
+// [c HROW, (c+1) HROW) (slots 0..HROW-1) and their mirrors M1 - k1 (slots
+// HROW..NROW-1; the mirror slot of row 0 holds row M1/2). Every bin's mirror
+// bin then lies in the same CTA, so the spectral step needs no DSMEM access.
+template <typename G>
+__device__ __forceinline__ int row_of_slot(int c, int r) {
+    const int base = c * G::HROW + (r % G::HROW);
+    if (r < G::HROW) return base;
+    return base == 0 ? G::M1 / 2 : G::M1 - base;
+}
+template <typename G>
+__device__ __forceinline__ void slot_of_row(int k1, int &c, int &r) {
+    if (k1 < G::M1 / 2) {
+        c = k1 / G::HROW;
+        r = k1 % G::HROW;
+    } else if (k1 == G::M1 / 2) {
+        c = 0;
+        r = G::HROW;
+    } else {
+        const int kb = G::M1 - k1;
+        c = kb / G::HROW;
+        r = G::HROW + kb % G::HROW;
+    }
+}
+
 // Per-thread coordinates and buffers of one CTA of the cluster.
 // TWID: apply the four-step twiddle W_MC^{n2 k1} between the two FFT stages
 // (1D: one transform of length MC); without it the two stages are the two
 // axes of a 2D transform of shape [M1][M2].
-template <typename G, bool TWID = true>
+// HALFX: columns n2 >= M2/2 hold zeros on input and are not needed on output
+// (2D, the zero-padded half of the x axis): they are neither transformed nor sent.
+template <typename G, bool TWID, bool HALFX>
 struct ClusterCtx {
-    // Twiddle table length: W_M, M = 2 MC (1D); for 2D the table must cover
-    // both axes and the real-packing twiddle: W_{2 M2} with 2 M2 >= M1 (see the plan).
+    // Twiddle table length: 1D, W_M with M = 2 MC; 2D, W_{2 M2} with 2 M2 >= M1.
     static constexpr int TWM = TWID ? 2 * G::MC : (2 * G::M2 >= G::M1 ? 2 * G::M2 : G::M1);
-    cg::cluster_group cluster;
     float *col_re, *col_im, *row_re, *row_im;
+    int crank;
     int j, t1, n2;   // column phase: local column, FFT lane, global column
-    int r, t2, k1;   // row phase: local row, FFT lane, global row
+    int r, t2, k1;   // row phase: local slot, FFT lane, global row
+    int rm;          // slot of the mirror row of k1
+    bool col_live;   // this CTA owns at least one column that carries data
 
-    __device__ __forceinline__ ClusterCtx(float *smem) : cluster(cg::this_cluster()) {
-        const int crank = (int)cluster.block_rank();
+    __device__ __forceinline__ ClusterCtx(float *smem) {
+        crank = (int)cg::this_cluster().block_rank();
         col_re = smem;
         col_im = col_re + G::PER_CTA;
-        row_re = G::TWO_BUF ? col_im + G::PER_CTA : col_re;
+        row_re = col_im + G::PER_CTA;
         row_im = row_re + G::PER_CTA;
         const int tid = threadIdx.x;
         j = tid % G::NCOL;
@@ -89,47 +119,60 @@ struct ClusterCtx {
         n2 = crank * G::NCOL + j;
         r = tid % G::NROW;
         t2 = tid / G::NROW;
-        k1 = crank * G::NROW + r;
+        k1 = row_of_slot<G>(crank, r);
+        rm = (k1 == 0 || k1 == G::M1 / 2) ? r : (r < G::HROW ? r + G::HROW : r - G::HROW);
+        col_live = !HALFX || crank * G::NCOL < G::M2 / 2;
     }
 
-    // Position (complex index) of column-layout register q: n = M2 * (t1 + q T1) + n2.
+    // Complex index of column-layout register q: n = M2 * (t1 + q T1) + n2.
     __device__ __forceinline__ int64_t col_index(int q) const { return (int64_t)G::M2 * (t1 + q * G::T1) + n2; }
-    // Bin of row-layout register q: k = k1 + M1 * (t2 + q T2).
-    __device__ __forceinline__ int row_bin(int q) const { return k1 + G::M1 * (t2 + q * G::T2); }
 
-    // Column layout (time domain) -> row layout (natural bins).
-    // HALF_COL: the upper half of every column is zero (n1 >= M1/2);
-    // HALF_ROW: the upper half of every row is zero after the first stage (n2 >= M2/2).
-    template <bool HALF_COL = true, bool HALF_ROW = false>
+    // v[q] *= base * step^q, q = 0..E-1 (product tree of depth <= 4, then one multiply).
+    __device__ __forceinline__ static void twiddle_ramp(c32 (&v)[G::E], c32 base, c32 step) {
+        twiddle_powers<G::E, 1, 0>(v, step);
+#pragma unroll
+        for (int q = 0; q < G::E; ++q) v[q] = mul(v[q], base);
+    }
+
+    // Column layout (time domain, upper half of every column zero unless
+    // !HALF_COL) -> row layout (natural bins, register q = bin k2 = t2 + q T2 of row k1).
+    template <bool HALF_COL>
     __device__ __forceinline__ void forward(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
-        fft_cta<G::M1, E, -1, HALF_COL, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
-        if constexpr (TWID) {
+        if (col_live) {
+            fft_cta<G::M1, E, -1, HALF_COL, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
+            if constexpr (TWID) {
+                constexpr int M = 2 * G::MC;
+                const c32 b = ldg_c(tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
+                const c32 st = ldg_c(tw + ((2 * (int64_t)n2 * G::T1) & (M - 1)));
+                twiddle_ramp(v, b, st);
+            }
+            if (!HALFX || 2 * n2 < G::M2) {
 #pragma unroll
-            for (int q = 0; q < E; ++q) {
-                const int kk = t1 + q * G::T1;
-                v[q] = mul(v[q], ldg_c(tw + ((2 * (int64_t)n2 * kk) & (TWM - 1))));
+                for (int q = 0; q < E; ++q) {
+                    int dst, slot;
+                    slot_of_row<G>(t1 + q * G::T1, dst, slot);
+                    const uint32_t ad = dsmem_map(smem_u32(row_re + iaddr<G::NROW>(n2, slot)), dst);
+                    dsmem_st(ad, v[q].x);
+                    dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
+                }
             }
         }
-        if constexpr (!G::TWO_BUF) cluster.sync();    // every CTA done reading its buffer
+        cluster_sync_mem();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int kk = t1 + q * G::T1;
-            const uint32_t ad = dsmem_map(smem_u32(row_re + iaddr<G::NROW>(n2, kk % G::NROW)), kk / G::NROW);
-            dsmem_st(ad, v[q].x);
-            dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
-        }
-        cluster.sync();
-#pragma unroll
-        for (int q = 0; q < E; ++q) {
-            const int ad = iaddr<G::NROW>(t2 + q * G::T2, r);
-            v[q] = mk(row_re[ad], row_im[ad]);
+            if (HALFX && q >= E / 2) {
+                v[q] = mk(0.f, 0.f);
+            } else {
+                const int ad = iaddr<G::NROW>(t2 + q * G::T2, r);
+                v[q] = mk(row_re[ad], row_im[ad]);
+            }
         }
         __syncthreads();
-        fft_cta<G::M2, E, -1, HALF_ROW, TWM, G::NROW>(v, row_re, row_im, t2, tw, r);
+        fft_cta<G::M2, E, -1, HALFX, TWM, G::NROW>(v, row_re, row_im, t2, tw, r);
     }
 
-    // Publish the row-layout spectrum so any CTA can read mirror bins (ends with a cluster barrier).
+    // Store the row-layout bins so the mirror bins can be read (ends with a CTA barrier).
     __device__ __forceinline__ void publish(const c32 (&v)[G::E]) {
 #pragma unroll
         for (int q = 0; q < G::E; ++q) {
@@ -137,58 +180,58 @@ struct ClusterCtx {
             row_re[ad] = v[q].x;
             row_im[ad] = v[q].y;
         }
-        cluster.sync();
+        __syncthreads();
     }
-
-    // Published bin k (any CTA).
-    __device__ __forceinline__ c32 bin(int k) {
-        const int kr = k % G::M1, kc = k / G::M1;
-        const int ad = iaddr<G::NROW>(kc, kr % G::NROW);
-        const uint32_t ra = dsmem_map(smem_u32(row_re + ad), kr / G::NROW);
-        return mk(dsmem_ld(ra), dsmem_ld(ra + 4 * G::PER_CTA));
+    // Published bin (mirror row, column k2m) from this CTA's own buffer.
+    __device__ __forceinline__ c32 mirror_bin(int k2m) const {
+        const int ad = iaddr<G::NROW>(k2m, rm);
+        return mk(row_re[ad], row_im[ad]);
     }
 
     // Row layout (bins) -> column layout (time domain, unscaled inverse).
+    // Must follow a CTA barrier after the last read of the published bins.
     __device__ __forceinline__ void inverse(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
         fft_cta<G::M2, E, +1, false, TWM, G::NROW>(v, row_re, row_im, t2, tw, r);
         if constexpr (TWID) {
-#pragma unroll
-            for (int q = 0; q < E; ++q) {
-                const int nn = t2 + q * G::T2;
-                v[q] = mul(v[q], conj(ldg_c(tw + ((2 * (int64_t)nn * k1) & (TWM - 1)))));
-            }
+            constexpr int M = 2 * G::MC;
+            const c32 b = conj(ldg_c(tw + ((2 * (int64_t)t2 * k1) & (M - 1))));
+            const c32 st = conj(ldg_c(tw + ((2 * (int64_t)G::T2 * k1) & (M - 1))));
+            twiddle_ramp(v, b, st);
         }
-        if constexpr (!G::TWO_BUF) cluster.sync();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int nn = t2 + q * G::T2;
+            if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
             const uint32_t ad = dsmem_map(smem_u32(col_re + iaddr<G::NCOL>(k1, nn % G::NCOL)), nn / G::NCOL);
             dsmem_st(ad, v[q].x);
             dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
         }
-        cluster.sync();
+        cluster_sync_mem();
+        if (col_live) {
 #pragma unroll
-        for (int q = 0; q < E; ++q) {
-            const int ad = iaddr<G::NCOL>(t1 + q * G::T1, j);
-            v[q] = mk(col_re[ad], col_im[ad]);
+            for (int q = 0; q < E; ++q) {
+                const int ad = iaddr<G::NCOL>(t1 + q * G::T1, j);
+                v[q] = mk(col_re[ad], col_im[ad]);
+            }
+            __syncthreads();
+            fft_cta<G::M1, E, +1, false, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
         }
-        __syncthreads();
-        fft_cta<G::M1, E, +1, false, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
     }
 };
 
 // Fused order-N forward, one cluster per row (rows visited d-major, b-minor).
 template <typename G, typename IO, bool EVEN>
 __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1dArgs a) {
-    constexpr int MC = G::MC, E = G::E;
+    constexpr int MC = G::MC, E = G::E, M1 = G::M1;
     extern __shared__ float smem[];
-    ClusterCtx<G> cx(smem);
+    ClusterCtx<G, true, false> cx(smem);
     const int64_t ord = (int64_t)blockIdx.x / G::C;     // one cluster per row
     const int64_t d = ord / a.B;
     const int64_t b = ord - d * a.B;
     const int64_t row = b * a.D + d;
     const int64_t L = a.L;
+    const c32 wb = ldg_c(a.tw + cx.k1 + M1 * cx.t2);     // W_M^{k1 + M1 t2}
 
     c32 v[E];
     {
@@ -207,17 +250,19 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
         const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
 
-        cx.forward(v, a.tw);
+        cx.template forward<true>(v, a.tw);
         cx.publish(v);
         constexpr float s = 0.5f / (float)MC;
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int k = cx.row_bin(q);
-            const c32 Zm = cx.bin((MC - k) & (MC - 1));
+            const int k2 = cx.t2 + q * G::T2;
+            const int k = cx.k1 + M1 * k2;
+            const int km = (MC - k) & (MC - 1);
+            const c32 Zm = cx.mirror_bin(km / M1);
             const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-            const c32 w = ldg_c(a.tw + k);
+            const c32 w = mul(wb, w2e<E>(q));              // W_M^k, k = k1 + M1 (t2 + q T2)
             const c32 wO = mul(w, Ok);
             const c32 Xk = add(Ek, wO);
             const c32 Xm = conj(sub(Ek, wO));
@@ -232,7 +277,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
             v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
             if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
         }
-        cx.cluster.sync();                              // mirror reads done before buffers are rewritten
+        __syncthreads();                                // mirror reads done before the row buffer is rewritten
         cx.inverse(v, a.tw);
 
         // gate (registers q >= E/2 hold positions >= MC, i.e. padding)
@@ -254,13 +299,13 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
 // Spectrum of long causal filters (same layout as hyena_spectrum_1d), one
 // cluster per filter row. h row o starts at h + o * h_stride and has L taps.
 // In place (h == Hout) is allowed: every CTA reads its part of the row before
-// the first cluster barrier, and bins are written after the last one.
+// the first cluster barrier, and bins are written after it.
 template <typename G>
 __global__ void __launch_bounds__(G::THREADS, 1)
     hyena_spectrum_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, const c32 *__restrict__ tw) {
-    constexpr int MC = G::MC, E = G::E;
+    constexpr int MC = G::MC, E = G::E, M1 = G::M1;
     extern __shared__ float smem[];
-    ClusterCtx<G> cx(smem);
+    ClusterCtx<G, true, false> cx(smem);
     const int64_t o = (int64_t)blockIdx.x / G::C;
     const float *hrow = h + o * h_stride;
     c32 v[E];
@@ -271,28 +316,20 @@ __global__ void __launch_bounds__(G::THREADS, 1)
     }
 #pragma unroll
     for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
-    cx.cluster.sync();                                  // whole row read before any bin is written
-    cx.forward(v, tw);
+    cx.template forward<true>(v, tw);                   // contains a cluster barrier after all reads
     cx.publish(v);
+    const c32 wb = ldg_c(tw + cx.k1 + M1 * cx.t2);
     c32 *Hrow = Hout + o * (MC + 1);
-    c32 outv[E];
-    c32 nyq = mk(0.f, 0.f);
 #pragma unroll
     for (int q = 0; q < E; ++q) {
-        const int k = cx.row_bin(q);
-        const c32 Zm = cx.bin((MC - k) & (MC - 1));
+        const int k = cx.k1 + M1 * (cx.t2 + q * G::T2);
+        const int km = (MC - k) & (MC - 1);
+        const c32 Zm = cx.mirror_bin(km / M1);
         const c32 Zk = v[q];
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        outv[q] = add(Ek, mul(ldg_c(tw + k), Ok));
-        if (k == 0) nyq = mk(Ek.x - Ok.x, 0.f);
-    }
-    cx.cluster.sync();                                  // all mirror reads done; no CTA touches DSMEM after this
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-        const int k = cx.row_bin(q);
-        Hrow[k] = outv[q];
-        if (k == 0) Hrow[MC] = nyq;
+        Hrow[k] = add(Ek, mul(mul(wb, w2e<E>(q)), Ok));
+        if (k == 0) Hrow[MC] = mk(Ek.x - Ok.x, 0.f);  // Nyquist bin: E_0 - O_0, real
     }
 }
 

@@ -34,7 +34,7 @@ struct Fwd2dArgs {
 // Fused order-N 2D forward (planes visited c-major, b-minor).
 template <typename G, typename IO>
 __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2dArgs a) {
-    using Ctx = ClusterCtx<G, false>;
+    using Ctx = ClusterCtx<G, false, true>;
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
     constexpr int Hh = M1 / 2, Ww = M2;                 // plane extents
     constexpr int TWM = Ctx::TWM;
@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
     const int64_t b = ord - c * a.B;
     const int64_t plane = b * a.C + c;
     const bool xin = 2 * cx.n2 < Ww;                    // this column carries data
+    const c32 wb = ldg_c(a.tw + cx.t2 * (TWM / (2 * M2)));   // W_{2 M2}^{t2}
 
     // column-layout register q holds (y = t1 + q T1, x' = n2)
     auto pos_of = [&](int q) -> int64_t { return (int64_t)(cx.t1 + q * G::T1) * Ww + 2 * cx.n2; };
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.C + c) : 0.f;
         const c32 *Kp = a.K + ((int64_t)n * a.C + c) * (M1 * (M2 + 1));
 
-        cx.template forward<true, true>(v, a.tw);
+        cx.template forward<true>(v, a.tw);
         cx.publish(v);
         constexpr float s = 0.5f / (float)(M1 * M2);
         const int ky = cx.k1;
@@ -75,12 +76,11 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int kx = cx.t2 + q * G::T2;
-            const int kxm = (M2 - kx) & (M2 - 1);
-            const c32 Zm = cx.bin(kym + M1 * kxm);
+            const c32 Zm = cx.mirror_bin((M2 - kx) & (M2 - 1));
             const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-            const c32 w = ldg_c(a.tw + kx * (TWM / (2 * M2)));
+            const c32 w = mul(wb, w2e<E>(q));            // W_{2 M2}^{kx}
             const c32 wO = mul(w, Ok);
             const c32 Xk = add(Ek, wO);                  // bin (ky, kx)
             const c32 Xm = conj(sub(Ek, wO));            // bin (-ky, M2 - kx)
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
             v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
             if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
         }
-        cx.cluster.sync();
+        __syncthreads();                                // mirror reads done before the row buffer is rewritten
         cx.inverse(v, a.tw);
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
@@ -116,11 +116,11 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
 // 2D kernel spectra. Kernel (n, c) starts at K + o * cs (o = n * C + c); row iy
 // of its offset grid (offset oy = iy - H) starts at + iy * rs and holds 2W
 // floats (ox = ix - W). In place (K == Kout, rs = 2W + 2, cs = 2H (2W + 2)) is
-// allowed: every read precedes the first cluster barrier.
+// allowed: every read precedes the first cluster barrier, every write follows it.
 template <typename G>
 __global__ void __launch_bounds__(G::THREADS, 1)
     hyena_spectrum_2d_cluster(const float *K, int64_t rs, int64_t cs, c32 *Kout, const c32 *__restrict__ tw) {
-    using Ctx = ClusterCtx<G, false>;
+    using Ctx = ClusterCtx<G, false, false>;
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
     constexpr int Hh = M1 / 2, Ww = M2;
     constexpr int TWM = Ctx::TWM;
@@ -136,31 +136,22 @@ __global__ void __launch_bounds__(G::THREADS, 1)
         const float *rowp = Kp + iy * rs;
         v[q] = mk(rowp[ix], rowp[ix + 1]);
     }
-    cx.cluster.sync();                                  // every read done before anything is written
-    cx.template forward<false, false>(v, tw);
+    cx.template forward<false>(v, tw);                  // contains a cluster barrier after all reads
     cx.publish(v);
     const int ky = cx.k1;
     const int kym = (M1 - ky) & (M1 - 1);
-    c32 outv[E];
-    c32 nyq = mk(0.f, 0.f);
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-        const int kx = cx.t2 + q * G::T2;
-        const c32 Zm = cx.bin(kym + M1 * ((M2 - kx) & (M2 - 1)));
-        const c32 Zk = v[q];
-        const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
-        const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        const c32 wO = mul(ldg_c(tw + kx * (TWM / (2 * M2))), Ok);
-        outv[q] = add(Ek, wO);
-        if (kx == 0) nyq = conj(sub(Ek, wO));            // bin (-ky, M2)
-    }
-    cx.cluster.sync();
+    const c32 wb = ldg_c(tw + cx.t2 * (TWM / (2 * M2)));
     c32 *Ko = Kout + o * (M1 * (M2 + 1));
 #pragma unroll
     for (int q = 0; q < E; ++q) {
         const int kx = cx.t2 + q * G::T2;
-        Ko[(int64_t)ky * (M2 + 1) + kx] = outv[q];
-        if (kx == 0) Ko[(int64_t)kym * (M2 + 1) + M2] = nyq;
+        const c32 Zm = cx.mirror_bin((M2 - kx) & (M2 - 1));
+        const c32 Zk = v[q];
+        const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
+        const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
+        const c32 wO = mul(mul(wb, w2e<E>(q)), Ok);
+        Ko[(int64_t)ky * (M2 + 1) + kx] = add(Ek, wO);
+        if (kx == 0) Ko[(int64_t)kym * (M2 + 1) + M2] = conj(sub(Ek, wO));   // bin (-ky, M2)
     }
 }
 
