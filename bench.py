@@ -136,6 +136,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job time)."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(elements_per_rank, world, ms):
+    """Weak scaling: every rank processes its own full workload; the job's
+    throughput is all ranks' elements over the slowest rank's time."""
+    return elements_per_rank * world / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, w, rank, world, dist):
     import torch
@@ -222,10 +239,7 @@ def run_ours(args, w, rank, world, dist):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    if dist is not None:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist, dev)
     io = 4 if w.dtype == "f32" else 2
     h2d = (w.order + 1) * w.elements * io
     d2h = w.elements * io
@@ -373,7 +387,7 @@ def main():
     achieved_tflops = cost["flops"] / sec / 1e12
     achieved_gbs = cost["bytes"] / sec / 1e9
     t_roof = max(cost["bytes"] / (HBM_NOMINAL_GBS * 1e9), cost["flops"] / (fp32_peak * 1e12))
-    value = w.elements * world / sec
+    value = job_throughput(w.elements, world, ms)
     traffic = None
     prof = os.path.join(ROOT, "profiles", "traffic_%s.json" % w.name)
     try:

@@ -115,10 +115,19 @@ __constant__ float2 c_w64[64] = {
     {9.807852804e-01f, 1.950903220e-01f},
     {9.951847267e-01f, 9.801714033e-02f}};
 
-// W_{2E}^q for a compile-time q (E <= 32).
+// A zero the compiler cannot see through: adding it to a constant-table index
+// keeps the (cheap) constant loads inside loops instead of hoisting them into
+// registers for the whole kernel.
+__device__ __forceinline__ int opaque_zero() {
+    int z;
+    asm volatile("mov.u32 %0, 0;" : "=r"(z));
+    return z;
+}
+
+// W_{2E}^q (E <= 32); z must be opaque_zero().
 template <int E>
-__device__ __forceinline__ c32 w2e(int q) {
-    const float2 f = c_w64[q * (32 / E)];
+__device__ __forceinline__ c32 w2e(int q, int z) {
+    const float2 f = c_w64[q * (32 / E) + z];
     return c32{f.x, f.y};
 }
 
@@ -258,33 +267,34 @@ __device__ __forceinline__ void dftR(c32 (&x)[NR]) {
     else dft2r<DIR, st, o>(x);
 }
 
-// Powers w^1..w^(R-1) of a twiddle applied to x[o + st*r], built by a product
-// tree of depth <= 4 from one table value.
+// Powers w^1..w^(R-1) of a twiddle applied to x[o + st*r]. Four running
+// products p_i = w^i, w^(i+4), w^(i+8), w^(i+12) (each power at most four
+// multiplications from w), applied as they are formed so that few powers are
+// live at once.
 template <int R, int st, int o, int NR>
 __device__ __forceinline__ void twiddle_powers(c32 (&x)[NR], c32 w1) {
-    if constexpr (R >= 2) x[o + st] = mul(x[o + st], w1);
-    if constexpr (R >= 4) {
-        c32 w2 = mul(w1, w1);
-        c32 w3 = mul(w2, w1);
-        x[o + 2 * st] = mul(x[o + 2 * st], w2);
-        x[o + 3 * st] = mul(x[o + 3 * st], w3);
+    if constexpr (R == 2) {
+        x[o + st] = mul(x[o + st], w1);
+    } else {
+        c32 p1 = w1;
+        c32 p2 = mul(w1, w1);
+        c32 p3 = mul(p2, w1);
+        x[o + st] = mul(x[o + st], p1);
+        x[o + 2 * st] = mul(x[o + 2 * st], p2);
+        x[o + 3 * st] = mul(x[o + 3 * st], p3);
         if constexpr (R >= 8) {
-            c32 w4 = mul(w2, w2);
-            c32 w5 = mul(w4, w1), w6 = mul(w4, w2), w7 = mul(w4, w3);
-            x[o + 4 * st] = mul(x[o + 4 * st], w4);
-            x[o + 5 * st] = mul(x[o + 5 * st], w5);
-            x[o + 6 * st] = mul(x[o + 6 * st], w6);
-            x[o + 7 * st] = mul(x[o + 7 * st], w7);
-            if constexpr (R >= 16) {
-                c32 w8 = mul(w4, w4);
-                x[o + 8 * st] = mul(x[o + 8 * st], w8);
-                x[o + 9 * st] = mul(x[o + 9 * st], mul(w8, w1));
-                x[o + 10 * st] = mul(x[o + 10 * st], mul(w8, w2));
-                x[o + 11 * st] = mul(x[o + 11 * st], mul(w8, w3));
-                x[o + 12 * st] = mul(x[o + 12 * st], mul(w8, w4));
-                x[o + 13 * st] = mul(x[o + 13 * st], mul(w8, w5));
-                x[o + 14 * st] = mul(x[o + 14 * st], mul(w8, w6));
-                x[o + 15 * st] = mul(x[o + 15 * st], mul(w8, w7));
+            const c32 w4 = mul(p2, p2);
+            c32 p0 = w4;
+#pragma unroll
+            for (int g = 1; g < R / 4; ++g) {
+                x[o + (4 * g) * st] = mul(x[o + (4 * g) * st], p0);
+                p1 = mul(p1, w4);
+                p2 = mul(p2, w4);
+                p3 = mul(p3, w4);
+                x[o + (4 * g + 1) * st] = mul(x[o + (4 * g + 1) * st], p1);
+                x[o + (4 * g + 2) * st] = mul(x[o + (4 * g + 2) * st], p2);
+                x[o + (4 * g + 3) * st] = mul(x[o + (4 * g + 3) * st], p3);
+                if (g + 1 < R / 4) p0 = mul(p0, w4);
             }
         }
     }

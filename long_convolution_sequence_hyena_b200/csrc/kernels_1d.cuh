@@ -133,6 +133,7 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
     if (Hs) cp_async_wait_all();
     __syncthreads();
     constexpr float s = 0.5f / (float)MC;
+    const int z0 = opaque_zero();
 #pragma unroll
     for (int q = 0; q < E; ++q) {
         const int k = t + q * T;
@@ -141,7 +142,7 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
         const c32 Zm = mk(sre[km], sim[km]);
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        const c32 w = mul(wt, w2e<E>(q));            // W_M^{t + qT} = W_M^t W_{2E}^q
+        const c32 w = mul(wt, w2e<E>(q, z0));            // W_M^{t + qT} = W_M^t W_{2E}^q
         const c32 wO = mul(w, Ok);
         const c32 Xk = add(Ek, wO);
         const c32 Xm = conj(sub(Ek, wO));

@@ -148,10 +148,11 @@ struct ClusterCtx {
                 twiddle_ramp(v, b, st);
             }
             if (!HALFX || 2 * n2 < G::M2) {
+                const int z = opaque_zero();   // recompute addresses per order rather than keep them live
 #pragma unroll
                 for (int q = 0; q < E; ++q) {
                     int dst, slot;
-                    slot_of_row<G>(t1 + q * G::T1, dst, slot);
+                    slot_of_row<G>(t1 + q * G::T1 + z, dst, slot);
                     const uint32_t ad = dsmem_map(smem_u32(row_re + iaddr<G::NROW>(n2, slot)), dst);
                     dsmem_st(ad, v[q].x);
                     dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
@@ -199,9 +200,10 @@ struct ClusterCtx {
             const c32 st = conj(ldg_c(tw + ((2 * (int64_t)G::T2 * k1) & (M - 1))));
             twiddle_ramp(v, b, st);
         }
+        const int z = opaque_zero();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int nn = t2 + q * G::T2;
+            const int nn = t2 + q * G::T2 + z;
             if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
             const uint32_t ad = dsmem_map(smem_u32(col_re + iaddr<G::NCOL>(k1, nn % G::NCOL)), nn / G::NCOL);
             dsmem_st(ad, v[q].x);
@@ -253,6 +255,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
         cx.template forward<true>(v, a.tw);
         cx.publish(v);
         constexpr float s = 0.5f / (float)MC;
+        const int z0 = opaque_zero();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int k2 = cx.t2 + q * G::T2;
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
             const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-            const c32 w = mul(wb, w2e<E>(q));              // W_M^k, k = k1 + M1 (t2 + q T2)
+            const c32 w = mul(wb, w2e<E>(q, z0));              // W_M^k, k = k1 + M1 (t2 + q T2)
             const c32 wO = mul(w, Ok);
             const c32 Xk = add(Ek, wO);
             const c32 Xm = conj(sub(Ek, wO));
@@ -320,6 +323,7 @@ __global__ void __launch_bounds__(G::THREADS, 1)
     cx.publish(v);
     const c32 wb = ldg_c(tw + cx.k1 + M1 * cx.t2);
     c32 *Hrow = Hout + o * (MC + 1);
+    const int z0 = opaque_zero();
 #pragma unroll
     for (int q = 0; q < E; ++q) {
         const int k = cx.k1 + M1 * (cx.t2 + q * G::T2);
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(G::THREADS, 1)
         const c32 Zk = v[q];
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        Hrow[k] = add(Ek, mul(mul(wb, w2e<E>(q)), Ok));
+        Hrow[k] = add(Ek, mul(mul(wb, w2e<E>(q, z0)), Ok));
         if (k == 0) Hrow[MC] = mk(Ek.x - Ok.x, 0.f);  // Nyquist bin: E_0 - O_0, real
     }
 }

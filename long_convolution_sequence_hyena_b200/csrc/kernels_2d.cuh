@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
         constexpr float s = 0.5f / (float)(M1 * M2);
         const int ky = cx.k1;
         const int kym = (M1 - ky) & (M1 - 1);
+        const int z0 = opaque_zero();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int kx = cx.t2 + q * G::T2;
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
             const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-            const c32 w = mul(wb, w2e<E>(q));            // W_{2 M2}^{kx}
+            const c32 w = mul(wb, w2e<E>(q, z0));            // W_{2 M2}^{kx}
             const c32 wO = mul(w, Ok);
             const c32 Xk = add(Ek, wO);                  // bin (ky, kx)
             const c32 Xm = conj(sub(Ek, wO));            // bin (-ky, M2 - kx)
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(G::THREADS, 1)
     const int kym = (M1 - ky) & (M1 - 1);
     const c32 wb = ldg_c(tw + cx.t2 * (TWM / (2 * M2)));
     c32 *Ko = Kout + o * (M1 * (M2 + 1));
+    const int z0 = opaque_zero();
 #pragma unroll
     for (int q = 0; q < E; ++q) {
         const int kx = cx.t2 + q * G::T2;
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(G::THREADS, 1)
         const c32 Zk = v[q];
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
-        const c32 wO = mul(mul(wb, w2e<E>(q)), Ok);
+        const c32 wO = mul(mul(wb, w2e<E>(q, z0)), Ok);
         Ko[(int64_t)ky * (M2 + 1) + kx] = add(Ek, wO);
         if (kx == 0) Ko[(int64_t)kym * (M2 + 1) + M2] = conj(sub(Ek, wO));   // bin (-ky, M2)
     }
