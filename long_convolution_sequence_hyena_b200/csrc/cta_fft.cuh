@@ -4,10 +4,11 @@
 // Two shared-memory layouts:
 //  * NSEQ == 0: one sequence per buffer, contiguous; the Stockham write
 //    pattern is made bank-conflict-free by swz<NS>() (see fft_regs.cuh).
-//  * NSEQ  > 0: NSEQ sequences interleaved, element i of sequence s at
-//    i * NSEQ + (s ^ (i & (NSEQ - 1))). Warps span the sequence index, and
-//    the XOR keeps both "same i, all s" and "same s, consecutive i" accesses
-//    on distinct banks (NSEQ = 32).
+//  * NSEQ  > 0: NSEQ sequences, sequence-major, element i of sequence s at
+//    s * LEN + (i ^ (s & 31)). Warps span the sequence index with a common i,
+//    so the XOR puts the lanes on distinct banks; and lanes that span 32
+//    consecutive i of one sequence touch one contiguous 128-byte block (what
+//    a remote, distributed-shared-memory store wants).
 //
 // Twiddles come from one table of W_TWM^m = exp(-2 pi i m / TWM), m < TWM,
 // with TWM a multiple of LEN.
@@ -26,10 +27,16 @@
 
 namespace hyena {
 
-template <int NS, int NSEQ>
+// Sequence-major address of element i of sequence s (sequences of length LEN >= 32).
+template <int LEN>
+__device__ __forceinline__ int maddr(int i, int s) {
+    return s * LEN + (i ^ (s & 31));
+}
+
+template <int NS, int NSEQ, int LEN>
 __device__ __forceinline__ int saddr(int i, int seq) {
     if constexpr (NSEQ == 0) return swz<NS>(i);
-    else return i * NSEQ + (seq ^ (i & (NSEQ - 1)));
+    else return maddr<LEN>(i, seq);
 }
 
 // One Stockham pass p of a length-LEN FFT (register layout in fft_regs.cuh).
@@ -48,7 +55,7 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
         __syncthreads();  // writes of pass p-1 visible
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int i = saddr<NSP, NSEQ>(t + q * T, seq);
+            const int i = saddr<NSP, NSEQ, LEN>(t + q * T, seq);
             v[q] = mk(sre[i], sim[i]);
         }
         __syncthreads();  // every read done before pass p writes
@@ -67,7 +74,7 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
             const int base = (j / NS) * NS * R + k;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const int i = saddr<NS, NSEQ>(base + r * NS, seq);
+                const int i = saddr<NS, NSEQ, LEN>(base + r * NS, seq);
                 sre[i] = v[s + r * S].x;
                 sim[i] = v[s + r * S].y;
             }

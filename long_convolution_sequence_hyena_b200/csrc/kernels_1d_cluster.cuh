@@ -39,7 +39,8 @@ struct ClusterGeom {
     static constexpr int PER_CTA = MC / C;       // complex elements per CTA per buffer
     static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8;   // column buffer + row buffer
     static_assert(THREADS == NROW * T2, "both phases must use the same thread count");
-    static_assert(NCOL >= 16 && NROW >= 16, "interleaved layouts need at least 16 sequences");
+    static_assert(NCOL >= 16 && NROW >= 16, "warps must span at least 16 sequences");
+    static_assert(M1 >= 32 && M2 >= 32, "sequence-major layouts need sequences of at least 32");
     static_assert(THREADS <= 1024, "too many threads");
     static_assert(SMEM <= 200 * 1024, "two buffers must fit in shared memory");
 };
@@ -57,12 +58,6 @@ __device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
 // Cluster barrier that also orders shared::cluster memory (release / acquire).
 __device__ __forceinline__ void cluster_sync_mem() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Interleaved address of element i of sequence s (NSEQ sequences), matching saddr<.., NSEQ>.
-template <int NSEQ>
-__device__ __forceinline__ int iaddr(int i, int s) {
-    return i * NSEQ + (s ^ (i & (NSEQ - 1)));
 }
 
 // Rows of the row phase are held in mirror pairs: CTA c owns rows k1 in
@@ -153,7 +148,7 @@ struct ClusterCtx {
                 for (int q = 0; q < E; ++q) {
                     int dst, slot;
                     slot_of_row<G>(t1 + q * G::T1 + z, dst, slot);
-                    const uint32_t ad = dsmem_map(smem_u32(row_re + iaddr<G::NROW>(n2, slot)), dst);
+                    const uint32_t ad = dsmem_map(smem_u32(row_re + maddr<G::M2>(n2, slot)), dst);
                     dsmem_st(ad, v[q].x);
                     dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
                 }
@@ -165,7 +160,7 @@ struct ClusterCtx {
             if (HALFX && q >= E / 2) {
                 v[q] = mk(0.f, 0.f);
             } else {
-                const int ad = iaddr<G::NROW>(t2 + q * G::T2, r);
+                const int ad = maddr<G::M2>(t2 + q * G::T2, r);
                 v[q] = mk(row_re[ad], row_im[ad]);
             }
         }
@@ -177,7 +172,7 @@ struct ClusterCtx {
     __device__ __forceinline__ void publish(const c32 (&v)[G::E]) {
 #pragma unroll
         for (int q = 0; q < G::E; ++q) {
-            const int ad = iaddr<G::NROW>(t2 + q * G::T2, r);
+            const int ad = maddr<G::M2>(t2 + q * G::T2, r);
             row_re[ad] = v[q].x;
             row_im[ad] = v[q].y;
         }
@@ -185,7 +180,7 @@ struct ClusterCtx {
     }
     // Published bin (mirror row, column k2m) from this CTA's own buffer.
     __device__ __forceinline__ c32 mirror_bin(int k2m) const {
-        const int ad = iaddr<G::NROW>(k2m, rm);
+        const int ad = maddr<G::M2>(k2m, rm);
         return mk(row_re[ad], row_im[ad]);
     }
 
@@ -205,7 +200,7 @@ struct ClusterCtx {
         for (int q = 0; q < E; ++q) {
             const int nn = t2 + q * G::T2 + z;
             if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
-            const uint32_t ad = dsmem_map(smem_u32(col_re + iaddr<G::NCOL>(k1, nn % G::NCOL)), nn / G::NCOL);
+            const uint32_t ad = dsmem_map(smem_u32(col_re + maddr<G::M1>(k1, nn % G::NCOL)), nn / G::NCOL);
             dsmem_st(ad, v[q].x);
             dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
         }
@@ -213,7 +208,7 @@ struct ClusterCtx {
         if (col_live) {
 #pragma unroll
             for (int q = 0; q < E; ++q) {
-                const int ad = iaddr<G::NCOL>(t1 + q * G::T1, j);
+                const int ad = maddr<G::M1>(t1 + q * G::T1, j);
                 v[q] = mk(col_re[ad], col_im[ad]);
             }
             __syncthreads();
