@@ -100,6 +100,13 @@ __device__ __forceinline__ void cp_async8(void *smem_dst, const void *gmem_src) 
                  "l"(gmem_src)
                  : "memory");
 }
+template <int BYTES>
+__device__ __forceinline__ void cp_async_n(void *smem_dst, const void *gmem_src) {
+    static_assert(BYTES == 4 || BYTES == 8 || BYTES == 16, "cp.async size");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+                 "l"(gmem_src), "n"(BYTES)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 

@@ -37,12 +37,14 @@ struct ClusterGeom {
     static constexpr int T2 = M2 / E;            // threads per row FFT
     static constexpr int THREADS = NCOL * T1;
     static constexpr int PER_CTA = MC / C;       // complex elements per CTA per buffer
-    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8;   // column buffer + row buffer
+    // column buffer + row buffer + staging for one order's gates (E/2 pairs per thread)
+    static constexpr size_t GATE_STAGE = (size_t)THREADS * (E / 2) * 8;
+    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8 + GATE_STAGE;
     static_assert(THREADS == NROW * T2, "both phases must use the same thread count");
     static_assert(NCOL >= 16 && NROW >= 16, "warps must span at least 16 sequences");
     static_assert(M1 >= 32 && M2 >= 32, "sequence-major layouts need sequences of at least 32");
     static_assert(THREADS <= 1024, "too many threads");
-    static_assert(SMEM <= 200 * 1024, "two buffers must fit in shared memory");
+    static_assert(SMEM <= 200 * 1024, "buffers must fit in shared memory");
 };
 
 // Distributed shared memory through 32-bit shared::cluster addresses.
@@ -239,11 +241,21 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
         for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
+    // this order's gates are staged in shared memory (thread-private slots)
+    // while the transforms run, instead of occupying registers
+    using P = typename io<IO>::pair_t;
+    P *gst = reinterpret_cast<P *>(smem + 4 * G::PER_CTA) + threadIdx.x;
     for (int n = 0; n < a.order; ++n) {
         const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + row * L;
-        typename io<IO>::pair_t g[E / 2];
+        if constexpr (EVEN) {
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) g[q] = load_pair_raw<IO, EVEN>(grow, 2 * cx.col_index(q), L);
+            for (int q = 0; q < E / 2; ++q) {
+                const int64_t pos = 2 * cx.col_index(q);
+                if (pos < L) cp_async_n<sizeof(P)>(gst + q * G::THREADS, grow + pos);
+                else gst[q * G::THREADS] = io<IO>::zero();
+            }
+            cp_async_commit();
+        }
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
         const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
 
@@ -279,10 +291,11 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
         cx.inverse(v, a.tw);
 
         // gate (registers q >= E/2 hold positions >= MC, i.e. padding)
+        if constexpr (EVEN) cp_async_wait_all();
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
             const int64_t pos = 2 * cx.col_index(q);
-            const c32 gq = io<IO>::unpack(g[q]);
+            const c32 gq = EVEN ? io<IO>::unpack(gst[q * G::THREADS]) : load_pair<IO, false>(grow, pos, L);
             v[q] = mk(pos < L ? gq.x * v[q].x : 0.f, pos + 1 < L ? gq.y * v[q].y : 0.f);
         }
 #pragma unroll
