@@ -46,6 +46,54 @@ template <int DIR>
 __device__ __forceinline__ c32 rot90(c32 a) {
     return DIR > 0 ? c32{-a.y, a.x} : c32{a.y, -a.x};
 }
+// a + rot90(b) and a - rot90(b)
+template <int DIR>
+__device__ __forceinline__ c32 add_rot(c32 a, c32 b) { return add(a, rot90<DIR>(b)); }
+template <int DIR>
+__device__ __forceinline__ c32 sub_rot(c32 a, c32 b) { return sub(a, rot90<DIR>(b)); }
+
+// Two complex values of two independent rows carried in lockstep: re = (row a,
+// row b) real parts, im = imaginary parts. Every operation is one packed
+// fp32x2 instruction per component, so two rows cost the instructions of one.
+struct c32x2 {
+    float2 re, im;
+};
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.f, -1.f), a); }
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ c32x2 add(c32x2 a, c32x2 b) { return c32x2{f2add(a.re, b.re), f2add(a.im, b.im)}; }
+__device__ __forceinline__ c32x2 sub(c32x2 a, c32x2 b) { return c32x2{f2sub(a.re, b.re), f2sub(a.im, b.im)}; }
+// both lanes times the same complex scalar w
+__device__ __forceinline__ c32x2 mul(c32x2 a, c32 w) {
+    return c32x2{f2fma(a.im, f2(-w.y, -w.y), f2mul(a.re, f2(w.x, w.x))),
+                 f2fma(a.im, f2(w.x, w.x), f2mul(a.re, f2(w.y, w.y)))};
+}
+// lane-wise product of two pairs
+__device__ __forceinline__ c32x2 mul(c32x2 a, c32x2 b) {
+    return c32x2{f2fma(f2(-a.im.x, -a.im.y), b.im, f2mul(a.re, b.re)), f2fma(a.im, b.re, f2mul(a.re, b.im))};
+}
+// a complex scalar as the value type V (both lanes equal for pairs)
+template <typename V>
+__device__ __forceinline__ V bcast(c32 w);
+template <>
+__device__ __forceinline__ c32 bcast<c32>(c32 w) { return w; }
+template <>
+__device__ __forceinline__ c32x2 bcast<c32x2>(c32 w) { return c32x2{f2(w.x, w.x), f2(w.y, w.y)}; }
+
+template <int DIR>
+__device__ __forceinline__ c32x2 rot90(c32x2 a) {
+    return DIR > 0 ? c32x2{f2mul(a.im, f2(-1.f, -1.f)), a.re} : c32x2{a.im, f2mul(a.re, f2(-1.f, -1.f))};
+}
+template <int DIR>
+__device__ __forceinline__ c32x2 add_rot(c32x2 a, c32x2 b) {   // a + (DIR i) b
+    return DIR > 0 ? c32x2{f2sub(a.re, b.im), f2add(a.im, b.re)} : c32x2{f2add(a.re, b.im), f2sub(a.im, b.re)};
+}
+template <int DIR>
+__device__ __forceinline__ c32x2 sub_rot(c32x2 a, c32x2 b) {   // a - (DIR i) b
+    return DIR > 0 ? c32x2{f2add(a.re, b.im), f2sub(a.im, b.re)} : c32x2{f2sub(a.re, b.im), f2add(a.im, b.re)};
+}
 
 // W_64^m = exp(-2 pi i m / 64), m = 0..63 (cos and sin of m pi / 32, rounded to
 // float). Indexed with compile-time offsets, they become constant-bank operands.
@@ -137,8 +185,8 @@ __device__ __forceinline__ c32 w2e(int q, int z) {
 #define HY_R2 0.70710678118654752440f  // sqrt(1/2)
 
 // W_16^m = exp(DIR * 2 pi i m / 16) for the m that a 4x4 split needs.
-template <int DIR, int m>
-__device__ __forceinline__ c32 tw16(c32 a) {
+template <int DIR, int m, typename V>
+__device__ __forceinline__ V tw16(V a) {
     constexpr float s = (float)DIR;
     if constexpr (m == 0) return a;
     else if constexpr (m == 1) return mul(a, c32{HY_C1, s * HY_S1});
@@ -150,8 +198,8 @@ __device__ __forceinline__ c32 tw16(c32 a) {
     else return a;  // not reached
 }
 
-template <int DIR, int m>
-__device__ __forceinline__ c32 tw8(c32 a) {
+template <int DIR, int m, typename V>
+__device__ __forceinline__ V tw8(V a) {
     constexpr float s = (float)DIR;
     if constexpr (m == 0) return a;
     else if constexpr (m == 1) return mul(a, c32{HY_R2, s * HY_R2});
@@ -160,37 +208,37 @@ __device__ __forceinline__ c32 tw8(c32 a) {
 }
 
 // In-place 4-point DFT, X[k] = sum_n a[n] W_4^{nk}, W_4 = exp(DIR 2 pi i / 4).
-template <int DIR>
-__device__ __forceinline__ void dft4(c32 &a0, c32 &a1, c32 &a2, c32 &a3) {
-    c32 s02 = add(a0, a2), d02 = sub(a0, a2);
-    c32 s13 = add(a1, a3), d13 = rot90<DIR>(sub(a1, a3));
+template <int DIR, typename V>
+__device__ __forceinline__ void dft4(V &a0, V &a1, V &a2, V &a3) {
+    V s02 = add(a0, a2), d02 = sub(a0, a2);
+    V s13 = add(a1, a3), d13 = sub(a1, a3);
     a0 = add(s02, s13);
     a2 = sub(s02, s13);
-    a1 = add(d02, d13);
-    a3 = sub(d02, d13);
+    a1 = add_rot<DIR>(d02, d13);
+    a3 = sub_rot<DIR>(d02, d13);
 }
 
 // 4-point DFT of (a0, a1, 0, 0).
-template <int DIR>
-__device__ __forceinline__ void dft4_half(c32 &a0, c32 &a1, c32 &a2, c32 &a3) {
-    c32 j1 = rot90<DIR>(a1);
+template <int DIR, typename V>
+__device__ __forceinline__ void dft4_half(V &a0, V &a1, V &a2, V &a3) {
     a2 = sub(a0, a1);
-    a3 = sub(a0, j1);
-    c32 t = a0;
+    a3 = sub_rot<DIR>(a0, a1);
+    V t = a0;
     a0 = add(t, a1);
-    a1 = add(t, j1);
+    a1 = add_rot<DIR>(t, a1);
 }
 
-__device__ __forceinline__ void dft2(c32 &a0, c32 &a1) {
-    c32 t = a0;
+template <typename V>
+__device__ __forceinline__ void dft2(V &a0, V &a1) {
+    V t = a0;
     a0 = add(t, a1);
     a1 = sub(t, a1);
 }
 
 // 16-point DFT on x[o + st*n], n = 0..15, result in natural order at the same
 // positions. Split n = 4 n1 + n2, k = k1 + 4 k2. HALF: inputs n >= 8 are zero.
-template <int DIR, bool HALF, int st, int o, int NR>
-__device__ __forceinline__ void dft16(c32 (&x)[NR]) {
+template <int DIR, bool HALF, int st, int o, typename V, int NR>
+__device__ __forceinline__ void dft16(V (&x)[NR]) {
 #define X(i) x[o + st * (i)]
     // DFT4 over n1 for each n2; result A[n2][k1] kept at position 4*k1 + n2
     if constexpr (HALF) {
@@ -220,7 +268,7 @@ __device__ __forceinline__ void dft16(c32 (&x)[NR]) {
     dft4<DIR>(X(8), X(9), X(10), X(11));
     dft4<DIR>(X(12), X(13), X(14), X(15));
     // transpose 4x4 back to natural order
-    c32 t;
+    V t;
     t = X(1); X(1) = X(4); X(4) = t;
     t = X(2); X(2) = X(8); X(8) = t;
     t = X(3); X(3) = X(12); X(12) = t;
@@ -231,8 +279,8 @@ __device__ __forceinline__ void dft16(c32 (&x)[NR]) {
 }
 
 // 8-point DFT on x[o + st*n], n = 0..7 (split n = 2 n1 + n2, k = k1 + 4 k2).
-template <int DIR, int st, int o, int NR>
-__device__ __forceinline__ void dft8(c32 (&x)[NR]) {
+template <int DIR, int st, int o, typename V, int NR>
+__device__ __forceinline__ void dft8(V (&x)[NR]) {
 #define X(i) x[o + st * (i)]
     dft4<DIR>(X(0), X(2), X(4), X(6));   // n2 = 0 -> A[0][k1] at 2*k1
     dft4<DIR>(X(1), X(3), X(5), X(7));   // n2 = 1 -> A[1][k1] at 2*k1 + 1
@@ -243,24 +291,24 @@ __device__ __forceinline__ void dft8(c32 (&x)[NR]) {
     dft2(X(2), X(3));
     dft2(X(4), X(5));
     dft2(X(6), X(7));
-    c32 t;                               // positions 2k1+k2 -> k1+4k2
+    V t;                                 // positions 2k1+k2 -> k1+4k2
     t = X(1); X(1) = X(2); X(2) = X(4); X(4) = t;
     t = X(3); X(3) = X(6); X(6) = X(5); X(5) = t;
 #undef X
 }
 
-template <int DIR, int st, int o, int NR>
-__device__ __forceinline__ void dft4r(c32 (&x)[NR]) {
+template <int DIR, int st, int o, typename V, int NR>
+__device__ __forceinline__ void dft4r(V (&x)[NR]) {
     dft4<DIR>(x[o], x[o + st], x[o + 2 * st], x[o + 3 * st]);
 }
 
-template <int DIR, int st, int o, int NR>
-__device__ __forceinline__ void dft2r(c32 (&x)[NR]) {
+template <int DIR, int st, int o, typename V, int NR>
+__device__ __forceinline__ void dft2r(V (&x)[NR]) {
     dft2(x[o], x[o + st]);
 }
 
-template <int R, int DIR, bool HALF, int st, int o, int NR>
-__device__ __forceinline__ void dftR(c32 (&x)[NR]) {
+template <int R, int DIR, bool HALF, int st, int o, typename V, int NR>
+__device__ __forceinline__ void dftR(V (&x)[NR]) {
     if constexpr (R == 16) dft16<DIR, HALF, st, o>(x);
     else if constexpr (R == 8) dft8<DIR, st, o>(x);
     else if constexpr (R == 4) dft4r<DIR, st, o>(x);
@@ -271,20 +319,21 @@ __device__ __forceinline__ void dftR(c32 (&x)[NR]) {
 // products p_i = w^i, w^(i+4), w^(i+8), w^(i+12) (each power at most four
 // multiplications from w), applied as they are formed so that few powers are
 // live at once.
-template <int R, int st, int o, int NR>
-__device__ __forceinline__ void twiddle_powers(c32 (&x)[NR], c32 w1) {
+template <int R, int st, int o, typename V, int NR>
+__device__ __forceinline__ void twiddle_powers(V (&x)[NR], c32 w) {
+    const V w1 = bcast<V>(w);
     if constexpr (R == 2) {
         x[o + st] = mul(x[o + st], w1);
     } else {
-        c32 p1 = w1;
-        c32 p2 = mul(w1, w1);
-        c32 p3 = mul(p2, w1);
+        V p1 = w1;
+        V p2 = mul(w1, w1);
+        V p3 = mul(p2, w1);
         x[o + st] = mul(x[o + st], p1);
         x[o + 2 * st] = mul(x[o + 2 * st], p2);
         x[o + 3 * st] = mul(x[o + 3 * st], p3);
         if constexpr (R >= 8) {
-            const c32 w4 = mul(p2, p2);
-            c32 p0 = w4;
+            const V w4 = mul(p2, p2);
+            V p0 = w4;
 #pragma unroll
             for (int g = 1; g < R / 4; ++g) {
                 x[o + (4 * g) * st] = mul(x[o + (4 * g) * st], p0);

@@ -255,9 +255,13 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     a.B = batch;
     a.order = plan->order;
     const bool even = (plan->L % 2) == 0;
-    cudaError_t e = plan->path == HYENA_PATH_CTA
-                        ? launch_fwd_1d(a, plan->MC, plan->dtype, even, (cudaStream_t)stream)
-                        : launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
+    cudaError_t e;
+    if (plan->path == HYENA_PATH_CLUSTER)
+        e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
+    else if (pair_path_supported(plan->MC, batch))
+        e = launch_fwd_1d_pair(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
+    else
+        e = launch_fwd_1d(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 

@@ -1,0 +1,206 @@
+// 1D fused order-N forward for two rows of one channel per thread group.
+//
+// Rows (b, d) and (b+1, d) share the filter, the feedthrough and every
+// twiddle, so one thread group carries both in lockstep as packed fp32x2
+// values (c32x2): every butterfly add, every multiply and every shared-memory
+// access is one instruction for the two rows, and the spectrum row is staged
+// once for both. The algorithm is the one of hyena_fwd_1d_cta (real-input
+// packing into a half-length complex FFT, radix-16 Stockham passes, spectral
+// step with the feedthrough as a constant gain, inverse, gate), applied lane
+// by lane.
+#pragma once
+#include "kernels_1d.cuh"
+
+namespace hyena {
+
+// Swizzle of the pair exchange buffer (8-byte words): within every half-warp
+// the 16 lanes hit 16 distinct 8-byte bank pairs for the consecutive reads and
+// for the Stockham write patterns of every pass (checked on the CPU for
+// MC = 256..8192). It only permutes within aligned blocks of 16 words.
+__device__ __forceinline__ int swz2(int i) { return i ^ ((i >> 4) & 15); }
+
+template <int LEN, int E, int DIR, bool HALF_IN, int p>
+__device__ __forceinline__ void fft_pass_x2(c32x2 (&v)[E], float2 *__restrict__ sre, float2 *__restrict__ sim, int t,
+                                            const c32 *__restrict__ tw) {
+    constexpr int T = LEN / E;
+    constexpr int P = num_passes(LEN);
+    constexpr int R = pass_radix(LEN, p);
+    constexpr int NS = pass_stride(LEN, p);
+    constexpr int S = E / R;
+    constexpr bool LAST = (p == P - 1);
+    constexpr int TWM = 2 * LEN;
+    if constexpr (p > 0) {
+        __syncthreads();  // writes of pass p-1 visible
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const int i = swz2(t + q * T);
+            v[q] = c32x2{sre[i], sim[i]};
+        }
+        __syncthreads();  // every read done before pass p writes
+    }
+    static_for<S>([&](auto sc) {
+        constexpr int s = decltype(sc)::value;
+        const int j = t + s * T;
+        const int k = j & (NS - 1);
+        (void)k;
+        if constexpr (NS > 1) {
+            const float2 wf = __ldg(reinterpret_cast<const float2 *>(tw) + (size_t)k * (TWM / (NS * R)));
+            twiddle_powers<R, S, s>(v, DIR > 0 ? mk(wf.x, -wf.y) : mk(wf.x, wf.y));
+        }
+        dftR<R, DIR, HALF_IN && p == 0, S, s>(v);
+        if constexpr (!LAST) {
+            const int base = (j / NS) * NS * R + k;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int i = swz2(base + r * NS);
+                sre[i] = v[s + r * S].re;
+                sim[i] = v[s + r * S].im;
+            }
+        }
+    });
+    if constexpr (!LAST) fft_pass_x2<LEN, E, DIR, false, p + 1>(v, sre, sim, t, tw);
+}
+
+// Length-LEN FFT of two rows in lockstep (natural order in and out; the
+// table is W_{2 LEN}, the plan's table for M = 2 LEN).
+template <int LEN, int E, int DIR, bool HALF_IN>
+__device__ __forceinline__ void fft_cta_x2(c32x2 (&v)[E], float2 *sre, float2 *sim, int t,
+                                           const c32 *__restrict__ tw) {
+    fft_pass_x2<LEN, E, DIR, HALF_IN, 0>(v, sre, sim, t, tw);
+}
+
+// Spectral step for both rows (see spectral_product in kernels_1d.cuh). The
+// unpacking is written without its factors 1/2; those and the 1/MC of the
+// inverse are folded into the (shared) filter gain.
+template <int MC, int E>
+__device__ __forceinline__ void spectral_product_x2(c32x2 (&v)[E], float2 *__restrict__ sre,
+                                                    float2 *__restrict__ sim, int t, const c32 *Hs, float dsk,
+                                                    c32 wt) {
+    constexpr int T = MC / E;
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        sre[t + q * T] = v[q].re;
+        sim[t + q * T] = v[q].im;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    constexpr float s = 0.25f / (float)MC;
+    const int z0 = opaque_zero();
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int k = t + q * T;
+        const int km = (MC - k) & (MC - 1);
+        const c32x2 Zk = v[q];
+        const float2 mre = sre[km], mim = sim[km];
+        // 2E = Zk + conj Zm, 2O = (Zk - conj Zm) / i
+        const c32x2 E2{f2add(Zk.re, mre), f2sub(Zk.im, mim)};
+        const c32x2 O2{f2add(Zk.im, mim), f2sub(mre, Zk.re)};
+        const c32 w = mul(wt, w2e<E>(q, z0));          // W_M^{t + qT}
+        const c32x2 wO = mul(O2, w);
+        const c32x2 Xk = add(E2, wO);                   // 2 X[k]
+        const c32x2 Xm{f2sub(E2.re, wO.re), f2sub(wO.im, E2.im)};   // 2 X[MC-k] = conj(2E - 2wO)
+        c32 Hk = Hs[k], Hm = Hs[MC - k];
+        Hk = mk(s * (Hk.x + dsk), s * Hk.y);
+        Hm = mk(s * (Hm.x + dsk), s * Hm.y);
+        const c32x2 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
+        const c32x2 Ye{f2add(Yk.re, Ym.re), f2sub(Yk.im, Ym.im)};   // Yk + conj Ym
+        const c32x2 Yd{f2sub(Yk.re, Ym.re), f2add(Yk.im, Ym.im)};   // Yk - conj Ym
+        const c32x2 Yo = mul(Yd, conj(w));
+        v[q] = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};   // Ye + i Yo
+    }
+    __syncthreads();
+}
+
+constexpr int pair_pairs_per_cta(int MC, int E) { return (MC / E) >= 128 ? 1 : 128 / (MC / E); }
+constexpr int pair_threads(int MC, int E) { return pair_pairs_per_cta(MC, E) * (MC / E); }
+constexpr int pair_min_blocks(int MC, int E) {
+    return pair_threads(MC, E) >= 512 ? 1 : (pair_threads(MC, E) >= 256 ? 1 : 3);
+}
+// Shared bytes per row pair: exchange buffer (two float2 planes) + staged spectrum row.
+constexpr size_t pair_smem_bytes_per_pair(int MC) { return (size_t)MC * 16 + (size_t)(MC + 1) * 8; }
+
+// Fused order-N forward, one group of MC/E threads per pair of rows
+// (b, d), (b+1, d); B must be even. Pairs are visited d-major so the B/2
+// pairs that read the same spectrum row run together.
+template <int MC, int E, typename IO, bool EVEN>
+__global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
+    hyena_fwd_1d_pair(const Fwd1dArgs a) {
+    constexpr int T = MC / E;
+    constexpr int PPC = pair_pairs_per_cta(MC, E);
+    extern __shared__ float4 smem4[];
+    const int lp = threadIdx.x / T;
+    const int t = threadIdx.x - lp * T;
+    const int64_t npairs = a.rows / 2;
+    const int64_t pidx = (int64_t)blockIdx.x * PPC + lp;
+    const bool active = pidx < npairs;
+    const int64_t hb = a.B / 2;
+    const int64_t d = active ? pidx / hb : 0;
+    const int64_t b0 = active ? 2 * (pidx - d * hb) : 0;
+    const int64_t row0 = b0 * a.D + d, row1 = row0 + a.D;
+    unsigned char *base = reinterpret_cast<unsigned char *>(smem4) + lp * pair_smem_bytes_per_pair(MC);
+    float2 *sre = reinterpret_cast<float2 *>(base);
+    float2 *sim = sre + MC;
+    c32 *Hs = reinterpret_cast<c32 *>(sim + MC);
+    const int64_t L = a.L;
+    const c32 wt = ldg_c(a.tw + t);                       // W_M^t
+
+    c32x2 v[E];
+    {
+        const IO *r0 = reinterpret_cast<const IO *>(a.v) + row0 * L;
+        const IO *r1 = reinterpret_cast<const IO *>(a.v) + row1 * L;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = 2 * (int64_t)(t + q * T);
+            const c32 x0 = active ? load_pair<IO, EVEN>(r0, pos, L) : mk(0.f, 0.f);
+            const c32 x1 = active ? load_pair<IO, EVEN>(r1, pos, L) : mk(0.f, 0.f);
+            v[q] = c32x2{f2(x0.x, x1.x), f2(x0.y, x1.y)};
+        }
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
+    }
+
+    for (int n = 0; n < a.order; ++n) {
+        const IO *g0 = reinterpret_cast<const IO *>(a.gates[n]) + row0 * L;
+        const IO *g1 = reinterpret_cast<const IO *>(a.gates[n]) + row1 * L;
+        typename io<IO>::pair_t ga[E / 2], gb[E / 2];
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = 2 * (int64_t)(t + q * T);
+            ga[q] = active ? load_pair_raw<IO, EVEN>(g0, pos, L) : io<IO>::zero();
+            gb[q] = active ? load_pair_raw<IO, EVEN>(g1, pos, L) : io<IO>::zero();
+        }
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);   // staged while the FFT runs
+        cp_async_commit();
+
+        fft_cta_x2<MC, E, -1, true>(v, sre, sim, t, a.tw);
+        spectral_product_x2<MC, E>(v, sre, sim, t, Hs, dsk, wt);
+        fft_cta_x2<MC, E, +1, false>(v, sre, sim, t, a.tw);
+
+        // gate; positions >= L are cleared so the next order sees a zero-padded row
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = 2 * (int64_t)(t + q * T);
+            const c32 ca = io<IO>::unpack(ga[q]), cb = io<IO>::unpack(gb[q]);
+            const bool in0 = pos < L, in1 = pos + 1 < L;
+            v[q] = c32x2{in0 ? f2mul(v[q].re, f2(ca.x, cb.x)) : f2(0.f, 0.f),
+                         in1 ? f2mul(v[q].im, f2(ca.y, cb.y)) : f2(0.f, 0.f)};
+        }
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
+    }
+
+    if (active) {
+        IO *y0 = reinterpret_cast<IO *>(a.y) + row0 * L;
+        IO *y1 = reinterpret_cast<IO *>(a.y) + row1 * L;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = 2 * (int64_t)(t + q * T);
+            store_pair<IO, EVEN>(y0, pos, L, mk(v[q].re.x, v[q].im.x));
+            store_pair<IO, EVEN>(y1, pos, L, mk(v[q].re.y, v[q].im.y));
+        }
+    }
+}
+
+}  // namespace hyena
