@@ -121,7 +121,12 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
     }
     if (cudaGetDevice(&p.device) != cudaSuccess) return HYENA_ERR_CUDA;
 
+    // main table W_tw_len, followed by W_1024 for the short sub-transforms of the cluster paths
     std::vector<float2> tw = twiddle_table(p.tw_len);
+    {
+        std::vector<float2> sub = twiddle_table(HYENA_SUB_TWIDDLES);
+        tw.insert(tw.end(), sub.begin(), sub.end());
+    }
     if (cudaMalloc(&p.tw, sizeof(float2) * tw.size()) != cudaSuccess) {
         cudaGetLastError();
         return HYENA_ERR_NOMEM;

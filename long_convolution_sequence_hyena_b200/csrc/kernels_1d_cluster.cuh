@@ -96,7 +96,10 @@ __device__ __forceinline__ void slot_of_row(int k1, int &c, int &r) {
 template <typename G, bool TWID, bool HALFX>
 struct ClusterCtx {
     // Twiddle table length: 1D, W_M with M = 2 MC; 2D, W_{2 M2} with 2 M2 >= M1.
+    // The plan appends W_1024 to it for the sub-transforms (kept L1-resident).
     static constexpr int TWM = TWID ? 2 * G::MC : (2 * G::M2 >= G::M1 ? 2 * G::M2 : G::M1);
+    static constexpr int TWS = 1024;
+    static_assert(TWS % G::M1 == 0 && TWS % G::M2 == 0, "sub-transform twiddles");
     float *col_re, *col_im, *row_re, *row_im;
     int crank;
     int j, t1, n2;   // column phase: local column, FFT lane, global column
@@ -137,7 +140,7 @@ struct ClusterCtx {
     __device__ __forceinline__ void forward(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
         if (col_live) {
-            fft_cta<G::M1, E, -1, HALF_COL, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
+            fft_cta<G::M1, E, -1, HALF_COL, TWS, G::NCOL>(v, col_re, col_im, t1, tw + TWM, j);
             if constexpr (TWID) {
                 constexpr int M = 2 * G::MC;
                 const c32 b = ldg_c(tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
@@ -167,7 +170,7 @@ struct ClusterCtx {
             }
         }
         __syncthreads();
-        fft_cta<G::M2, E, -1, HALFX, TWM, G::NROW>(v, row_re, row_im, t2, tw, r);
+        fft_cta<G::M2, E, -1, HALFX, TWS, G::NROW>(v, row_re, row_im, t2, tw + TWM, r);
     }
 
     // Store the row-layout bins so the mirror bins can be read (ends with a CTA barrier).
@@ -190,7 +193,7 @@ struct ClusterCtx {
     // Must follow a CTA barrier after the last read of the published bins.
     __device__ __forceinline__ void inverse(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
-        fft_cta<G::M2, E, +1, false, TWM, G::NROW>(v, row_re, row_im, t2, tw, r);
+        fft_cta<G::M2, E, +1, false, TWS, G::NROW>(v, row_re, row_im, t2, tw + TWM, r);
         if constexpr (TWID) {
             constexpr int M = 2 * G::MC;
             const c32 b = conj(ldg_c(tw + ((2 * (int64_t)t2 * k1) & (M - 1))));
@@ -214,7 +217,7 @@ struct ClusterCtx {
                 v[q] = mk(col_re[ad], col_im[ad]);
             }
             __syncthreads();
-            fft_cta<G::M1, E, +1, false, TWM, G::NCOL>(v, col_re, col_im, t1, tw, j);
+            fft_cta<G::M1, E, +1, false, TWS, G::NCOL>(v, col_re, col_im, t1, tw + TWM, j);
         }
     }
 };

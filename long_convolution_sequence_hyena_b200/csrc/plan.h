@@ -7,6 +7,7 @@
 
 #define HYENA_MAX_L_1D 131072    // longest 1D sequence (M = 262144)
 #define HYENA_MAX_M_CTA 32768    // longest padded length the single-CTA path runs
+#define HYENA_SUB_TWIDDLES 1024  // W_1024 table appended to the main one (cluster sub-transforms)
 
 struct hyena_plan_s {
     int ndim = 1;
@@ -24,5 +25,5 @@ struct hyena_plan_s {
     int64_t spectrum_elems = 0;  // complex bins per (order, channel)
     // device tables (owned)
     int64_t tw_len = 0;          // 1D: M; 2D: 2W
-    float2 *tw = nullptr;        // W_tw_len^m, m in [0, tw_len)
+    float2 *tw = nullptr;        // W_tw_len^m, m in [0, tw_len), then W_1024^m, m in [0, 1024)
 };
