@@ -10,7 +10,7 @@ cudaError_t launch_fwd_1d_pair_t(const Fwd1dArgs &a, cudaStream_t st) {
     constexpr int E = 16;
     constexpr int PPC = pair_pairs_per_cta(MC, E);
     auto kern = hyena_fwd_1d_pair<MC, E, IO, EVEN>;
-    const size_t sm = (size_t)PPC * pair_smem_bytes_per_pair(MC);
+    const size_t sm = pair_smem_bytes<IO, EVEN>(MC, E);
     if (sm > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
@@ -29,7 +29,7 @@ cudaError_t launch_fwd_1d_pair_mc(const Fwd1dArgs &a, hyena_dtype_t dt, bool eve
                 : launch_fwd_1d_pair_t<MC, __nv_bfloat16, false>(a, st);
 }
 
-bool pair_path_supported(int64_t MC, int64_t B) { return B % 2 == 0 && MC >= 16 && MC <= 2048; }
+bool pair_path_supported(int64_t MC, int64_t B) { return B % 2 == 0 && MC >= 16 && MC <= 8192; }
 
 cudaError_t launch_fwd_1d_pair(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
     switch (MC) {
@@ -41,6 +41,8 @@ cudaError_t launch_fwd_1d_pair(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt,
         case 512: return launch_fwd_1d_pair_mc<512>(a, dt, even, st);
         case 1024: return launch_fwd_1d_pair_mc<1024>(a, dt, even, st);
         case 2048: return launch_fwd_1d_pair_mc<2048>(a, dt, even, st);
+        case 4096: return launch_fwd_1d_pair_mc<4096>(a, dt, even, st);
+        case 8192: return launch_fwd_1d_pair_mc<8192>(a, dt, even, st);
         default: return cudaErrorInvalidValue;
     }
 }

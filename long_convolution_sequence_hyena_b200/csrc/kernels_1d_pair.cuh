@@ -113,11 +113,33 @@ __device__ __forceinline__ void spectral_product_x2(c32x2 (&v)[E], float2 *__res
 
 constexpr int pair_pairs_per_cta(int MC, int E) { return (MC / E) >= 128 ? 1 : 128 / (MC / E); }
 constexpr int pair_threads(int MC, int E) { return pair_pairs_per_cta(MC, E) * (MC / E); }
+// Resident CTAs per SM the register budget is sized for (128 threads: 3 -> 168
+// registers; 256 threads: 2 -> 128; 512 threads: 1 -> 128).
+#ifndef HYENA_PAIR_MINB_128
+#define HYENA_PAIR_MINB_128 3
+#endif
 constexpr int pair_min_blocks(int MC, int E) {
-    return pair_threads(MC, E) >= 512 ? 1 : (pair_threads(MC, E) >= 256 ? 1 : 3);
+    return pair_threads(MC, E) >= 512 ? 1 : (pair_threads(MC, E) >= 256 ? 2 : HYENA_PAIR_MINB_128);
 }
 // Shared bytes per row pair: exchange buffer (two float2 planes) + staged spectrum row.
 constexpr size_t pair_smem_bytes_per_pair(int MC) { return (size_t)MC * 16 + (size_t)(MC + 1) * 8; }
+// Staging for one order's gates of both rows (E/2 element pairs per row and thread).
+template <typename IO>
+constexpr size_t pair_gate_stage_bytes(int MC, int E) {
+    return (size_t)pair_threads(MC, E) * E * sizeof(typename io<IO>::pair_t);
+}
+// Gates are staged in shared memory (freeing registers) when the row length
+// is even and the stage fits next to the buffers.
+template <typename IO, bool EVEN>
+constexpr bool pair_stage_gates(int MC, int E) {
+    return EVEN && pair_pairs_per_cta(MC, E) * pair_smem_bytes_per_pair(MC) + pair_gate_stage_bytes<IO>(MC, E) <=
+                       227 * 1024;
+}
+template <typename IO, bool EVEN>
+constexpr size_t pair_smem_bytes(int MC, int E) {
+    return pair_pairs_per_cta(MC, E) * pair_smem_bytes_per_pair(MC) +
+           (pair_stage_gates<IO, EVEN>(MC, E) ? pair_gate_stage_bytes<IO>(MC, E) : 0);
+}
 
 // Fused order-N forward, one group of MC/E threads per pair of rows
 // (b, d), (b+1, d); B must be even. Pairs are visited d-major so the B/2
@@ -159,15 +181,34 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
         for (int q = E / 2; q < E; ++q) v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
     }
 
+    using P = typename io<IO>::pair_t;
+    constexpr bool GST = pair_stage_gates<IO, EVEN>(MC, E);
+    constexpr int NT = pair_threads(MC, E);
+    P *gst = reinterpret_cast<P *>(reinterpret_cast<unsigned char *>(smem4) + PPC * pair_smem_bytes_per_pair(MC)) +
+             threadIdx.x;   // thread-private slots gst[(2 q + row) * NT]
     for (int n = 0; n < a.order; ++n) {
         const IO *g0 = reinterpret_cast<const IO *>(a.gates[n]) + row0 * L;
         const IO *g1 = reinterpret_cast<const IO *>(a.gates[n]) + row1 * L;
-        typename io<IO>::pair_t ga[E / 2], gb[E / 2];
+        P ga[GST ? 1 : E / 2], gb[GST ? 1 : E / 2];
+        if constexpr (GST) {   // staged while the transforms run
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) {
-            const int64_t pos = 2 * (int64_t)(t + q * T);
-            ga[q] = active ? load_pair_raw<IO, EVEN>(g0, pos, L) : io<IO>::zero();
-            gb[q] = active ? load_pair_raw<IO, EVEN>(g1, pos, L) : io<IO>::zero();
+            for (int q = 0; q < E / 2; ++q) {
+                const int64_t pos = 2 * (int64_t)(t + q * T);
+                if (active && pos < L) {
+                    cp_async_n<sizeof(P)>(gst + (2 * q) * NT, g0 + pos);
+                    cp_async_n<sizeof(P)>(gst + (2 * q + 1) * NT, g1 + pos);
+                } else {
+                    gst[(2 * q) * NT] = io<IO>::zero();
+                    gst[(2 * q + 1) * NT] = io<IO>::zero();
+                }
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < E / 2; ++q) {
+                const int64_t pos = 2 * (int64_t)(t + q * T);
+                ga[q] = active ? load_pair_raw<IO, EVEN>(g0, pos, L) : io<IO>::zero();
+                gb[q] = active ? load_pair_raw<IO, EVEN>(g1, pos, L) : io<IO>::zero();
+            }
         }
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
         const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
@@ -182,7 +223,8 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
             const int64_t pos = 2 * (int64_t)(t + q * T);
-            const c32 ca = io<IO>::unpack(ga[q]), cb = io<IO>::unpack(gb[q]);
+            const c32 ca = io<IO>::unpack(GST ? gst[(2 * q) * NT] : ga[q]);
+            const c32 cb = io<IO>::unpack(GST ? gst[(2 * q + 1) * NT] : gb[q]);
             const bool in0 = pos < L, in1 = pos + 1 < L;
             v[q] = c32x2{in0 ? f2mul(v[q].re, f2(ca.x, cb.x)) : f2(0.f, 0.f),
                          in1 ? f2mul(v[q].im, f2(ca.y, cb.y)) : f2(0.f, 0.f)};
