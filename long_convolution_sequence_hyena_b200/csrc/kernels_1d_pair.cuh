@@ -122,7 +122,9 @@ constexpr int pair_min_blocks(int MC, int E) {
     return pair_threads(MC, E) >= 512 ? 1 : (pair_threads(MC, E) >= 256 ? 2 : HYENA_PAIR_MINB_128);
 }
 // Shared bytes per row pair: exchange buffer (two float2 planes) + staged spectrum row.
-constexpr size_t pair_smem_bytes_per_pair(int MC) { return (size_t)MC * 16 + (size_t)(MC + 1) * 8; }
+// (rounded up to 16 bytes so every pair's region, and the gate stage after
+// them, start 16-byte aligned)
+constexpr size_t pair_smem_bytes_per_pair(int MC) { return ((size_t)MC * 16 + (size_t)(MC + 1) * 8 + 15) & ~(size_t)15; }
 // Staging for one order's gates of both rows (E/2 element pairs per row and thread).
 template <typename IO>
 constexpr size_t pair_gate_stage_bytes(int MC, int E) {
