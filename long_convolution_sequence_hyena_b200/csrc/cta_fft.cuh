@@ -4,11 +4,13 @@
 // Two shared-memory layouts:
 //  * NSEQ == 0: one sequence per buffer, contiguous; the Stockham write
 //    pattern is made bank-conflict-free by swz<NS>() (see fft_regs.cuh).
-//  * NSEQ  > 0: NSEQ sequences, sequence-major, element i of sequence s at
-//    s * LEN + (i ^ (s & 31)). Warps span the sequence index with a common i,
-//    so the XOR puts the lanes on distinct banks; and lanes that span 32
-//    consecutive i of one sequence touch one contiguous 128-byte block (what
-//    a remote, distributed-shared-memory store wants).
+//  * NSEQ  > 0: NSEQ sequences, sequence-major, interleaved complex (one
+//    8-byte float2 per element, in the buffer passed as `sre`; `sim` is
+//    unused), element i of sequence s at s * LEN + (i ^ (s & 31)). Warps span
+//    the sequence index with a common i, so the XOR puts each half-warp on
+//    distinct 8-byte bank pairs; and lanes that span 32 consecutive i of one
+//    sequence touch one contiguous 256-byte block (what a remote,
+//    distributed-shared-memory store wants).
 //
 // Twiddles come from one table of W_TWM^m = exp(-2 pi i m / TWM), m < TWM,
 // with TWM a multiple of LEN.
@@ -56,7 +58,12 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int i = saddr<NSP, NSEQ, LEN>(t + q * T, seq);
-            v[q] = mk(sre[i], sim[i]);
+            if constexpr (NSEQ > 0) {
+                const float2 f = reinterpret_cast<const float2 *>(sre)[i];
+                v[q] = mk(f.x, f.y);
+            } else {
+                v[q] = mk(sre[i], sim[i]);
+            }
         }
         __syncthreads();  // every read done before pass p writes
     }
@@ -75,8 +82,12 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const int i = saddr<NS, NSEQ, LEN>(base + r * NS, seq);
-                sre[i] = v[s + r * S].x;
-                sim[i] = v[s + r * S].y;
+                if constexpr (NSEQ > 0) {
+                    reinterpret_cast<float2 *>(sre)[i] = make_float2(v[s + r * S].x, v[s + r * S].y);
+                } else {
+                    sre[i] = v[s + r * S].x;
+                    sim[i] = v[s + r * S].y;
+                }
             }
         }
     });

@@ -54,8 +54,8 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t local, int rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
     return remote;
 }
-__device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+__device__ __forceinline__ void dsmem_st2(uint32_t addr, c32 v) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
 }
 // Cluster barrier that also orders shared::cluster memory (release / acquire).
 __device__ __forceinline__ void cluster_sync_mem() {
@@ -100,7 +100,7 @@ struct ClusterCtx {
     static constexpr int TWM = TWID ? 2 * G::MC : (2 * G::M2 >= G::M1 ? 2 * G::M2 : G::M1);
     static constexpr int TWS = 1024;
     static_assert(TWS % G::M1 == 0 && TWS % G::M2 == 0, "sub-transform twiddles");
-    float *col_re, *col_im, *row_re, *row_im;
+    float2 *colb, *rowb;   // column and row buffers, interleaved complex, sequence-major
     int crank;
     int j, t1, n2;   // column phase: local column, FFT lane, global column
     int r, t2, k1;   // row phase: local slot, FFT lane, global row
@@ -109,10 +109,8 @@ struct ClusterCtx {
 
     __device__ __forceinline__ ClusterCtx(float *smem) {
         crank = (int)cg::this_cluster().block_rank();
-        col_re = smem;
-        col_im = col_re + G::PER_CTA;
-        row_re = col_im + G::PER_CTA;
-        row_im = row_re + G::PER_CTA;
+        colb = reinterpret_cast<float2 *>(smem);
+        rowb = colb + G::PER_CTA;
         const int tid = threadIdx.x;
         j = tid % G::NCOL;
         t1 = tid / G::NCOL;
@@ -140,7 +138,7 @@ struct ClusterCtx {
     __device__ __forceinline__ void forward(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
         if (col_live) {
-            fft_cta<G::M1, E, -1, HALF_COL, TWS, G::NCOL>(v, col_re, col_im, t1, tw + TWM, j);
+            fft_cta<G::M1, E, -1, HALF_COL, TWS, G::NCOL>(v, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
             if constexpr (TWID) {
                 constexpr int M = 2 * G::MC;
                 const c32 b = ldg_c(tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
@@ -153,9 +151,7 @@ struct ClusterCtx {
                 for (int q = 0; q < E; ++q) {
                     int dst, slot;
                     slot_of_row<G>(t1 + q * G::T1 + z, dst, slot);
-                    const uint32_t ad = dsmem_map(smem_u32(row_re + maddr<G::M2>(n2, slot)), dst);
-                    dsmem_st(ad, v[q].x);
-                    dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
+                    dsmem_st2(dsmem_map(smem_u32(rowb + maddr<G::M2>(n2, slot)), dst), v[q]);
                 }
             }
         }
@@ -166,11 +162,11 @@ struct ClusterCtx {
                 v[q] = mk(0.f, 0.f);
             } else {
                 const int ad = maddr<G::M2>(t2 + q * G::T2, r);
-                v[q] = mk(row_re[ad], row_im[ad]);
+                v[q] = mk(rowb[ad].x, rowb[ad].y);
             }
         }
         __syncthreads();
-        fft_cta<G::M2, E, -1, HALFX, TWS, G::NROW>(v, row_re, row_im, t2, tw + TWM, r);
+        fft_cta<G::M2, E, -1, HALFX, TWS, G::NROW>(v, reinterpret_cast<float *>(rowb), nullptr, t2, tw + TWM, r);
     }
 
     // Store the row-layout bins so the mirror bins can be read (ends with a CTA barrier).
@@ -178,22 +174,21 @@ struct ClusterCtx {
 #pragma unroll
         for (int q = 0; q < G::E; ++q) {
             const int ad = maddr<G::M2>(t2 + q * G::T2, r);
-            row_re[ad] = v[q].x;
-            row_im[ad] = v[q].y;
+            rowb[ad] = make_float2(v[q].x, v[q].y);
         }
         __syncthreads();
     }
     // Published bin (mirror row, column k2m) from this CTA's own buffer.
     __device__ __forceinline__ c32 mirror_bin(int k2m) const {
         const int ad = maddr<G::M2>(k2m, rm);
-        return mk(row_re[ad], row_im[ad]);
+        return mk(rowb[ad].x, rowb[ad].y);
     }
 
     // Row layout (bins) -> column layout (time domain, unscaled inverse).
     // Must follow a CTA barrier after the last read of the published bins.
     __device__ __forceinline__ void inverse(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
-        fft_cta<G::M2, E, +1, false, TWS, G::NROW>(v, row_re, row_im, t2, tw + TWM, r);
+        fft_cta<G::M2, E, +1, false, TWS, G::NROW>(v, reinterpret_cast<float *>(rowb), nullptr, t2, tw + TWM, r);
         if constexpr (TWID) {
             constexpr int M = 2 * G::MC;
             const c32 b = conj(ldg_c(tw + ((2 * (int64_t)t2 * k1) & (M - 1))));
@@ -205,19 +200,17 @@ struct ClusterCtx {
         for (int q = 0; q < E; ++q) {
             const int nn = t2 + q * G::T2 + z;
             if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
-            const uint32_t ad = dsmem_map(smem_u32(col_re + maddr<G::M1>(k1, nn % G::NCOL)), nn / G::NCOL);
-            dsmem_st(ad, v[q].x);
-            dsmem_st(ad + 4 * G::PER_CTA, v[q].y);
+            dsmem_st2(dsmem_map(smem_u32(colb + maddr<G::M1>(k1, nn % G::NCOL)), nn / G::NCOL), v[q]);
         }
         cluster_sync_mem();
         if (col_live) {
 #pragma unroll
             for (int q = 0; q < E; ++q) {
                 const int ad = maddr<G::M1>(t1 + q * G::T1, j);
-                v[q] = mk(col_re[ad], col_im[ad]);
+                v[q] = mk(colb[ad].x, colb[ad].y);
             }
             __syncthreads();
-            fft_cta<G::M1, E, +1, false, TWS, G::NCOL>(v, col_re, col_im, t1, tw + TWM, j);
+            fft_cta<G::M1, E, +1, false, TWS, G::NCOL>(v, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
         }
     }
 };
