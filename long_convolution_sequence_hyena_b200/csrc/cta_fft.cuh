@@ -46,14 +46,16 @@ template <int LEN, int E, int DIR, bool HALF_IN, int p, int TWM, int NSEQ>
 __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim, int t,
                                          int seq, const c32 *__restrict__ tw) {
     constexpr int T = LEN / E;
-    constexpr int P = num_passes(LEN);
-    constexpr int R = pass_radix(LEN, p);
-    constexpr int NS = pass_stride(LEN, p);
+    constexpr int LR = pass_lr(E);
+    constexpr int P = num_passes(LEN, LR);
+    constexpr int R = pass_radix(LEN, p, LR);
+    constexpr int NS = pass_stride(LEN, p, LR);
+    static_assert(NSEQ > 0 || LR == 4, "the contiguous swizzled layout assumes radix-16 passes");
     constexpr int S = E / R;
     constexpr bool LAST = (p == P - 1);
     static_assert(TWM % LEN == 0, "twiddle table must cover the transform");
     if constexpr (p > 0) {
-        constexpr int NSP = pass_stride(LEN, p - 1);
+        constexpr int NSP = pass_stride(LEN, p - 1, LR);
         __syncthreads();  // writes of pass p-1 visible
 #pragma unroll
         for (int q = 0; q < E; ++q) {

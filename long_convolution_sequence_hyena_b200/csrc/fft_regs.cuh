@@ -357,13 +357,15 @@ __device__ __forceinline__ int swz(int i) {
     else return i;
 }
 
-// Radix of pass p for an FFT of length Mc: radix-16 passes, then one radix
-// 2/4/8 pass for the remaining factor.
 constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
-constexpr int num_passes(int Mc) { return (ilog2(Mc) + 3) / 4; }
-constexpr int pass_radix(int Mc, int p) {
-    return (p < ilog2(Mc) / 4) ? 16 : (1 << (ilog2(Mc) % 4));
+// Pass plan with passes of radix 2^LR (LR = 4: radix 16, the default; LR = 3
+// when a thread holds only 8 values), then one pass for the remaining factor.
+constexpr int num_passes(int Mc, int LR = 4) { return (ilog2(Mc) + LR - 1) / LR; }
+constexpr int pass_radix(int Mc, int p, int LR = 4) {
+    return (p < ilog2(Mc) / LR) ? (1 << LR) : (1 << (ilog2(Mc) % LR));
 }
-constexpr int pass_stride(int Mc, int p) { return 1 << (4 * p); }  // Ns = 16^p
+constexpr int pass_stride(int Mc, int p, int LR = 4) { return 1 << (LR * p); }  // Ns = (2^LR)^p
+// log2 of the largest pass radix a thread holding E values can run
+constexpr int pass_lr(int E) { return E >= 16 ? 4 : ilog2(E); }
 
 }  // namespace hyena
