@@ -4,8 +4,8 @@
 
 namespace hyena {
 
-using G1_32K = ClusterGeom<32768, 4, 128, 16>;    // 1D, 32768 < M <= 65536
-using G1_64K = ClusterGeom<65536, 8, 256, 16>;    // 1D, M = 131072
+using G1_32K = ClusterGeom<32768, 8, 128, 16, 2>;    // 1D, 32768 < M <= 65536
+using G1_64K = ClusterGeom<65536, 16, 256, 16, 2>;   // 1D, M = 131072 (16-CTA cluster)
 using G1_128K = ClusterGeom<131072, 16, 512, 16>; // 1D, M = 262144 (16-CTA cluster)
 using G2_32 = ClusterGeom<2048, 1, 64, 16>;       // 2D, 32 x 32 grid (64 x 64 padded)
 using G2_64 = ClusterGeom<8192, 2, 128, 16>;      // 2D, 64 x 64

@@ -27,9 +27,11 @@ namespace hyena {
 
 namespace cg = cooperative_groups;
 
-template <int MC_, int C_, int M1_, int E_>
+// MINB: CTAs resident per SM (the launch bounds); with 2, one cluster's
+// barrier waits are covered by another cluster's work on the same SMs.
+template <int MC_, int C_, int M1_, int E_, int MINB_ = 1>
 struct ClusterGeom {
-    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_;
+    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_, MINB = MINB_;
     static constexpr int NCOL = M2 / C;          // columns per CTA (column phase)
     static constexpr int NROW = M1 / C;          // rows per CTA (row phase), in mirror pairs
     static constexpr int HROW = NROW / 2;        // rows k1 < M1/2 per CTA
@@ -45,6 +47,8 @@ struct ClusterGeom {
     static_assert(M1 >= 32 && M2 >= 32, "sequence-major layouts need sequences of at least 32");
     static_assert(THREADS <= 1024, "too many threads");
     static_assert(SMEM <= 200 * 1024, "buffers must fit in shared memory");
+    static_assert(MINB * (SMEM + 1024) <= 228 * 1024, "MINB CTAs must fit in one SM's shared memory");
+    static_assert(MINB * THREADS <= 2048, "MINB CTAs must fit in one SM's thread slots");
 };
 
 // Distributed shared memory through 32-bit shared::cluster addresses.
@@ -217,7 +221,7 @@ struct ClusterCtx {
 
 // Fused order-N forward, one cluster per row (rows visited d-major, b-minor).
 template <typename G, typename IO, bool EVEN>
-__global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1dArgs a) {
+__global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(const Fwd1dArgs a) {
     constexpr int MC = G::MC, E = G::E, M1 = G::M1;
     extern __shared__ float smem[];
     ClusterCtx<G, true, false> cx(smem);
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_1d_cluster(const Fwd1
 // In place (h == Hout) is allowed: every CTA reads its part of the row before
 // the first cluster barrier, and bins are written after it.
 template <typename G>
-__global__ void __launch_bounds__(G::THREADS, 1)
+__global__ void __launch_bounds__(G::THREADS, G::MINB)
     hyena_spectrum_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, const c32 *__restrict__ tw) {
     constexpr int MC = G::MC, E = G::E, M1 = G::M1;
     extern __shared__ float smem[];

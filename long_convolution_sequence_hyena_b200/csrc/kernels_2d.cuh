@@ -33,7 +33,7 @@ struct Fwd2dArgs {
 
 // Fused order-N 2D forward (planes visited c-major, b-minor).
 template <typename G, typename IO>
-__global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2dArgs a) {
+__global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(const Fwd2dArgs a) {
     using Ctx = ClusterCtx<G, false, true>;
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
     constexpr int Hh = M1 / 2, Ww = M2;                 // plane extents
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(G::THREADS, 1) hyena_fwd_2d_cluster(const Fwd2
 // floats (ox = ix - W). In place (K == Kout, rs = 2W + 2, cs = 2H (2W + 2)) is
 // allowed: every read precedes the first cluster barrier, every write follows it.
 template <typename G>
-__global__ void __launch_bounds__(G::THREADS, 1)
+__global__ void __launch_bounds__(G::THREADS, G::MINB)
     hyena_spectrum_2d_cluster(const float *K, int64_t rs, int64_t cs, c32 *Kout, const c32 *__restrict__ tw) {
     using Ctx = ClusterCtx<G, false, false>;
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
