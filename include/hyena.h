@@ -141,9 +141,10 @@ HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_im
  *           the implicit network, inside H_out, with no other memory.
  *   params  implicit network, or NULL (then h must not be NULL)
  *   H_out   1D: [N, D, M/2 + 1] complex64, bin k = sum_t h[t] e^{-2πi k t / M};
- *           2D: [N, C, 2H, W + 1] complex64, the 2D DFT of the kernel placed
+ *           2D: [N, C, W + 1, 2H] complex64, the 2D DFT of the kernel placed
  *           cyclically (offset o at index o mod 2H, o mod 2W), bins over the
- *           full row axis and the non-negative half of the column axis.
+ *           full row axis and the non-negative half of the column axis,
+ *           stored column-bin-major: bin (ky, kx) at [kx][ky].
  *           Unnormalised. Must not overlap h.
  */
 HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,

@@ -77,7 +77,7 @@ class Plan:
         if self.ndim == 1:
             return (self.order, self.channels, self.spectrum_elems)
         H, W = self.shape
-        return (self.order, self.channels, 2 * H, W + 1)
+        return (self.order, self.channels, W + 1, 2 * H)   # bin (ky, kx) at [kx][ky]
 
     def workspace_bytes(self, batch: int) -> int:
         return capi.hyena_workspace_bytes(self.handle, batch)

@@ -6,7 +6,7 @@
 //    pattern is made bank-conflict-free by swz<NS>() (see fft_regs.cuh).
 //  * NSEQ  > 0: NSEQ sequences, sequence-major, interleaved complex (one
 //    8-byte float2 per element, in the buffer passed as `sre`; `sim` is
-//    unused), element i of sequence s at s * LEN + (i ^ (s & 31)). Warps span
+//    unused), element i of sequence s at maddr<LEN, NSEQ>(i, s). Warps span
 //    the sequence index with a common i, so the XOR puts each half-warp on
 //    distinct 8-byte bank pairs; and lanes that span 32 consecutive i of one
 //    sequence touch one contiguous 256-byte block (what a remote,
@@ -30,15 +30,23 @@
 namespace hyena {
 
 // Sequence-major address of element i of sequence s (sequences of length LEN >= 32).
-template <int LEN>
+// NSW: the number of sequences a warp spans at a common i. With 16 or more,
+// each half-warp holds 16 sequences and XOR-ing the sequence index into i
+// puts them on distinct 8-byte bank pairs. With 8, each half-warp holds 8
+// sequences at two elements i, i' that differ in bit 0 or in bit 3 (every
+// Stockham pattern of radix-8 passes); XOR-ing 2s into bits 1..3 and bit 3
+// of i into bit 0 separates them.
+template <int LEN, int NSW = 32>
 __device__ __forceinline__ int maddr(int i, int s) {
-    return s * LEN + (i ^ (s & 31));
+    static_assert(NSW == 8 || NSW >= 16, "sequence-major layout needs 8 or at least 16 sequences per warp");
+    if constexpr (NSW >= 16) return s * LEN + (i ^ (s & 31));
+    else return s * LEN + (i ^ (((2 * s) & 15) | ((i >> 3) & 1)));
 }
 
 template <int NS, int NSEQ, int LEN>
 __device__ __forceinline__ int saddr(int i, int seq) {
     if constexpr (NSEQ == 0) return swz<NS>(i);
-    else return maddr<LEN>(i, seq);
+    else return maddr<LEN, NSEQ>(i, seq);
 }
 
 // One Stockham pass p of a length-LEN FFT (register layout in fft_regs.cuh).

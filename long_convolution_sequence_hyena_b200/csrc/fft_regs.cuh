@@ -279,11 +279,17 @@ __device__ __forceinline__ void dft16(V (&x)[NR]) {
 }
 
 // 8-point DFT on x[o + st*n], n = 0..7 (split n = 2 n1 + n2, k = k1 + 4 k2).
-template <int DIR, int st, int o, typename V, int NR>
+// HALF: inputs n >= 4 are zero.
+template <int DIR, bool HALF, int st, int o, typename V, int NR>
 __device__ __forceinline__ void dft8(V (&x)[NR]) {
 #define X(i) x[o + st * (i)]
-    dft4<DIR>(X(0), X(2), X(4), X(6));   // n2 = 0 -> A[0][k1] at 2*k1
-    dft4<DIR>(X(1), X(3), X(5), X(7));   // n2 = 1 -> A[1][k1] at 2*k1 + 1
+    if constexpr (HALF) {
+        dft4_half<DIR>(X(0), X(2), X(4), X(6));   // n2 = 0 -> A[0][k1] at 2*k1
+        dft4_half<DIR>(X(1), X(3), X(5), X(7));   // n2 = 1 -> A[1][k1] at 2*k1 + 1
+    } else {
+        dft4<DIR>(X(0), X(2), X(4), X(6));
+        dft4<DIR>(X(1), X(3), X(5), X(7));
+    }
     X(3) = tw8<DIR, 1>(X(3));
     X(5) = tw8<DIR, 2>(X(5));
     X(7) = tw8<DIR, 3>(X(7));
@@ -310,7 +316,7 @@ __device__ __forceinline__ void dft2r(V (&x)[NR]) {
 template <int R, int DIR, bool HALF, int st, int o, typename V, int NR>
 __device__ __forceinline__ void dftR(V (&x)[NR]) {
     if constexpr (R == 16) dft16<DIR, HALF, st, o>(x);
-    else if constexpr (R == 8) dft8<DIR, st, o>(x);
+    else if constexpr (R == 8) dft8<DIR, HALF, st, o>(x);
     else if constexpr (R == 4) dft4r<DIR, st, o>(x);
     else dft2r<DIR, st, o>(x);
 }

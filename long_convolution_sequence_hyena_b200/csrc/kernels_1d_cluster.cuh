@@ -96,9 +96,18 @@ __device__ __forceinline__ void slot_of_row(int k1, int &c, int &r) {
 // (1D: one transform of length MC); without it the two stages are the two
 // axes of a 2D transform of shape [M1][M2].
 // HALFX: columns n2 >= M2/2 hold zeros on input and are not needed on output
-// (2D, the zero-padded half of the x axis): they are neither transformed nor sent.
+// (2D, the zero-padded half of the x axis): they are neither transformed nor
+// sent, and the M2/2 data columns are spread over all C CTAs (NCOLP = NCOL/2
+// per CTA, twice the threads per column, E/2 values per thread), so that no
+// CTA idles through the column phase.
 template <typename G, bool TWID, bool HALFX>
 struct ClusterCtx {
+    static constexpr int NCOLP = HALFX ? G::NCOL / 2 : G::NCOL;   // columns per CTA, column phase
+    static constexpr int T1P = G::THREADS / NCOLP;                // threads per column FFT
+    static constexpr int E1 = G::M1 / T1P;                        // values per thread, column phase
+    static_assert(NCOLP * T1P == G::THREADS && E1 * T1P == G::M1, "column phase must use every thread");
+    static_assert(E1 == 8 || E1 == 16, "column FFTs run radix-8 or radix-16 passes");
+    static_assert(NCOLP == 8 || NCOLP >= 16, "warps must span 8 or at least 16 columns");
     // Twiddle table length: 1D, W_M with M = 2 MC; 2D, W_{2 M2} with 2 M2 >= M1.
     // The plan appends W_1024 to it for the sub-transforms (kept L1-resident).
     static constexpr int TWM = TWID ? 2 * G::MC : (2 * G::M2 >= G::M1 ? 2 * G::M2 : G::M1);
@@ -109,25 +118,28 @@ struct ClusterCtx {
     int j, t1, n2;   // column phase: local column, FFT lane, global column
     int r, t2, k1;   // row phase: local slot, FFT lane, global row
     int rm;          // slot of the mirror row of k1
-    bool col_live;   // this CTA owns at least one column that carries data
 
     __device__ __forceinline__ ClusterCtx(float *smem) {
         crank = (int)cg::this_cluster().block_rank();
         colb = reinterpret_cast<float2 *>(smem);
         rowb = colb + G::PER_CTA;
         const int tid = threadIdx.x;
-        j = tid % G::NCOL;
-        t1 = tid / G::NCOL;
-        n2 = crank * G::NCOL + j;
+        j = tid % NCOLP;
+        t1 = tid / NCOLP;
+        n2 = crank * NCOLP + j;
         r = tid % G::NROW;
         t2 = tid / G::NROW;
         k1 = row_of_slot<G>(crank, r);
         rm = (k1 == 0 || k1 == G::M1 / 2) ? r : (r < G::HROW ? r + G::HROW : r - G::HROW);
-        col_live = !HALFX || crank * G::NCOL < G::M2 / 2;
     }
 
-    // Complex index of column-layout register q: n = M2 * (t1 + q T1) + n2.
-    __device__ __forceinline__ int64_t col_index(int q) const { return (int64_t)G::M2 * (t1 + q * G::T1) + n2; }
+    // The column-phase registers: the first E1 of the E.
+    __device__ __forceinline__ static c32 (&col_regs(c32 (&v)[G::E]))[E1] {
+        return *reinterpret_cast<c32 (*)[E1]>(&v[0]);
+    }
+
+    // Complex index of column-layout register q: n = M2 * (t1 + q T1P) + n2.
+    __device__ __forceinline__ int64_t col_index(int q) const { return (int64_t)G::M2 * (t1 + q * T1P) + n2; }
 
     // v[q] *= base * step^q, q = 0..E-1 (product tree of depth <= 4, then one multiply).
     __device__ __forceinline__ static void twiddle_ramp(c32 (&v)[G::E], c32 base, c32 step) {
@@ -136,27 +148,28 @@ struct ClusterCtx {
         for (int q = 0; q < G::E; ++q) v[q] = mul(v[q], base);
     }
 
-    // Column layout (time domain, upper half of every column zero unless
-    // !HALF_COL) -> row layout (natural bins, register q = bin k2 = t2 + q T2 of row k1).
+    // Column layout (registers q < E1: time domain, upper half of every column
+    // zero unless !HALF_COL) -> row layout (natural bins, register q = bin
+    // k2 = t2 + q T2 of row k1).
     template <bool HALF_COL>
     __device__ __forceinline__ void forward(c32 (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
-        if (col_live) {
-            fft_cta<G::M1, E, -1, HALF_COL, TWS, G::NCOL>(v, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
-            if constexpr (TWID) {
-                constexpr int M = 2 * G::MC;
-                const c32 b = ldg_c(tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
-                const c32 st = ldg_c(tw + ((2 * (int64_t)n2 * G::T1) & (M - 1)));
-                twiddle_ramp(v, b, st);
-            }
-            if (!HALFX || 2 * n2 < G::M2) {
-                const int z = opaque_zero();   // recompute addresses per order rather than keep them live
+        c32 (&vc)[E1] = col_regs(v);
+        fft_cta<G::M1, E1, -1, HALF_COL, TWS, NCOLP>(vc, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
+        if constexpr (TWID) {
+            static_assert(E1 == E, "the four-step twiddle assumes one column layout");
+            constexpr int M = 2 * G::MC;
+            const c32 b = ldg_c(tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
+            const c32 st = ldg_c(tw + ((2 * (int64_t)n2 * T1P) & (M - 1)));
+            twiddle_ramp(v, b, st);
+        }
+        {
+            const int z = opaque_zero();   // recompute addresses per order rather than keep them live
 #pragma unroll
-                for (int q = 0; q < E; ++q) {
-                    int dst, slot;
-                    slot_of_row<G>(t1 + q * G::T1 + z, dst, slot);
-                    dsmem_st2(dsmem_map(smem_u32(rowb + maddr<G::M2>(n2, slot)), dst), v[q]);
-                }
+            for (int q = 0; q < E1; ++q) {
+                int dst, slot;
+                slot_of_row<G>(t1 + q * T1P + z, dst, slot);
+                dsmem_st2(dsmem_map(smem_u32(rowb + maddr<G::M2>(n2, slot)), dst), vc[q]);
             }
         }
         cluster_sync_mem();
@@ -204,18 +217,17 @@ struct ClusterCtx {
         for (int q = 0; q < E; ++q) {
             const int nn = t2 + q * G::T2 + z;
             if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
-            dsmem_st2(dsmem_map(smem_u32(colb + maddr<G::M1>(k1, nn % G::NCOL)), nn / G::NCOL), v[q]);
+            dsmem_st2(dsmem_map(smem_u32(colb + maddr<G::M1, NCOLP>(k1, nn % NCOLP)), nn / NCOLP), v[q]);
         }
         cluster_sync_mem();
-        if (col_live) {
+        c32 (&vc)[E1] = col_regs(v);
 #pragma unroll
-            for (int q = 0; q < E; ++q) {
-                const int ad = maddr<G::M1>(t1 + q * G::T1, j);
-                v[q] = mk(colb[ad].x, colb[ad].y);
-            }
-            __syncthreads();
-            fft_cta<G::M1, E, +1, false, TWS, G::NCOL>(v, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
+        for (int q = 0; q < E1; ++q) {
+            const int ad = maddr<G::M1, NCOLP>(t1 + q * T1P, j);
+            vc[q] = mk(colb[ad].x, colb[ad].y);
         }
+        __syncthreads();
+        fft_cta<G::M1, E1, +1, false, TWS, NCOLP>(vc, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
     }
 };
 

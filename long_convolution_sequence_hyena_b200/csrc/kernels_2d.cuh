@@ -21,7 +21,7 @@ namespace hyena {
 struct Fwd2dArgs {
     const void *v;
     const void *gates[HYENA_MAX_ORDER];
-    const c32 *K;         // [N, C, 2H, W + 1]
+    const c32 *K;         // [N, C, W + 1, 2H]: bin (ky, kx) at kx * 2H + ky
     const float *dskip;   // [N, C] or nullptr
     void *y;
     const c32 *tw;        // W_TWM^m
@@ -44,27 +44,28 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
     const int64_t c = ord / a.B;
     const int64_t b = ord - c * a.B;
     const int64_t plane = b * a.C + c;
-    const bool xin = 2 * cx.n2 < Ww;                    // this column carries data
     const c32 wb = ldg_c(a.tw + cx.t2 * (TWM / (2 * M2)));   // W_{2 M2}^{t2}
 
-    // column-layout register q holds (y = t1 + q T1, x' = n2)
-    auto pos_of = [&](int q) -> int64_t { return (int64_t)(cx.t1 + q * G::T1) * Ww + 2 * cx.n2; };
+    // Column-layout register q < E1 holds (y = t1 + q T1P, x' = n2); every
+    // column of the column phase carries data (x' < W/2), and the registers
+    // q < E1/2 hold the data rows y < H.
+    constexpr int E1 = Ctx::E1;
+    auto pos_of = [&](int q) -> int64_t { return (int64_t)(cx.t1 + q * Ctx::T1P) * Ww + 2 * cx.n2; };
 
     c32 v[E];
     {
         const IO *vp = reinterpret_cast<const IO *>(a.v) + plane * Hh * Ww;
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) v[q] = xin ? load_pair<IO, true>(vp, pos_of(q), (int64_t)Hh * Ww) : mk(0.f, 0.f);
+        for (int q = 0; q < E1 / 2; ++q) v[q] = load_pair<IO, true>(vp, pos_of(q), (int64_t)Hh * Ww);
 #pragma unroll
-        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+        for (int q = E1 / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
     for (int n = 0; n < a.order; ++n) {
         const IO *gp = reinterpret_cast<const IO *>(a.gates[n]) + plane * Hh * Ww;
-        typename io<IO>::pair_t g[E / 2];
+        typename io<IO>::pair_t g[E1 / 2];
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q)
-            g[q] = xin ? load_pair_raw<IO, true>(gp, pos_of(q), (int64_t)Hh * Ww) : io<IO>::zero();
+        for (int q = 0; q < E1 / 2; ++q) g[q] = load_pair_raw<IO, true>(gp, pos_of(q), (int64_t)Hh * Ww);
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.C + c) : 0.f;
         const c32 *Kp = a.K + ((int64_t)n * a.C + c) * (M1 * (M2 + 1));
 
@@ -85,8 +86,8 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
             const c32 wO = mul(w, Ok);
             const c32 Xk = add(Ek, wO);                  // bin (ky, kx)
             const c32 Xm = conj(sub(Ek, wO));            // bin (-ky, M2 - kx)
-            c32 Hk = ldg_c(Kp + (int64_t)ky * (M2 + 1) + kx);
-            c32 Hm = ldg_c(Kp + (int64_t)kym * (M2 + 1) + (M2 - kx));
+            c32 Hk = ldg_c(Kp + (int64_t)kx * M1 + ky);              // lanes run along ky: coalesced
+            c32 Hm = ldg_c(Kp + (int64_t)(M2 - kx) * M1 + kym);
             Hk.x += dsk;
             Hm.x += dsk;
             const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
@@ -99,22 +100,21 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
         __syncthreads();                                // mirror reads done before the row buffer is rewritten
         cx.inverse(v, a.tw);
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) {
+        for (int q = 0; q < E1 / 2; ++q) {
             const c32 gq = io<IO>::unpack(g[q]);
-            v[q] = xin ? mk(gq.x * v[q].x, gq.y * v[q].y) : mk(0.f, 0.f);
+            v[q] = mk(gq.x * v[q].x, gq.y * v[q].y);
         }
 #pragma unroll
-        for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
+        for (int q = E1 / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
-    if (xin) {
-        IO *yp = reinterpret_cast<IO *>(a.y) + plane * Hh * Ww;
+    IO *yp = reinterpret_cast<IO *>(a.y) + plane * Hh * Ww;
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) store_pair<IO, true>(yp, pos_of(q), (int64_t)Hh * Ww, v[q]);
-    }
+    for (int q = 0; q < E1 / 2; ++q) store_pair<IO, true>(yp, pos_of(q), (int64_t)Hh * Ww, v[q]);
 }
 
-// 2D kernel spectra. Kernel (n, c) starts at K + o * cs (o = n * C + c); row iy
+// 2D kernel spectra, stored kx-major ([W + 1][2H] per kernel: the spectral step's
+// lanes run along ky). Kernel (n, c) starts at K + o * cs (o = n * C + c); row iy
 // of its offset grid (offset oy = iy - H) starts at + iy * rs and holds 2W
 // floats (ox = ix - W). In place (K == Kout, rs = 2W + 2, cs = 2H (2W + 2)) is
 // allowed: every read precedes the first cluster barrier, every write follows it.
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB)
     const int ix = (2 * cx.n2 + Ww) & (2 * Ww - 1);    // cyclic column 2 n2 -> offset-grid column
 #pragma unroll
     for (int q = 0; q < E; ++q) {
-        const int iy = (cx.t1 + q * G::T1 + Hh) & (M1 - 1);
+        const int iy = (cx.t1 + q * Ctx::T1P + Hh) & (M1 - 1);
         const float *rowp = Kp + iy * rs;
         v[q] = mk(rowp[ix], rowp[ix + 1]);
     }
@@ -152,8 +152,8 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB)
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
         const c32 wO = mul(mul(wb, w2e<E>(q, z0)), Ok);
-        Ko[(int64_t)ky * (M2 + 1) + kx] = add(Ek, wO);
-        if (kx == 0) Ko[(int64_t)kym * (M2 + 1) + M2] = conj(sub(Ek, wO));   // bin (-ky, M2)
+        Ko[(int64_t)kx * M1 + ky] = add(Ek, wO);
+        if (kx == 0) Ko[(int64_t)M2 * M1 + kym] = conj(sub(Ek, wO));   // bin (-ky, M2)
     }
 }
 

@@ -87,8 +87,9 @@ def test_2d_spectrum_matches_dft(api, Hw):
     torch.cuda.synchronize()
     k64 = inp["h"].double().numpy()
     cyc = np.roll(k64, shift=(-Hw, -Hw), axis=(-2, -1))     # offset o at index o mod 2H, o mod 2W
-    ref = np.fft.rfft2(cyc)
-    err = np.abs(K.cpu().numpy().astype(np.complex128) - ref).max() / np.abs(k64).sum(axis=(-2, -1)).max()
+    ref = np.fft.rfft2(cyc)                                   # [.., ky, kx]; the library stores [.., kx, ky]
+    assert K.shape[-2:] == (Hw + 1, 2 * Hw)
+    err = np.abs(K.transpose(-1, -2).cpu().numpy().astype(np.complex128) - ref).max() / np.abs(k64).sum(axis=(-2, -1)).max()
     assert err < 2e-6, (Hw, err)
 
 
