@@ -43,6 +43,24 @@ __device__ __forceinline__ int maddr(int i, int s) {
     else return s * LEN + (i ^ (((2 * s) & 15) | ((i >> 3) & 1)));
 }
 
+// Shared-memory element of a value type in the sequence-major layout: one
+// 8-byte float2 per complex value, one 16-byte float4 (re a, re b, im a, im b)
+// per pair of complex values.
+template <typename V>
+struct selem;
+template <>
+struct selem<c32> {
+    using T = float2;
+    __device__ __forceinline__ static c32 ld(const float2 &f) { return mk(f.x, f.y); }
+    __device__ __forceinline__ static float2 st(c32 v) { return make_float2(v.x, v.y); }
+};
+template <>
+struct selem<c32x2> {
+    using T = float4;
+    __device__ __forceinline__ static c32x2 ld(const float4 &f) { return c32x2{f2(f.x, f.y), f2(f.z, f.w)}; }
+    __device__ __forceinline__ static float4 st(c32x2 v) { return make_float4(v.re.x, v.re.y, v.im.x, v.im.y); }
+};
+
 template <int NS, int NSEQ, int LEN>
 __device__ __forceinline__ int saddr(int i, int seq) {
     if constexpr (NSEQ == 0) return swz<NS>(i);
@@ -50,9 +68,12 @@ __device__ __forceinline__ int saddr(int i, int seq) {
 }
 
 // One Stockham pass p of a length-LEN FFT (register layout in fft_regs.cuh).
-template <int LEN, int E, int DIR, bool HALF_IN, int p, int TWM, int NSEQ>
-__device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim, int t,
+// V is c32, or c32x2 (two sequences in lockstep, sequence-major layout only).
+template <int LEN, int E, int DIR, bool HALF_IN, int p, int TWM, int NSEQ, typename V>
+__device__ __forceinline__ void fft_pass(V (&v)[E], float *__restrict__ sre, float *__restrict__ sim, int t,
                                          int seq, const c32 *__restrict__ tw) {
+    using SE = selem<V>;
+    static_assert(NSEQ > 0 || sizeof(V) == sizeof(c32), "lockstep pairs need the sequence-major layout");
     constexpr int T = LEN / E;
     constexpr int LR = pass_lr(E);
     constexpr int P = num_passes(LEN, LR);
@@ -69,15 +90,14 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
         for (int q = 0; q < E; ++q) {
             const int i = saddr<NSP, NSEQ, LEN>(t + q * T, seq);
             if constexpr (NSEQ > 0) {
-                const float2 f = reinterpret_cast<const float2 *>(sre)[i];
-                v[q] = mk(f.x, f.y);
+                v[q] = SE::ld(reinterpret_cast<const typename SE::T *>(sre)[i]);
             } else {
                 v[q] = mk(sre[i], sim[i]);
             }
         }
         __syncthreads();  // every read done before pass p writes
     }
-    static_for<S>([&](auto sc) {
+    static_for<S>([&](auto sc) __attribute__((always_inline)) {
         constexpr int s = decltype(sc)::value;
         const int j = t + s * T;
         const int k = j & (NS - 1);
@@ -93,7 +113,7 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
             for (int r = 0; r < R; ++r) {
                 const int i = saddr<NS, NSEQ, LEN>(base + r * NS, seq);
                 if constexpr (NSEQ > 0) {
-                    reinterpret_cast<float2 *>(sre)[i] = make_float2(v[s + r * S].x, v[s + r * S].y);
+                    reinterpret_cast<typename SE::T *>(sre)[i] = SE::st(v[s + r * S]);
                 } else {
                     sre[i] = v[s + r * S].x;
                     sim[i] = v[s + r * S].y;
@@ -109,8 +129,8 @@ __device__ __forceinline__ void fft_pass(c32 (&v)[E], float *__restrict__ sre, f
 // When the FFT has more than one pass, every shared-memory read it makes is
 // complete in all threads of the block on return (the last exchange ends with
 // a barrier).
-template <int LEN, int E, int DIR, bool HALF_IN, int TWM = 2 * LEN, int NSEQ = 0>
-__device__ __forceinline__ void fft_cta(c32 (&v)[E], float *sre, float *sim, int t, const c32 *__restrict__ tw,
+template <int LEN, int E, int DIR, bool HALF_IN, int TWM = 2 * LEN, int NSEQ = 0, typename V>
+__device__ __forceinline__ void fft_cta(V (&v)[E], float *sre, float *sim, int t, const c32 *__restrict__ tw,
                                         int seq = 0) {
     fft_pass<LEN, E, DIR, HALF_IN, 0, TWM, NSEQ>(v, sre, sim, t, seq, tw);
 }

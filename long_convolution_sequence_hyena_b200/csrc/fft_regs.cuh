@@ -19,7 +19,10 @@
 
 namespace hyena {
 
-// Compile-time loop: f(std::integral_constant<int, i>) for i = 0..N-1.
+// Compile-time loop: f(std::integral_constant<int, i>) for i = 0..N-1. Bodies that
+// take register arrays by reference are marked always_inline: a lambda left
+// out of line makes its captured array addressable, and the array then lives
+// in local memory.
 template <typename F, int... I>
 __device__ __forceinline__ void static_for_impl(F &&f, std::integer_sequence<int, I...>) {
     (f(std::integral_constant<int, I>{}), ...);

@@ -29,9 +29,11 @@ namespace cg = cooperative_groups;
 
 // MINB: CTAs resident per SM (the launch bounds); with 2, one cluster's
 // barrier waits are covered by another cluster's work on the same SMs.
-template <int MC_, int C_, int M1_, int E_, int MINB_ = 1>
+// ROWS: rows per cluster, 1 (complex values) or 2 (two rows in lockstep as
+// c32x2: every shared element is 16 bytes).
+template <int MC_, int C_, int M1_, int E_, int MINB_ = 1, int ROWS_ = 1>
 struct ClusterGeom {
-    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_, MINB = MINB_;
+    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_, MINB = MINB_, ROWS = ROWS_;
     static constexpr int NCOL = M2 / C;          // columns per CTA (column phase)
     static constexpr int NROW = M1 / C;          // rows per CTA (row phase), in mirror pairs
     static constexpr int HROW = NROW / 2;        // rows k1 < M1/2 per CTA
@@ -39,9 +41,10 @@ struct ClusterGeom {
     static constexpr int T2 = M2 / E;            // threads per row FFT
     static constexpr int THREADS = NCOL * T1;
     static constexpr int PER_CTA = MC / C;       // complex elements per CTA per buffer
-    // column buffer + row buffer + staging for one order's gates (E/2 pairs per thread)
-    static constexpr size_t GATE_STAGE = (size_t)THREADS * (E / 2) * 8;
-    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8 + GATE_STAGE;
+    // column buffer + row buffer + staging for one order's gates (E/2 element pairs per thread and row)
+    static constexpr size_t GATE_STAGE = (size_t)THREADS * (E / 2) * 8 * ROWS;
+    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8 * ROWS + GATE_STAGE;
+    static_assert(ROWS == 1 || ROWS == 2, "one row or a lockstep pair per cluster");
     static_assert(THREADS == NROW * T2, "both phases must use the same thread count");
     static_assert(NCOL >= 16 && NROW >= 16, "warps must span at least 16 sequences");
     static_assert(M1 >= 32 && M2 >= 32, "sequence-major layouts need sequences of at least 32");
@@ -58,8 +61,13 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t local, int rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
     return remote;
 }
-__device__ __forceinline__ void dsmem_st2(uint32_t addr, c32 v) {
+__device__ __forceinline__ void dsmem_st(uint32_t addr, c32 v) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+__device__ __forceinline__ void dsmem_st(uint32_t addr, c32x2 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.re.x), "f"(v.re.y),
+                 "f"(v.im.x), "f"(v.im.y)
+                 : "memory");
 }
 // Cluster barrier that also orders shared::cluster memory (release / acquire).
 __device__ __forceinline__ void cluster_sync_mem() {
@@ -100,8 +108,11 @@ __device__ __forceinline__ void slot_of_row(int k1, int &c, int &r) {
 // sent, and the M2/2 data columns are spread over all C CTAs (NCOLP = NCOL/2
 // per CTA, twice the threads per column, E/2 values per thread), so that no
 // CTA idles through the column phase.
-template <typename G, bool TWID, bool HALFX>
+template <typename G, bool TWID, bool HALFX, typename V = c32>
 struct ClusterCtx {
+    using SE = selem<V>;
+    using ET = typename SE::T;
+    static_assert(sizeof(ET) == 8 * G::ROWS, "value type must match the geometry's rows per cluster");
     static constexpr int NCOLP = HALFX ? G::NCOL / 2 : G::NCOL;   // columns per CTA, column phase
     static constexpr int T1P = G::THREADS / NCOLP;                // threads per column FFT
     static constexpr int E1 = G::M1 / T1P;                        // values per thread, column phase
@@ -113,7 +124,7 @@ struct ClusterCtx {
     static constexpr int TWM = TWID ? 2 * G::MC : (2 * G::M2 >= G::M1 ? 2 * G::M2 : G::M1);
     static constexpr int TWS = 1024;
     static_assert(TWS % G::M1 == 0 && TWS % G::M2 == 0, "sub-transform twiddles");
-    float2 *colb, *rowb;   // column and row buffers, interleaved complex, sequence-major
+    ET *colb, *rowb;       // column and row buffers, interleaved complex, sequence-major
     int crank;
     int j, t1, n2;   // column phase: local column, FFT lane, global column
     int r, t2, k1;   // row phase: local slot, FFT lane, global row
@@ -121,7 +132,7 @@ struct ClusterCtx {
 
     __device__ __forceinline__ ClusterCtx(float *smem) {
         crank = (int)cg::this_cluster().block_rank();
-        colb = reinterpret_cast<float2 *>(smem);
+        colb = reinterpret_cast<ET *>(smem);
         rowb = colb + G::PER_CTA;
         const int tid = threadIdx.x;
         j = tid % NCOLP;
@@ -134,15 +145,16 @@ struct ClusterCtx {
     }
 
     // The column-phase registers: the first E1 of the E.
-    __device__ __forceinline__ static c32 (&col_regs(c32 (&v)[G::E]))[E1] {
-        return *reinterpret_cast<c32 (*)[E1]>(&v[0]);
+    __device__ __forceinline__ static V (&col_regs(V (&v)[G::E]))[E1] {
+        if constexpr (E1 == G::E) return v;
+        else return *reinterpret_cast<V (*)[E1]>(&v[0]);
     }
 
     // Complex index of column-layout register q: n = M2 * (t1 + q T1P) + n2.
     __device__ __forceinline__ int64_t col_index(int q) const { return (int64_t)G::M2 * (t1 + q * T1P) + n2; }
 
     // v[q] *= base * step^q, q = 0..E-1 (product tree of depth <= 4, then one multiply).
-    __device__ __forceinline__ static void twiddle_ramp(c32 (&v)[G::E], c32 base, c32 step) {
+    __device__ __forceinline__ static void twiddle_ramp(V (&v)[G::E], c32 base, c32 step) {
         twiddle_powers<G::E, 1, 0>(v, step);
 #pragma unroll
         for (int q = 0; q < G::E; ++q) v[q] = mul(v[q], base);
@@ -152,9 +164,9 @@ struct ClusterCtx {
     // zero unless !HALF_COL) -> row layout (natural bins, register q = bin
     // k2 = t2 + q T2 of row k1).
     template <bool HALF_COL>
-    __device__ __forceinline__ void forward(c32 (&v)[G::E], const c32 *__restrict__ tw) {
+    __device__ __forceinline__ void forward(V (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
-        c32 (&vc)[E1] = col_regs(v);
+        V (&vc)[E1] = col_regs(v);
         fft_cta<G::M1, E1, -1, HALF_COL, TWS, NCOLP>(vc, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
         if constexpr (TWID) {
             static_assert(E1 == E, "the four-step twiddle assumes one column layout");
@@ -169,17 +181,16 @@ struct ClusterCtx {
             for (int q = 0; q < E1; ++q) {
                 int dst, slot;
                 slot_of_row<G>(t1 + q * T1P + z, dst, slot);
-                dsmem_st2(dsmem_map(smem_u32(rowb + maddr<G::M2>(n2, slot)), dst), vc[q]);
+                dsmem_st(dsmem_map(smem_u32(rowb + maddr<G::M2>(n2, slot)), dst), vc[q]);
             }
         }
         cluster_sync_mem();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             if (HALFX && q >= E / 2) {
-                v[q] = mk(0.f, 0.f);
+                v[q] = SE::ld(ET{});
             } else {
-                const int ad = maddr<G::M2>(t2 + q * G::T2, r);
-                v[q] = mk(rowb[ad].x, rowb[ad].y);
+                v[q] = SE::ld(rowb[maddr<G::M2>(t2 + q * G::T2, r)]);
             }
         }
         __syncthreads();
@@ -187,23 +198,17 @@ struct ClusterCtx {
     }
 
     // Store the row-layout bins so the mirror bins can be read (ends with a CTA barrier).
-    __device__ __forceinline__ void publish(const c32 (&v)[G::E]) {
+    __device__ __forceinline__ void publish(const V (&v)[G::E]) {
 #pragma unroll
-        for (int q = 0; q < G::E; ++q) {
-            const int ad = maddr<G::M2>(t2 + q * G::T2, r);
-            rowb[ad] = make_float2(v[q].x, v[q].y);
-        }
+        for (int q = 0; q < G::E; ++q) rowb[maddr<G::M2>(t2 + q * G::T2, r)] = SE::st(v[q]);
         __syncthreads();
     }
     // Published bin (mirror row, column k2m) from this CTA's own buffer.
-    __device__ __forceinline__ c32 mirror_bin(int k2m) const {
-        const int ad = maddr<G::M2>(k2m, rm);
-        return mk(rowb[ad].x, rowb[ad].y);
-    }
+    __device__ __forceinline__ V mirror_bin(int k2m) const { return SE::ld(rowb[maddr<G::M2>(k2m, rm)]); }
 
     // Row layout (bins) -> column layout (time domain, unscaled inverse).
     // Must follow a CTA barrier after the last read of the published bins.
-    __device__ __forceinline__ void inverse(c32 (&v)[G::E], const c32 *__restrict__ tw) {
+    __device__ __forceinline__ void inverse(V (&v)[G::E], const c32 *__restrict__ tw) {
         constexpr int E = G::E;
         fft_cta<G::M2, E, +1, false, TWS, G::NROW>(v, reinterpret_cast<float *>(rowb), nullptr, t2, tw + TWM, r);
         if constexpr (TWID) {
@@ -215,17 +220,16 @@ struct ClusterCtx {
         const int z = opaque_zero();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
+            // zero-padding half (nn >= M2/2 exactly when q >= E/2): never read back,
+            // so the last row pass need not produce it
+            if (HALFX && q >= E / 2) continue;
             const int nn = t2 + q * G::T2 + z;
-            if (HALFX && 2 * nn >= G::M2) continue;   // zero-padding half: never read back
-            dsmem_st2(dsmem_map(smem_u32(colb + maddr<G::M1, NCOLP>(k1, nn % NCOLP)), nn / NCOLP), v[q]);
+            dsmem_st(dsmem_map(smem_u32(colb + maddr<G::M1, NCOLP>(k1, nn % NCOLP)), nn / NCOLP), v[q]);
         }
         cluster_sync_mem();
-        c32 (&vc)[E1] = col_regs(v);
+        V (&vc)[E1] = col_regs(v);
 #pragma unroll
-        for (int q = 0; q < E1; ++q) {
-            const int ad = maddr<G::M1, NCOLP>(t1 + q * T1P, j);
-            vc[q] = mk(colb[ad].x, colb[ad].y);
-        }
+        for (int q = 0; q < E1; ++q) vc[q] = SE::ld(colb[maddr<G::M1, NCOLP>(t1 + q * T1P, j)]);
         __syncthreads();
         fft_cta<G::M1, E1, +1, false, TWS, NCOLP>(vc, reinterpret_cast<float *>(colb), nullptr, t1, tw + TWM, j);
     }

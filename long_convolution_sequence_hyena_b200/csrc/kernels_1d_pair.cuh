@@ -38,7 +38,7 @@ __device__ __forceinline__ void fft_pass_x2(c32x2 (&v)[E], float2 *__restrict__ 
         }
         __syncthreads();  // every read done before pass p writes
     }
-    static_for<S>([&](auto sc) {
+    static_for<S>([&](auto sc) __attribute__((always_inline)) {
         constexpr int s = decltype(sc)::value;
         const int j = t + s * T;
         const int k = j & (NS - 1);

@@ -51,6 +51,18 @@ def test_cluster_lengths(api, L, N, dtype):
     compare(w, inp, oracle_filters_1d(w, inp), y, context="cluster L=%d N=%d" % (L, N))
 
 
+@pytest.mark.parametrize("L,B,D,N,dtype", [(16385, 3, 1, 2, "f32"), (40001, 1, 3, 1, "bf16"), (32768, 2, 3, 1, "f32"),
+                                         (65536, 2, 1, 1, "f32")])
+def test_cluster_batches_and_channels(api, L, B, D, N, dtype):
+    """Cluster rows over several batches and channels: odd row counts, B = 1, B odd and B even
+    (rows are visited d-major, b-minor)."""
+    w = explicit_case(B, D, L, N, dtype, seed=700 + L + B, alpha=(1e-4, 1e-2))
+    inp = make_inputs(w)
+    plan, _, y = _run(api, w, inp)
+    assert plan.path == 1
+    compare(w, inp, oracle_filters_1d(w, inp), y, context="cluster L=%d B=%d D=%d" % (L, B, D))
+
+
 def test_cluster_implicit_in_place(api):
     w = WORKLOADS["order2_bf16_b4_d1024_l8192_implicit"].scaled(B=1, D=2, shape=(20000,))
     inp = make_inputs(w)
