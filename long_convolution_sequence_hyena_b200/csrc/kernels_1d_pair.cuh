@@ -72,6 +72,13 @@ __device__ __forceinline__ void fft_cta_x2(c32x2 (&v)[E], float2 *sre, float2 *s
 // Spectral step for both rows (see spectral_product in kernels_1d.cuh). The
 // unpacking is written without its factors 1/2; those and the 1/MC of the
 // inverse are folded into the (shared) filter gain.
+//
+// Bins k and MC - k need the same intermediates: with A = Y[k], B = Y[MC-k],
+// Ye ~ A + conj B and Yo ~ (A - conj B) conj(W_M^k), the packed inverse input
+// is Ye + i Yo at k and conj(Ye - i Yo) at MC - k (W_M^{MC-k} = -conj W_M^k).
+// Each thread therefore takes its bins k = t + qT with q < E/2 (thread 0 also
+// k = MC/2, its own mirror) and produces both outputs; the mirror outputs
+// reach their owners (thread T - t, register E-1-q) through shared memory.
 template <int MC, int E>
 __device__ __forceinline__ void spectral_product_x2(c32x2 (&v)[E], float2 *__restrict__ sre,
                                                     float2 *__restrict__ sim, int t, const c32 *Hs, float dsk,
@@ -86,11 +93,10 @@ __device__ __forceinline__ void spectral_product_x2(c32x2 (&v)[E], float2 *__res
     __syncthreads();
     constexpr float s = 0.25f / (float)MC;
     const int z0 = opaque_zero();
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
+    // Ye and Yo of bin k from Z[k] (register) and Z[MC-k] (shared memory)
+    auto bin_pair = [&](int q, c32x2 Zk, c32x2 &Ye, c32x2 &Yo) __attribute__((always_inline)) {
         const int k = t + q * T;
         const int km = (MC - k) & (MC - 1);
-        const c32x2 Zk = v[q];
         const float2 mre = sre[km], mim = sim[km];
         // 2E = Zk + conj Zm, 2O = (Zk - conj Zm) / i
         const c32x2 E2{f2add(Zk.re, mre), f2sub(Zk.im, mim)};
@@ -103,11 +109,37 @@ __device__ __forceinline__ void spectral_product_x2(c32x2 (&v)[E], float2 *__res
         Hk = mk(s * (Hk.x + dsk), s * Hk.y);
         Hm = mk(s * (Hm.x + dsk), s * Hm.y);
         const c32x2 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
-        const c32x2 Ye{f2add(Yk.re, Ym.re), f2sub(Yk.im, Ym.im)};   // Yk + conj Ym
+        Ye = c32x2{f2add(Yk.re, Ym.re), f2sub(Yk.im, Ym.im)};   // Yk + conj Ym
         const c32x2 Yd{f2sub(Yk.re, Ym.re), f2add(Yk.im, Ym.im)};   // Yk - conj Ym
-        const c32x2 Yo = mul(Yd, conj(w));
-        v[q] = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};   // Ye + i Yo
+        Yo = mul(Yd, conj(w));
+    };
+    c32x2 vh = v[E / 2];
+    if (t == 0) {   // k = MC/2 is its own mirror
+        c32x2 Ye, Yo;
+        bin_pair(E / 2, v[E / 2], Ye, Yo);
+        vh = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};
     }
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        c32x2 Ye, Yo;
+        bin_pair(q, v[q], Ye, Yo);
+        v[q] = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};             // Ye + i Yo       (bin k)
+        v[E / 2 + q] = c32x2{f2add(Ye.re, Yo.im), f2sub(Yo.re, Ye.im)};    // conj(Ye - i Yo) (bin MC - k)
+    }
+    __syncthreads();   // every mirror read done
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        const int km = (MC - (t + q * T)) & (MC - 1);
+        sre[km] = v[E / 2 + q].re;
+        sim[km] = v[E / 2 + q].im;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = E / 2; q < E; ++q) {
+        const int k = t + q * T;
+        v[q] = c32x2{sre[k], sim[k]};
+    }
+    if (t == 0) v[E / 2] = vh;
     __syncthreads();
 }
 
