@@ -127,6 +127,13 @@ constexpr int fwd_smem_floats_per_row(int MC) { return 2 * MC + (stage_spectrum(
 // in the 1/2 of the repacking and the 1/MC of the inverse transform.
 // Hs: the spectrum row staged in shared memory (cp.async group pending), or
 // nullptr to read Hrow from global memory. wt = W_M^t.
+//
+// Bins k and MC - k need the same intermediates: with A = Y[k], B = Y[MC-k],
+// Ye = (A + conj B)/2 and Yo = (A - conj B) conj(W_M^k)/2, the packed inverse
+// input is Ye + i Yo at k and conj(Ye - i Yo) at MC - k (W_M^{MC-k} =
+// -conj W_M^k). Each thread takes its bins k = t + qT with q < E/2 (thread 0
+// also k = MC/2, its own mirror) and produces both; the mirror outputs reach
+// their owners (thread T - t, register E-1-q) through shared memory.
 template <int MC, int E>
 __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict__ sre, float *__restrict__ sim,
                                                  int t, const c32 *__restrict__ Hrow, const c32 *Hs, float dsk,
@@ -141,11 +148,9 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
     __syncthreads();
     constexpr float s = 0.5f / (float)MC;
     const int z0 = opaque_zero();
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
+    auto bin_pair = [&](int q, c32 Zk, c32 &Ye, c32 &Yo) __attribute__((always_inline)) {
         const int k = t + q * T;
         const int km = (MC - k) & (MC - 1);
-        const c32 Zk = v[q];
         const c32 Zm = mk(sre[km], sim[km]);
         const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
         const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
@@ -158,12 +163,38 @@ __device__ __forceinline__ void spectral_product(c32 (&v)[E], float *__restrict_
         Hk.x += dsk;
         Hm.x += dsk;
         const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
-        const c32 Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
+        Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
         const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
-        const c32 Yo = mul(Yd, conj(w));
-        v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+        Yo = mul(Yd, conj(w));
+    };
+    c32 vh = v[E / 2];
+    if (t == 0) {   // k = MC/2 is its own mirror
+        c32 Ye, Yo;
+        bin_pair(E / 2, v[E / 2], Ye, Yo);
+        vh = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+    }
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        c32 Ye, Yo;
+        bin_pair(q, v[q], Ye, Yo);
+        v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);              // Ye + i Yo       (bin k)
+        v[E / 2 + q] = mk(Ye.x + Yo.y, Yo.x - Ye.y);      // conj(Ye - i Yo) (bin MC - k)
         if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
     }
+    __syncthreads();   // every mirror read done
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        const int km = (MC - (t + q * T)) & (MC - 1);
+        sre[km] = v[E / 2 + q].x;
+        sim[km] = v[E / 2 + q].y;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = E / 2; q < E; ++q) {
+        const int k = t + q * T;
+        v[q] = mk(sre[k], sim[k]);
+    }
+    if (t == 0) v[E / 2] = vh;
     __syncthreads();
 }
 

@@ -205,6 +205,10 @@ struct ClusterCtx {
     }
     // Published bin (mirror row, column k2m) from this CTA's own buffer.
     __device__ __forceinline__ V mirror_bin(int k2m) const { return SE::ld(rowb[maddr<G::M2>(k2m, rm)]); }
+    // Hand a result to the owner of (mirror row, column k2m), after every mirror read.
+    __device__ __forceinline__ void set_mirror_bin(int k2m, V val) { rowb[maddr<G::M2>(k2m, rm)] = SE::st(val); }
+    // Row-layout register q from the buffer (results handed over by set_mirror_bin).
+    __device__ __forceinline__ V own_bin(int q) const { return SE::ld(rowb[maddr<G::M2>(t2 + q * G::T2, r)]); }
 
     // Row layout (bins) -> column layout (time domain, unscaled inverse).
     // Must follow a CTA barrier after the last read of the published bins.
@@ -277,15 +281,17 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(cons
 
         cx.template forward<true>(v, a.tw);
         cx.publish(v);
+        // Spectral step, bins in pairs (k, MC - k): the mirror of register q is
+        // register E-1-q of thread (rm, T2-1-t2) (in row 0: of thread (0, T2-t2),
+        // and register E-q when t2 = 0), so each thread takes q < E/2 and returns
+        // the mirror result conj(Ye - i Yo) to its owner; bin (0, M2/2) is its own mirror.
         constexpr float s = 0.5f / (float)MC;
         const int z0 = opaque_zero();
-#pragma unroll
-        for (int q = 0; q < E; ++q) {
+        auto bin_pair = [&](int q, c32 Zk, c32 &Ye, c32 &Yo) __attribute__((always_inline)) {
             const int k2 = cx.t2 + q * G::T2;
             const int k = cx.k1 + M1 * k2;
             const int km = (MC - k) & (MC - 1);
             const c32 Zm = cx.mirror_bin(km / M1);
-            const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
             const c32 w = mul(wb, w2e<E>(q, z0));              // W_M^k, k = k1 + M1 (t2 + q T2)
@@ -297,13 +303,36 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(cons
             Hk.x += dsk;
             Hm.x += dsk;
             const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
-            const c32 Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
+            Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
             const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
-            const c32 Yo = mul(Yd, conj(w));
-            v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+            Yo = mul(Yd, conj(w));
+        };
+        const bool self_half = cx.k1 == 0 && cx.t2 == 0;
+        c32 vh = v[E / 2];
+        if (self_half) {
+            c32 Ye, Yo;
+            bin_pair(E / 2, v[E / 2], Ye, Yo);
+            vh = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+        }
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            c32 Ye, Yo;
+            bin_pair(q, v[q], Ye, Yo);
+            v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);              // Ye + i Yo       (bin k)
+            v[E / 2 + q] = mk(Ye.x + Yo.y, Yo.x - Ye.y);      // conj(Ye - i Yo) (bin MC - k)
             if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
         }
-        __syncthreads();                                // mirror reads done before the row buffer is rewritten
+        __syncthreads();                                // every mirror read done
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int k = cx.k1 + M1 * (cx.t2 + q * G::T2);
+            cx.set_mirror_bin(((MC - k) & (MC - 1)) / M1, v[E / 2 + q]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = cx.own_bin(q);
+        if (self_half) v[E / 2] = vh;
+        __syncthreads();                                // row buffer reads done before the inverse rewrites it
         cx.inverse(v, a.tw);
 
         // gate (registers q >= E/2 hold positions >= MC, i.e. padding)

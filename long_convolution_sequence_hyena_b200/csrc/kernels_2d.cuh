@@ -71,15 +71,18 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
 
         cx.template forward<true>(v, a.tw);
         cx.publish(v);
+        // Spectral step, bins in pairs ((ky, kx), (-ky, -kx)): the mirror of register
+        // q is register E-1-q of thread (rm, T2-t2) (register E-q when t2 = 0), so
+        // each thread takes q < E/2 and returns the mirror result conj(Ye - i Yo) to
+        // its owner; threads with t2 = 0 also take q = E/2 (kx = M2/2, whose mirror
+        // is in the upper half of both owners).
         constexpr float s = 0.5f / (float)(M1 * M2);
         const int ky = cx.k1;
         const int kym = (M1 - ky) & (M1 - 1);
         const int z0 = opaque_zero();
-#pragma unroll
-        for (int q = 0; q < E; ++q) {
+        auto bin_pair = [&](int q, c32 Zk, c32 &Ye, c32 &Yo) __attribute__((always_inline)) {
             const int kx = cx.t2 + q * G::T2;
             const c32 Zm = cx.mirror_bin((M2 - kx) & (M2 - 1));
-            const c32 Zk = v[q];
             const c32 Ek = mk(0.5f * (Zk.x + Zm.x), 0.5f * (Zk.y - Zm.y));
             const c32 Ok = mk(0.5f * (Zk.y + Zm.y), -0.5f * (Zk.x - Zm.x));
             const c32 w = mul(wb, w2e<E>(q, z0));            // W_{2 M2}^{kx}
@@ -91,13 +94,33 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
             Hk.x += dsk;
             Hm.x += dsk;
             const c32 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
-            const c32 Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
+            Ye = mk(s * (Yk.x + Ym.x), s * (Yk.y - Ym.y));
             const c32 Yd = mk(s * (Yk.x - Ym.x), s * (Yk.y + Ym.y));
-            const c32 Yo = mul(Yd, conj(w));
-            v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+            Yo = mul(Yd, conj(w));
+        };
+        const bool self_half = cx.t2 == 0;
+        c32 vh = v[E / 2];
+        if (self_half) {
+            c32 Ye, Yo;
+            bin_pair(E / 2, v[E / 2], Ye, Yo);
+            vh = mk(Ye.x - Yo.y, Ye.y + Yo.x);
+        }
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            c32 Ye, Yo;
+            bin_pair(q, v[q], Ye, Yo);
+            v[q] = mk(Ye.x - Yo.y, Ye.y + Yo.x);              // Ye + i Yo       (bin (ky, kx))
+            v[E / 2 + q] = mk(Ye.x + Yo.y, Yo.x - Ye.y);      // conj(Ye - i Yo) (bin (-ky, -kx))
             if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
         }
-        __syncthreads();                                // mirror reads done before the row buffer is rewritten
+        __syncthreads();                                // every mirror read done
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) cx.set_mirror_bin((M2 - (cx.t2 + q * G::T2)) & (M2 - 1), v[E / 2 + q]);
+        __syncthreads();
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = cx.own_bin(q);
+        if (self_half) v[E / 2] = vh;
+        __syncthreads();                                // row buffer reads done before the inverse rewrites it
         cx.inverse(v, a.tw);
 #pragma unroll
         for (int q = 0; q < E1 / 2; ++q) {
