@@ -64,8 +64,10 @@ typedef enum {
 /* Which kernel family a plan runs (hyena_plan_info). */
 typedef enum {
     HYENA_PATH_CTA = 0,          /* 1D, M <= 32768: one CTA per row, all orders fused */
-    HYENA_PATH_CLUSTER = 1,      /* 1D, 32768 < M <= 262144: a thread-block cluster per row */
-    HYENA_PATH_2D = 2            /* 2D grid */
+    HYENA_PATH_CLUSTER = 1,      /* 1D, M = 262144: a thread-block cluster per row */
+    HYENA_PATH_2D = 2,           /* 2D grid */
+    HYENA_PATH_STAGED = 3        /* 1D, M in {65536, 131072}: column and row kernels per order,
+                                    the row's transform in a device workspace */
 } hyena_path_t;
 
 /*
@@ -121,7 +123,11 @@ HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);
  */
 HYENA_API hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path);
 
-/* Bytes of device workspace hyena_forward needs for `batch` (0 for on-chip paths). */
+/*
+ * Bytes of device workspace hyena_forward needs for `batch`: 0 except on
+ * HYENA_PATH_STAGED, where rows run in chunks that keep their transforms in
+ * L2, and the workspace holds one chunk: min(batch * D, chunk) * (M/2) * 8 bytes.
+ */
 HYENA_API size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch);
 
 /*

@@ -1,0 +1,61 @@
+// 1D staged long-row path: instantiations and the per-chunk launch sequence.
+#include "kernels_1d_staged.cuh"
+#include "launch.h"
+
+namespace hyena {
+
+using GS_32K = StagedGeom<32768, 128, 32, 16>;   // M = 65536: columns of 128, rows of 256
+using GS_64K = StagedGeom<65536, 256, 16, 16>;   // M = 131072: 256 x 256
+
+int64_t staged_chunk_rows(int64_t MC) {
+    // rows whose transforms (MC complex64 each) fit in 48 MB: the chunk stays in L2
+    const int64_t r = ((int64_t)48 << 20) / (MC * 8);
+    return r < 1 ? 1 : r;
+}
+
+bool staged_path_supported(int64_t MC) { return MC == 32768 || MC == 65536; }
+
+template <typename G, typename IO, bool EVEN>
+cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cudaStream_t st) {
+    for (int64_t o0 = 0; o0 < f.rows; o0 += chunk) {
+        const int64_t nr = (f.rows - o0) < chunk ? (f.rows - o0) : chunk;
+        StagedArgs a;
+        a.f = f;
+        a.ws = ws;
+        a.o0 = o0;
+        a.n = 0;
+        hyena_staged_cols<G, IO, EVEN, 0><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+        for (int n = 0; n < f.order; ++n) {
+            a.n = n;
+            hyena_staged_rows<G><<<(unsigned)(nr * G::RGROUPS), G::RT, G::RSMEM, st>>>(a);
+            if (n + 1 < f.order)
+                hyena_staged_cols<G, IO, EVEN, 1><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+            else
+                hyena_staged_cols<G, IO, EVEN, 2><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <typename G>
+cudaError_t launch_staged_g(const Fwd1dArgs &f, float2 *ws, int64_t chunk, hyena_dtype_t dt, bool even,
+                            cudaStream_t st) {
+    if (dt == HYENA_F32)
+        return even ? launch_staged_io<G, float, true>(f, ws, chunk, st) : launch_staged_io<G, float, false>(f, ws, chunk, st);
+    return even ? launch_staged_io<G, __nv_bfloat16, true>(f, ws, chunk, st)
+                : launch_staged_io<G, __nv_bfloat16, false>(f, ws, chunk, st);
+}
+
+cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &f, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
+                                 cudaStream_t st) {
+    const int64_t chunk = staged_chunk_rows(MC);
+    switch (MC) {
+        case 32768: return launch_staged_g<GS_32K>(f, ws, chunk, dt, even, st);
+        case 65536: return launch_staged_g<GS_64K>(f, ws, chunk, dt, even, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace hyena

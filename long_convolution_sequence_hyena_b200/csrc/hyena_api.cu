@@ -107,7 +107,8 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         p.M = next_pow2(2 * p.L);
         if (p.M < 32) p.M = 32;  // smallest FFT the kernels run (extra zero padding is exact)
         p.MC = p.M / 2;
-        p.path = p.M <= HYENA_MAX_M_CTA ? HYENA_PATH_CTA : HYENA_PATH_CLUSTER;
+        p.path = p.M <= HYENA_MAX_M_CTA ? HYENA_PATH_CTA
+                 : (staged_path_supported(p.MC) ? HYENA_PATH_STAGED : HYENA_PATH_CLUSTER);
         p.spectrum_elems = p.MC + 1;
         p.tw_len = p.M;
     } else {
@@ -162,7 +163,10 @@ hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spe
 
 size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch) {
     if (!plan || batch < 0) return 0;
-    return 0;
+    if (plan->path != HYENA_PATH_STAGED) return 0;
+    const int64_t rows = batch * plan->D;
+    const int64_t chunk = staged_chunk_rows(plan->MC);
+    return (size_t)(rows < chunk ? rows : chunk) * (size_t)plan->MC * sizeof(float2);
 }
 
 hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_implicit_params_t *params, float *h_out,
@@ -218,8 +222,6 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
 
 hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, const void *const *gates, const void *H,
                              const float *Dskip, void *y, void *workspace, size_t ws_bytes, void *stream) {
-    (void)workspace;
-    (void)ws_bytes;
     if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
     if (batch == 0) return HYENA_OK;  // nothing to read or write; pointers may be NULL
     if (!v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
@@ -228,6 +230,9 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     if (!aligned16(v) || !aligned16(H) || !aligned16(y) || (Dskip && !aligned4(Dskip))) return HYENA_ERR_ALIGNMENT;
     for (int n = 0; n < plan->order; ++n)
         if (!aligned16(gates[n])) return HYENA_ERR_ALIGNMENT;
+    const size_t ws_need = hyena_workspace_bytes(plan, batch);
+    if (ws_need && (!workspace || ws_bytes < ws_need)) return HYENA_ERR_WORKSPACE;
+    if (ws_need && !aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
     hyena_status_t s = check_device(plan);
     if (s != HYENA_OK) return s;
 
@@ -261,7 +266,10 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     a.order = plan->order;
     const bool even = (plan->L % 2) == 0;
     cudaError_t e;
-    if (plan->path == HYENA_PATH_CLUSTER)
+    if (plan->path == HYENA_PATH_STAGED)
+        e = launch_fwd_1d_staged(a, plan->MC, reinterpret_cast<float2 *>(workspace), plan->dtype, even,
+                                 (cudaStream_t)stream);
+    else if (plan->path == HYENA_PATH_CLUSTER)
         e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     else if (pair_path_supported(plan->MC, batch))
         e = launch_fwd_1d_pair(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);

@@ -1,5 +1,5 @@
-"""GPU parity of the cluster paths (1D rows with M > 32768, and 2D grids)
-against the fp64 oracle, through the C ABI."""
+"""GPU parity of the long-row paths (1D rows with M > 32768: staged and cluster)
+and of the 2D cluster path against the fp64 oracle, through the C ABI."""
 import numpy as np
 import pytest
 import torch
@@ -15,6 +15,11 @@ pytestmark = pytest.mark.gpu
 def api():
     from long_convolution_sequence_hyena_b200 import api as a
     return a
+
+
+def long_path(plan):
+    """Path the library takes for a 1D plan with M > 32768: staged up to M = 131072, else cluster."""
+    return 3 if plan.fft_len in (65536, 131072) else 1
 
 
 def _run(api, w, inp):
@@ -33,7 +38,7 @@ def test_cluster_spectrum_matches_dft(api, L):
     w = explicit_case(1, 3, L, 1, "f32", seed=L, alpha=(1e-4, 1e-2))
     inp = make_inputs(w)
     plan = api.Plan((L,), 3, 1, torch.float32)
-    assert plan.path == 1
+    assert plan.path == long_path(plan)
     H = plan.filter_spectrum(h=inp["h"].cuda())
     torch.cuda.synchronize()
     ref = np.fft.rfft(inp["h"].double().numpy(), n=plan.fft_len, axis=-1)
@@ -47,8 +52,8 @@ def test_cluster_lengths(api, L, N, dtype):
     w = explicit_case(1, 2, L, N, dtype, seed=500 + L, alpha=(1e-4, 1e-2))
     inp = make_inputs(w)
     plan, _, y = _run(api, w, inp)
-    assert plan.path == 1
-    compare(w, inp, oracle_filters_1d(w, inp), y, context="cluster L=%d N=%d" % (L, N))
+    assert plan.path == long_path(plan)
+    compare(w, inp, oracle_filters_1d(w, inp), y, context="long row L=%d N=%d" % (L, N))
 
 
 @pytest.mark.parametrize("L,B,D,N,dtype", [(16385, 3, 1, 2, "f32"), (40001, 1, 3, 1, "bf16"), (32768, 2, 3, 1, "f32"),
@@ -59,8 +64,38 @@ def test_cluster_batches_and_channels(api, L, B, D, N, dtype):
     w = explicit_case(B, D, L, N, dtype, seed=700 + L + B, alpha=(1e-4, 1e-2))
     inp = make_inputs(w)
     plan, _, y = _run(api, w, inp)
-    assert plan.path == 1
-    compare(w, inp, oracle_filters_1d(w, inp), y, context="cluster L=%d B=%d D=%d" % (L, B, D))
+    assert plan.path == long_path(plan)
+    compare(w, inp, oracle_filters_1d(w, inp), y, context="long row L=%d B=%d D=%d" % (L, B, D))
+
+
+def test_staged_chunks(api):
+    """More rows than one workspace chunk holds (M = 65536: 192 rows per chunk); rows on both
+    sides of the chunk boundary are checked."""
+    w = explicit_case(2, 100, 16385, 2, "bf16", seed=1234, alpha=(1e-4, 1e-2))
+    inp = make_inputs(w)
+    plan, _, y = _run(api, w, inp)
+    assert plan.path == 3 and plan.workspace_bytes(2) == 192 * 32768 * 8
+    # visit order is d-major, b-minor: visit index o -> flat row (o % B) * D + o // B
+    visits = np.array([0, 1, 190, 191, 192, 193, 198, 199])
+    rows = (visits % 2) * 100 + visits // 2
+    compare(w, inp, oracle_filters_1d(w, inp), y, rows=rows, context="staged chunks")
+
+
+def test_staged_workspace_checks(api):
+    from long_convolution_sequence_hyena_b200 import capi
+    plan = api.Plan((65536,), 2, 1, torch.bfloat16)
+    need = plan.workspace_bytes(3)
+    assert plan.path == 3 and need == 6 * 65536 * 8
+    v = torch.zeros(3, 2, 65536, dtype=torch.bfloat16, device="cuda")
+    H = torch.zeros(plan.spectrum_shape, dtype=torch.complex64, device="cuda")
+    ws = torch.empty(need + 16, dtype=torch.uint8, device="cuda")
+    args = (plan.handle, 3, v.data_ptr(), [v.data_ptr()], H.data_ptr(), None, v.data_ptr())
+    assert capi.hyena_forward(*args, None, 0) == capi.HYENA_ERR_WORKSPACE
+    assert capi.hyena_forward(*args, ws.data_ptr(), need - 8) == capi.HYENA_ERR_WORKSPACE
+    assert capi.hyena_forward(*args, ws.data_ptr() + 8, need) == capi.HYENA_ERR_ALIGNMENT
+    assert capi.hyena_forward(*args, ws.data_ptr(), need) == capi.HYENA_OK
+    torch.cuda.synchronize()
+    assert plan.workspace_bytes(0) == 0 and api.Plan((8192,), 2, 1).workspace_bytes(3) == 0
 
 
 def test_cluster_implicit_in_place(api):
