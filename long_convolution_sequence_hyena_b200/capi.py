@@ -17,7 +17,7 @@ HYENA_MAX_ORDER = 8
 HYENA_F32, HYENA_BF16 = 0, 1
 (HYENA_OK, HYENA_ERR_INVALID_ARG, HYENA_ERR_UNSUPPORTED, HYENA_ERR_ALIGNMENT,
  HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA, HYENA_ERR_NOMEM) = range(7)
-HYENA_PATH_CTA, HYENA_PATH_CLUSTER, HYENA_PATH_2D = 0, 1, 2
+HYENA_PATH_CTA, HYENA_PATH_CLUSTER, HYENA_PATH_2D, HYENA_PATH_STAGED = 0, 1, 2, 3
 
 STATUS_NAMES = {
     HYENA_OK: "HYENA_OK", HYENA_ERR_INVALID_ARG: "HYENA_ERR_INVALID_ARG",
