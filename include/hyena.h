@@ -176,6 +176,37 @@ HYENA_API hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const v
 /* Static, human-readable name of a status code. */
 HYENA_API const char *hyena_status_string(hyena_status_t status);
 
+/*
+ * hyena_forward for callers that cannot allocate device memory where they
+ * run the operator: a plain C host program linked to this library, which has
+ * no allocator of its own to hand out a workspace; a process whose device
+ * memory belongs to a framework's caching allocator; a latency-bound loop in
+ * which a cudaMalloc, which may synchronise the device, is not acceptable.
+ * The paper has no counterpart of this call: it changes only where the
+ * staged path's scratch lives, not what is computed.
+ *
+ * Plans on HYENA_PATH_STAGED only (1D, M in {65536, 131072}); any other plan
+ * returns HYENA_ERR_UNSUPPORTED (those paths need no workspace: call
+ * hyena_forward with workspace NULL). The other arguments are those of
+ * hyena_forward, and so is the result.
+ *
+ * The scratch is one array of HYENA_STATIC_SCRATCH_BYTES in device memory,
+ * per device, held from when the library is loaded until the process exits.
+ * Rows run in chunks of HYENA_STATIC_SCRATCH_BYTES / (M/2 * 8) rows (32 rows
+ * at M = 131072); a plan whose row transform would not fit returns
+ * HYENA_ERR_WORKSPACE. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current): make that first
+ * call before any stream capture. Nothing in the array has to start at zero
+ * (a chunk's transforms are written before they are read), but every call on
+ * a device uses the same array: calls whose kernels overlap on the GPU (on
+ * different streams, or from different host threads) race; order them on one
+ * stream or with events. This call allocates no memory.
+ */
+#define HYENA_STATIC_SCRATCH_BYTES (16u << 20)   /* 16 MiB */
+HYENA_API hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batch, const void *v,
+                                                const void *const *gates, const void *H, const float *Dskip,
+                                                void *y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

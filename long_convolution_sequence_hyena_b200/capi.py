@@ -30,6 +30,7 @@ STATUS_NAMES = {
 EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
+    "hyena_forward_no_alloc",
 )
 
 
@@ -59,6 +60,7 @@ def _load():
         "hyena_filter_spectrum": ([p, p, ctypes.POINTER(hyena_implicit_params_t), p, p], i32),
         "hyena_forward": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_status_string": ([i32], ctypes.c_char_p),
+        "hyena_forward_no_alloc": ([p, i64, p, ctypes.POINTER(p), p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -109,3 +111,10 @@ def hyena_forward(plan, batch: int, v: int, gates, H: int, Dskip, y: int, worksp
                   stream: int = 0) -> int:
     garr = None if gates is None else (ctypes.c_void_p * len(gates))(*gates)
     return lib.hyena_forward(plan, batch, v, garr, H, Dskip, y, workspace, ws_bytes, stream)
+
+
+def hyena_forward_no_alloc(plan, batch: int, v: int, gates, H: int, Dskip, y: int, stream: int = 0) -> int:
+    """hyena_forward without a workspace argument: the staged path's scratch is the library's
+    own fixed device array (for callers that cannot allocate device memory)."""
+    garr = None if gates is None else (ctypes.c_void_p * len(gates))(*gates)
+    return lib.hyena_forward_no_alloc(plan, batch, v, garr, H, Dskip, y, stream)
