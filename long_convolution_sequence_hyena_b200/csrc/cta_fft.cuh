@@ -61,9 +61,14 @@ struct selem<c32x2> {
     __device__ __forceinline__ static float4 st(c32x2 v) { return make_float4(v.re.x, v.re.y, v.im.x, v.im.y); }
 };
 
-template <int NS, int NSEQ, int LEN>
+// Exchange address of element i. Sequence-major layouts with 16-byte
+// elements (lockstep pairs) are read and written a quarter-warp (8 lanes) at
+// a time; with 8 or more sequences per warp at a common i, the plain XOR of
+// the sequence index already spreads those 8 over distinct 16-byte bank groups.
+template <int NS, int NSEQ, int LEN, int EB = 8>
 __device__ __forceinline__ int saddr(int i, int seq) {
     if constexpr (NSEQ == 0) return swz<NS>(i);
+    else if constexpr (EB == 16) return maddr<LEN, 32>(i, seq);
     else return maddr<LEN, NSEQ>(i, seq);
 }
 
@@ -73,7 +78,9 @@ template <int LEN, int E, int DIR, bool HALF_IN, int p, int TWM, int NSEQ, typen
 __device__ __forceinline__ void fft_pass(V (&v)[E], float *__restrict__ sre, float *__restrict__ sim, int t,
                                          int seq, const c32 *__restrict__ tw) {
     using SE = selem<V>;
+    constexpr int EB = (int)sizeof(typename SE::T);
     static_assert(NSEQ > 0 || sizeof(V) == sizeof(c32), "lockstep pairs need the sequence-major layout");
+    static_assert(EB == 8 || NSEQ >= 8, "16-byte elements need at least 8 sequences per warp");
     constexpr int T = LEN / E;
     constexpr int LR = pass_lr(E);
     constexpr int P = num_passes(LEN, LR);
@@ -88,7 +95,7 @@ __device__ __forceinline__ void fft_pass(V (&v)[E], float *__restrict__ sre, flo
         __syncthreads();  // writes of pass p-1 visible
 #pragma unroll
         for (int q = 0; q < E; ++q) {
-            const int i = saddr<NSP, NSEQ, LEN>(t + q * T, seq);
+            const int i = saddr<NSP, NSEQ, LEN, EB>(t + q * T, seq);
             if constexpr (NSEQ > 0) {
                 v[q] = SE::ld(reinterpret_cast<const typename SE::T *>(sre)[i]);
             } else {
@@ -111,7 +118,7 @@ __device__ __forceinline__ void fft_pass(V (&v)[E], float *__restrict__ sre, flo
             const int base = (j / NS) * NS * R + k;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const int i = saddr<NS, NSEQ, LEN>(base + r * NS, seq);
+                const int i = saddr<NS, NSEQ, LEN, EB>(base + r * NS, seq);
                 if constexpr (NSEQ > 0) {
                     reinterpret_cast<typename SE::T *>(sre)[i] = SE::st(v[s + r * S]);
                 } else {

@@ -4,12 +4,14 @@
 
 namespace hyena {
 
-using GS_32K = StagedGeom<32768, 128, 32, 16>;   // M = 65536: columns of 128, rows of 256
-using GS_64K = StagedGeom<65536, 256, 16, 16>;   // M = 131072: 256 x 256
+// two rows in lockstep per CTA, 128 threads (three CTAs per SM)
+using GS_32K = StagedGeom<32768, 128, 16, 8, 2>;   // M = 65536: columns of 128, rows of 256
+using GS_64K = StagedGeom<65536, 256, 8, 8, 2>;    // M = 131072: 256 x 256
 
 int64_t staged_chunk_rows(int64_t MC) {
-    // rows whose transforms (MC complex64 each) fit in 48 MB: the chunk stays in L2
-    const int64_t r = ((int64_t)48 << 20) / (MC * 8);
+    // rows whose transforms (MC complex64 each) fill 96 MB: most of a chunk stays
+    // in L2 between launches, and each launch spans several waves of CTAs
+    const int64_t r = ((int64_t)96 << 20) / (MC * 8);
     return r < 1 ? 1 : r;
 }
 
@@ -17,21 +19,24 @@ bool staged_path_supported(int64_t MC) { return MC == 32768 || MC == 65536; }
 
 template <typename G, typename IO, bool EVEN>
 cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cudaStream_t st) {
+    static_assert(G::ROWS == 2, "the launch sequence below runs the lockstep kernels");
     for (int64_t o0 = 0; o0 < f.rows; o0 += chunk) {
         const int64_t nr = (f.rows - o0) < chunk ? (f.rows - o0) : chunk;
+        const int64_t pairs = (nr + 1) / 2;
         StagedArgs a;
         a.f = f;
         a.ws = ws;
         a.o0 = o0;
         a.n = 0;
-        hyena_staged_cols<G, IO, EVEN, 0><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+        const unsigned cgrid = (unsigned)(pairs * G::CGROUPS), rgrid = (unsigned)(pairs * G::RGROUPS);
+        hyena_staged_cols_x2<G, IO, EVEN, 0><<<cgrid, G::CT, G::CSMEM, st>>>(a, nr);
         for (int n = 0; n < f.order; ++n) {
             a.n = n;
-            hyena_staged_rows<G><<<(unsigned)(nr * G::RGROUPS), G::RT, G::RSMEM, st>>>(a);
+            hyena_staged_rows_x2<G><<<rgrid, G::RT, G::RSMEM, st>>>(a, nr);
             if (n + 1 < f.order)
-                hyena_staged_cols<G, IO, EVEN, 1><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+                hyena_staged_cols_x2<G, IO, EVEN, 1><<<cgrid, G::CT, G::CSMEM, st>>>(a, nr);
             else
-                hyena_staged_cols<G, IO, EVEN, 2><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
+                hyena_staged_cols_x2<G, IO, EVEN, 2><<<cgrid, G::CT, G::CSMEM, st>>>(a, nr);
         }
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -21,9 +21,11 @@
 
 namespace hyena {
 
-template <int MC_, int M1_, int NCOL_, int NROW_>
+// ROWS: rows per CTA, 1 (complex values) or 2 (two rows in lockstep as c32x2;
+// 16-byte shared elements).
+template <int MC_, int M1_, int NCOL_, int NROW_, int ROWS_ = 1>
 struct StagedGeom {
-    static constexpr int MC = MC_, M1 = M1_, M2 = MC_ / M1_, E = 16;
+    static constexpr int MC = MC_, M1 = M1_, M2 = MC_ / M1_, E = 16, ROWS = ROWS_;
     static constexpr int NCOL = NCOL_;               // columns per column-kernel CTA
     static constexpr int NROW = NROW_;               // rows per row-kernel CTA (mirror pairs)
     static constexpr int HROW = NROW / 2;
@@ -33,12 +35,15 @@ struct StagedGeom {
     static constexpr int CGROUPS = M2 / NCOL;        // column CTAs per row
     static constexpr int RGROUPS = M1 / NROW;        // row CTAs per row
     static constexpr int TWS = 1024;                 // sub-transform twiddle table W_1024
-    static constexpr size_t CSMEM = (size_t)NCOL * M1 * 8;
-    static constexpr size_t RSMEM = (size_t)NROW * M2 * 8;
+    static constexpr size_t CSMEM = (size_t)NCOL * M1 * 8 * ROWS;
+    static constexpr size_t RSMEM = (size_t)NROW * M2 * 8 * ROWS;
     static_assert(M2 % NCOL == 0 && M1 % NROW == 0 && NROW % 2 == 0, "groups must tile the row");
-    static_assert(NCOL >= 16 && NROW >= 16, "warps must span at least 16 sequences");
+    static_assert((ROWS == 1 && NCOL >= 16 && NROW >= 16) || (ROWS == 2 && NCOL >= 8 && NROW >= 8),
+                  "warps must span enough sequences for conflict-free exchanges");
     static_assert(TWS % M1 == 0 && TWS % M2 == 0, "sub-transform twiddles");
     static_assert(CT <= 1024 && RT <= 1024, "too many threads");
+    static_assert(ROWS == 2 || RT == M2, "the row kernel copies one element of every row per thread");
+    static_assert(M2 % RT == 0, "row copies tile the row");
 };
 
 struct StagedArgs {
@@ -135,11 +140,10 @@ __global__ void __launch_bounds__(G::RT, 2) hyena_staged_rows(const StagedArgs a
     float2 *wrow = a.ws + lr * MC;
     const c32 *tws = a.f.tw + M;
 
-    // the group's rows, coalesced, into the sequence-major buffer
-    for (int e = threadIdx.x; e < NROW * M2; e += G::RT) {
-        const int s = e / M2, k2 = e % M2;
-        cp_async8(rowb + maddr<M2>(k2, s), wrow + (int64_t)row_of_slot<G>(g, s) * M2 + k2);
-    }
+    // the group's rows, coalesced, into the sequence-major buffer (thread = column k2)
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl)
+        cp_async8(rowb + maddr<M2>(threadIdx.x, sl), wrow + (int64_t)row_of_slot<G>(g, sl) * M2 + threadIdx.x);
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
@@ -227,9 +231,215 @@ __global__ void __launch_bounds__(G::RT, 2) hyena_staged_rows(const StagedArgs a
         rowb[maddr<M2>(t2 + q * T2, r)] = make_float2(o.x, o.y);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < NROW * M2; e += G::RT) {
-        const int sl = e / M2, k2 = e % M2;
-        wrow[(int64_t)row_of_slot<G>(g, sl) * M2 + k2] = rowb[maddr<M2>(k2, sl)];
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl)
+        wrow[(int64_t)row_of_slot<G>(g, sl) * M2 + threadIdx.x] = rowb[maddr<M2>(threadIdx.x, sl)];
+}
+
+// ---------------------------------------------------------------------------
+// The same two kernels for two rows of the chunk in lockstep (c32x2: lane a =
+// visit index o, lane b = o + 1). Butterflies, twiddle products and exchanges
+// are one instruction for both rows; each lane reads its own gate, spectrum
+// row and feedthrough. An odd row count leaves the last pair's lane b empty.
+
+template <typename G, typename IO, bool EVEN, int MODE>
+__global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArgs a, int64_t nr) {
+    static_assert(G::ROWS == 2, "lockstep geometry");
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T1 = G::T1, MC = G::MC, M = 2 * MC;
+    extern __shared__ float smem[];
+    const int64_t lp = blockIdx.x / G::CGROUPS;      // row pair within the chunk
+    const int cgp = blockIdx.x % G::CGROUPS;
+    const int j = threadIdx.x % G::NCOL, t1 = threadIdx.x / G::NCOL;
+    const int n2 = cgp * G::NCOL + j;
+    const bool has1 = 2 * lp + 1 < nr;
+    int64_t d0, d1;
+    const int64_t row0 = visit_row(a.f, a.o0 + 2 * lp, d0);
+    const int64_t row1 = visit_row(a.f, a.o0 + 2 * lp + (has1 ? 1 : 0), d1);
+    const int64_t L = a.f.L;
+    float2 *w0 = a.ws + (2 * lp) * MC;
+    float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
+    const c32 *tws = a.f.tw + M;                     // W_1024
+    auto pos_of = [&](int q) -> int64_t { return 2 * ((int64_t)M2 * (t1 + q * T1) + n2); };
+
+    c32x2 v[E];
+    if constexpr (MODE == 0) {
+        const IO *r0 = reinterpret_cast<const IO *>(a.f.v) + row0 * L;
+        const IO *r1 = reinterpret_cast<const IO *>(a.f.v) + row1 * L;
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const c32 x0 = load_pair<IO, EVEN>(r0, pos_of(q), L);
+            const c32 x1 = has1 ? load_pair<IO, EVEN>(r1, pos_of(q), L) : mk(0.f, 0.f);
+            v[q] = c32x2{f2(x0.x, x1.x), f2(x0.y, x1.y)};
+        }
+    } else {
+        using P = typename io<IO>::pair_t;
+        const IO *g0 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + row0 * L;
+        const IO *g1 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + row1 * L;
+        P ga[E / 2], gb[E / 2];   // this order's gates, loaded while the inverse transform runs
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            ga[q] = load_pair_raw<IO, EVEN>(g0, pos_of(q), L);
+            gb[q] = load_pair_raw<IO, EVEN>(g1, pos_of(q), L);
+        }
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const int ad = (t1 + q * T1) * M2 + n2;     // k1 = t1 + q T1
+            const float2 f0 = w0[ad], f1 = w1[ad];
+            v[q] = c32x2{f2(f0.x, f1.x), f2(f0.y, f1.y)};
+        }
+        fft_cta<M1, E, +1, false, G::TWS, G::NCOL>(v, smem, nullptr, t1, tws, j);
+#pragma unroll
+        for (int q = 0; q < E / 2; ++q) {
+            const int64_t pos = pos_of(q);
+            const c32 ca = io<IO>::unpack(ga[q]), cb = io<IO>::unpack(gb[q]);
+            v[q] = c32x2{pos < L ? f2mul(v[q].re, f2(ca.x, cb.x)) : f2(0.f, 0.f),
+                         pos + 1 < L ? f2mul(v[q].im, f2(ca.y, cb.y)) : f2(0.f, 0.f)};
+        }
+        if constexpr (MODE == 2) {
+            IO *y0 = reinterpret_cast<IO *>(a.f.y) + row0 * L;
+            IO *y1 = reinterpret_cast<IO *>(a.f.y) + row1 * L;
+#pragma unroll
+            for (int q = 0; q < E / 2; ++q) {
+                store_pair<IO, EVEN>(y0, pos_of(q), L, mk(v[q].re.x, v[q].im.x));
+                if (has1) store_pair<IO, EVEN>(y1, pos_of(q), L, mk(v[q].re.y, v[q].im.y));
+            }
+            return;
+        }
+    }
+    if constexpr (MODE != 2) {
+#pragma unroll
+        for (int q = E / 2; q < E; ++q) v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
+        fft_cta<M1, E, -1, true, G::TWS, G::NCOL>(v, smem, nullptr, t1, tws, j);
+        const c32 base = ldg_c(a.f.tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
+        const c32 step = ldg_c(a.f.tw + ((2 * (int64_t)n2 * T1) & (M - 1)));
+        twiddle_powers<E, 1, 0>(v, step);
+#pragma unroll
+        for (int q = 0; q < E; ++q) {
+            const c32x2 r = mul(v[q], base);
+            const int ad = (t1 + q * T1) * M2 + n2;
+            w0[ad] = make_float2(r.re.x, r.im.x);
+            if (has1) w1[ad] = make_float2(r.re.y, r.im.y);
+        }
+    }
+}
+
+template <typename G>
+__global__ void __launch_bounds__(G::RT, 3) hyena_staged_rows_x2(const StagedArgs a, int64_t nr) {
+    static_assert(G::ROWS == 2, "lockstep geometry");
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, MC = G::MC, M = 2 * MC;
+    constexpr int NROW = G::NROW, HROW = G::HROW, RT = G::RT;
+    extern __shared__ float smem[];
+    float4 *rowb = reinterpret_cast<float4 *>(smem);
+    const int64_t lp = blockIdx.x / G::RGROUPS;
+    const int g = blockIdx.x % G::RGROUPS;
+    const int r = threadIdx.x % NROW, t2 = threadIdx.x / NROW;
+    const int k1 = row_of_slot<G>(g, r);
+    const int rm = (k1 == 0 || k1 == M1 / 2) ? r : (r < HROW ? r + HROW : r - HROW);   // slot of row M1 - k1
+    const bool has1 = 2 * lp + 1 < nr;
+    int64_t d0, d1;
+    (void)visit_row(a.f, a.o0 + 2 * lp, d0);
+    (void)visit_row(a.f, a.o0 + 2 * lp + (has1 ? 1 : 0), d1);
+    float2 *w0 = a.ws + (2 * lp) * MC;
+    float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
+    const c32 *tws = a.f.tw + M;
+    // shared element (re a, re b, im a, im b)
+    auto ld = [&](int ad) -> c32x2 {
+        const float4 f = rowb[ad];
+        return c32x2{f2(f.x, f.y), f2(f.z, f.w)};
+    };
+    auto st = [&](int ad, c32x2 x) { rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y); };
+
+    // the group's rows of both lanes, coalesced, into the sequence-major buffer
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl) {
+        const int64_t base = (int64_t)row_of_slot<G>(g, sl) * M2;
+#pragma unroll
+        for (int k2 = threadIdx.x; k2 < M2; k2 += RT) {
+            const float2 f0 = w0[base + k2], f1 = w1[base + k2];
+            rowb[maddr<M2>(k2, sl)] = make_float4(f0.x, f1.x, f0.y, f1.y);
+        }
+    }
+    __syncthreads();
+    c32x2 v[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = ld(maddr<M2>(t2 + q * T2, r));
+    __syncthreads();
+    fft_cta<M2, E, -1, false, G::TWS, NROW>(v, smem, nullptr, t2, tws, r);
+#pragma unroll
+    for (int q = 0; q < E; ++q) st(maddr<M2>(t2 + q * T2, r), v[q]);
+    __syncthreads();
+
+    // spectral step on both lanes, bins in pairs (k, MC - k) as in hyena_staged_rows;
+    // the unpacking is written without its factors 1/2, folded into the gain
+    const float dsk0 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.D + d0) : 0.f;
+    const float dsk1 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.D + d1) : 0.f;
+    const c32 *H0 = a.f.H + ((int64_t)a.n * a.f.D + d0) * (MC + 1);
+    const c32 *H1 = a.f.H + ((int64_t)a.n * a.f.D + d1) * (MC + 1);
+    const c32 wb = ldg_c(a.f.tw + k1 + M1 * t2);     // W_M^{k1 + M1 t2}
+    constexpr float s = 0.25f / (float)MC;
+    const int z0 = opaque_zero();
+    auto bin_pair = [&](int q, c32x2 Zk, c32x2 &Ye, c32x2 &Yo) __attribute__((always_inline)) {
+        const int k = k1 + M1 * (t2 + q * T2);
+        const int km = (MC - k) & (MC - 1);
+        const c32x2 Zm = ld(maddr<M2>(km / M1, rm));
+        const c32x2 E2{f2add(Zk.re, Zm.re), f2sub(Zk.im, Zm.im)};   // Zk + conj Zm
+        const c32x2 O2{f2add(Zk.im, Zm.im), f2sub(Zm.re, Zk.re)};   // (Zk - conj Zm) / i
+        const c32 w = mul(wb, w2e<E>(q, z0));                        // W_M^k
+        const c32x2 wO = mul(O2, w);
+        const c32x2 Xk = add(E2, wO);
+        const c32x2 Xm{f2sub(E2.re, wO.re), f2sub(wO.im, E2.im)};
+        const c32 hk0 = ldg_c(H0 + k), hk1 = ldg_c(H1 + k);
+        const c32 hm0 = ldg_c(H0 + (MC - k)), hm1 = ldg_c(H1 + (MC - k));
+        const c32x2 Hk{f2(s * (hk0.x + dsk0), s * (hk1.x + dsk1)), f2(s * hk0.y, s * hk1.y)};
+        const c32x2 Hm{f2(s * (hm0.x + dsk0), s * (hm1.x + dsk1)), f2(s * hm0.y, s * hm1.y)};
+        const c32x2 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
+        Ye = c32x2{f2add(Yk.re, Ym.re), f2sub(Yk.im, Ym.im)};       // Yk + conj Ym
+        const c32x2 Yd{f2sub(Yk.re, Ym.re), f2add(Yk.im, Ym.im)};   // Yk - conj Ym
+        Yo = mul(Yd, conj(w));
+    };
+    const bool self_half = k1 == 0 && t2 == 0;
+    c32x2 vh = v[E / 2];
+    if (self_half) {
+        c32x2 Ye, Yo;
+        bin_pair(E / 2, v[E / 2], Ye, Yo);
+        vh = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};
+    }
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        c32x2 Ye, Yo;
+        bin_pair(q, v[q], Ye, Yo);
+        v[q] = c32x2{f2sub(Ye.re, Yo.im), f2add(Ye.im, Yo.re)};             // Ye + i Yo       (bin k)
+        v[E / 2 + q] = c32x2{f2add(Ye.re, Yo.im), f2sub(Yo.re, Ye.im)};    // conj(Ye - i Yo) (bin MC - k)
+        if ((q & 3) == 3) asm volatile("" ::: "memory");  // bound load hoisting (register pressure)
+    }
+    __syncthreads();                                      // every mirror read done
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        const int k = k1 + M1 * (t2 + q * T2);
+        st(maddr<M2>(((MC - k) & (MC - 1)) / M1, rm), v[E / 2 + q]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = E / 2; q < E; ++q) v[q] = ld(maddr<M2>(t2 + q * T2, r));
+    if (self_half) v[E / 2] = vh;
+    __syncthreads();                                      // buffer reads done before the inverse rewrites it
+
+    fft_cta<M2, E, +1, false, G::TWS, NROW>(v, smem, nullptr, t2, tws, r);
+    const c32 base = conj(ldg_c(a.f.tw + ((2 * (int64_t)t2 * k1) & (M - 1))));
+    const c32 step = conj(ldg_c(a.f.tw + ((2 * (int64_t)T2 * k1) & (M - 1))));
+    twiddle_powers<E, 1, 0>(v, step);
+#pragma unroll
+    for (int q = 0; q < E; ++q) st(maddr<M2>(t2 + q * T2, r), mul(v[q], base));
+    __syncthreads();
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl) {
+        const int64_t base_ad = (int64_t)row_of_slot<G>(g, sl) * M2;
+#pragma unroll
+        for (int k2 = threadIdx.x; k2 < M2; k2 += RT) {
+            const float4 f = rowb[maddr<M2>(k2, sl)];
+            w0[base_ad + k2] = make_float2(f.x, f.z);
+            if (has1) w1[base_ad + k2] = make_float2(f.y, f.w);
+        }
     }
 }
 
