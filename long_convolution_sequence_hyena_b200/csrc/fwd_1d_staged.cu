@@ -9,9 +9,9 @@ using GS_32K = StagedGeom<32768, 128, 16, 8, 2>;   // M = 65536: columns of 128,
 using GS_64K = StagedGeom<65536, 256, 8, 8, 2>;    // M = 131072: 256 x 256
 
 int64_t staged_chunk_rows(int64_t MC) {
-    // rows whose transforms (MC complex64 each) fill 96 MB: most of a chunk stays
+    // rows whose transforms (MC complex64 each) fill 64 MB: most of a chunk stays
     // in L2 between launches, and each launch spans several waves of CTAs
-    const int64_t r = ((int64_t)96 << 20) / (MC * 8);
+    const int64_t r = ((int64_t)64 << 20) / (MC * 8);
     return r < 1 ? 1 : r;
 }
 

@@ -53,6 +53,34 @@ struct StagedArgs {
     int n;            // order: gate x^n (column kernel), spectrum H^n (row kernel)
 };
 
+// L2 eviction priorities. The chunk's workspace is written and read again by
+// the next launch, so it is kept (evict_last); the spectrum rows are read once
+// per launch and must not push it out (evict_first).
+__device__ __forceinline__ uint64_t l2_keep() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_stream() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ float2 ld_pol(const float2 *ptr, uint64_t pol) {
+    float2 v;
+    asm volatile("ld.global.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;" : "=f"(v.x), "=f"(v.y) : "l"(ptr), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ c32 ldc_pol(const c32 *ptr, uint64_t pol) {   // read-only data
+    float2 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;" : "=f"(v.x), "=f"(v.y) : "l"(ptr), "l"(pol));
+    return mk(v.x, v.y);
+}
+__device__ __forceinline__ void st_pol(float2 *ptr, float2 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(ptr), "f"(v.x), "f"(v.y), "l"(pol)
+                 : "memory");
+}
+
 // Flat row of visit index o (d-major, b-minor: the B rows of one channel run together).
 __device__ __forceinline__ int64_t visit_row(const Fwd1dArgs &f, int64_t o, int64_t &d) {
     d = o / f.B;
@@ -281,10 +309,12 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
             ga[q] = load_pair_raw<IO, EVEN>(g0, pos_of(q), L);
             gb[q] = load_pair_raw<IO, EVEN>(g1, pos_of(q), L);
         }
+        // the last read of the chunk's workspace releases it (evict_first)
+        const uint64_t pol = MODE == 2 ? l2_stream() : l2_keep();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int ad = (t1 + q * T1) * M2 + n2;     // k1 = t1 + q T1
-            const float2 f0 = w0[ad], f1 = w1[ad];
+            const float2 f0 = ld_pol(w0 + ad, pol), f1 = ld_pol(w1 + ad, pol);
             v[q] = c32x2{f2(f0.x, f1.x), f2(f0.y, f1.y)};
         }
         fft_cta<M1, E, +1, false, G::TWS, G::NCOL>(v, smem, nullptr, t1, tws, j);
@@ -313,12 +343,13 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
         const c32 base = ldg_c(a.f.tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
         const c32 step = ldg_c(a.f.tw + ((2 * (int64_t)n2 * T1) & (M - 1)));
         twiddle_powers<E, 1, 0>(v, step);
+        const uint64_t keep = l2_keep();
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const c32x2 r = mul(v[q], base);
             const int ad = (t1 + q * T1) * M2 + n2;
-            w0[ad] = make_float2(r.re.x, r.im.x);
-            if (has1) w1[ad] = make_float2(r.re.y, r.im.y);
+            st_pol(w0 + ad, make_float2(r.re.x, r.im.x), keep);
+            if (has1) st_pol(w1 + ad, make_float2(r.re.y, r.im.y), keep);
         }
     }
 }
@@ -350,12 +381,13 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged_rows_x2(const StagedArg
     auto st = [&](int ad, c32x2 x) { rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y); };
 
     // the group's rows of both lanes, coalesced, into the sequence-major buffer
+    const uint64_t keep = l2_keep(), stream = l2_stream();
 #pragma unroll
     for (int sl = 0; sl < NROW; ++sl) {
         const int64_t base = (int64_t)row_of_slot<G>(g, sl) * M2;
 #pragma unroll
         for (int k2 = threadIdx.x; k2 < M2; k2 += RT) {
-            const float2 f0 = w0[base + k2], f1 = w1[base + k2];
+            const float2 f0 = ld_pol(w0 + base + k2, keep), f1 = ld_pol(w1 + base + k2, keep);
             rowb[maddr<M2>(k2, sl)] = make_float4(f0.x, f1.x, f0.y, f1.y);
         }
     }
@@ -388,8 +420,8 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged_rows_x2(const StagedArg
         const c32x2 wO = mul(O2, w);
         const c32x2 Xk = add(E2, wO);
         const c32x2 Xm{f2sub(E2.re, wO.re), f2sub(wO.im, E2.im)};
-        const c32 hk0 = ldg_c(H0 + k), hk1 = ldg_c(H1 + k);
-        const c32 hm0 = ldg_c(H0 + (MC - k)), hm1 = ldg_c(H1 + (MC - k));
+        const c32 hk0 = ldc_pol(H0 + k, stream), hk1 = ldc_pol(H1 + k, stream);
+        const c32 hm0 = ldc_pol(H0 + (MC - k), stream), hm1 = ldc_pol(H1 + (MC - k), stream);
         const c32x2 Hk{f2(s * (hk0.x + dsk0), s * (hk1.x + dsk1)), f2(s * hk0.y, s * hk1.y)};
         const c32x2 Hm{f2(s * (hm0.x + dsk0), s * (hm1.x + dsk1)), f2(s * hm0.y, s * hm1.y)};
         const c32x2 Yk = mul(Xk, Hk), Ym = mul(Xm, Hm);
@@ -437,8 +469,8 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged_rows_x2(const StagedArg
 #pragma unroll
         for (int k2 = threadIdx.x; k2 < M2; k2 += RT) {
             const float4 f = rowb[maddr<M2>(k2, sl)];
-            w0[base_ad + k2] = make_float2(f.x, f.z);
-            if (has1) w1[base_ad + k2] = make_float2(f.y, f.w);
+            st_pol(w0 + base_ad + k2, make_float2(f.x, f.z), keep);
+            if (has1) st_pol(w1 + base_ad + k2, make_float2(f.y, f.w), keep);
         }
     }
 }
