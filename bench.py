@@ -176,11 +176,14 @@ def run_ours(args, w, rank, world, dist):
     y = torch.empty_like(v)
     ws_bytes = plan.workspace_bytes(w.B)
     # kernel launches per forward: one, except on the staged long-row path, which runs
-    # 2N + 1 launches (column, row, column, ...) per chunk of rows that fits the workspace
+    # 2N + 1 launches (column, row, column, ...) per chunk of rows; the workspace holds
+    # all rows (one chunk) or two chunks in flight
     launches = 1
     if ws_bytes:
-        chunk_rows = ws_bytes // ((plan.fft_len // 2) * 8)
-        launches = -(-(w.B * w.D) // chunk_rows) * (2 * w.order + 1)
+        rows = w.B * w.D
+        ws_rows = ws_bytes // ((plan.fft_len // 2) * 8)
+        chunks = 1 if ws_rows >= rows else -(-rows // (ws_rows // 2))
+        launches = chunks * (2 * w.order + 1)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()

@@ -9,23 +9,31 @@ using GS_32K = StagedGeom<32768, 128, 16, 8, 2>;   // M = 65536: columns of 128,
 using GS_64K = StagedGeom<65536, 256, 8, 8, 2>;    // M = 131072: 256 x 256
 
 int64_t staged_chunk_rows(int64_t MC) {
-    // rows whose transforms (MC complex64 each) fill 64 MB: most of a chunk stays
-    // in L2 between launches, and each launch spans several waves of CTAs
-    const int64_t r = ((int64_t)64 << 20) / (MC * 8);
+    // rows whose transforms (MC complex64 each) fill 32 MB; two chunks are in
+    // flight at a time (64 MB), which mostly stays in L2 between launches
+    const int64_t r = ((int64_t)32 << 20) / (MC * 8);
     return r < 1 ? 1 : r;
+}
+
+int64_t staged_workspace_rows(int64_t MC, int64_t rows) {
+    const int64_t r = staged_chunk_rows(MC);
+    return rows <= r ? rows : 2 * r;
 }
 
 bool staged_path_supported(int64_t MC) { return MC == 32768 || MC == 65536; }
 
+// Chunk c runs on lane c % nst (a stream of its own) with its own workspace
+// slot, so that two chunks' launch sequences overlap on the GPU.
 template <typename G, typename IO, bool EVEN>
-cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cudaStream_t st) {
+cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, const cudaStream_t *lanes, int nst) {
     static_assert(G::ROWS == 2, "the launch sequence below runs the lockstep kernels");
-    for (int64_t o0 = 0; o0 < f.rows; o0 += chunk) {
+    for (int64_t o0 = 0, c = 0; o0 < f.rows; o0 += chunk, ++c) {
         const int64_t nr = (f.rows - o0) < chunk ? (f.rows - o0) : chunk;
         const int64_t pairs = (nr + 1) / 2;
+        const cudaStream_t st = lanes[c % nst];
         StagedArgs a;
         a.f = f;
-        a.ws = ws;
+        a.ws = ws + (c % nst) * chunk * G::MC;
         a.o0 = o0;
         a.n = 0;
         const unsigned cgrid = (unsigned)(pairs * G::CGROUPS), rgrid = (unsigned)(pairs * G::RGROUPS);
@@ -46,21 +54,37 @@ cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cuda
 
 template <typename G>
 cudaError_t launch_staged_g(const Fwd1dArgs &f, float2 *ws, int64_t chunk, hyena_dtype_t dt, bool even,
-                            cudaStream_t st) {
+                            const cudaStream_t *lanes, int nst) {
     if (dt == HYENA_F32)
-        return even ? launch_staged_io<G, float, true>(f, ws, chunk, st) : launch_staged_io<G, float, false>(f, ws, chunk, st);
-    return even ? launch_staged_io<G, __nv_bfloat16, true>(f, ws, chunk, st)
-                : launch_staged_io<G, __nv_bfloat16, false>(f, ws, chunk, st);
+        return even ? launch_staged_io<G, float, true>(f, ws, chunk, lanes, nst)
+                    : launch_staged_io<G, float, false>(f, ws, chunk, lanes, nst);
+    return even ? launch_staged_io<G, __nv_bfloat16, true>(f, ws, chunk, lanes, nst)
+                : launch_staged_io<G, __nv_bfloat16, false>(f, ws, chunk, lanes, nst);
 }
 
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &f, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, const StagedLanes &sl) {
     const int64_t chunk = staged_chunk_rows(MC);
-    switch (MC) {
-        case 32768: return launch_staged_g<GS_32K>(f, ws, chunk, dt, even, st);
-        case 65536: return launch_staged_g<GS_64K>(f, ws, chunk, dt, even, st);
-        default: return cudaErrorInvalidValue;
+    auto run = [&](const cudaStream_t *lanes, int nst) -> cudaError_t {
+        switch (MC) {
+            case 32768: return launch_staged_g<GS_32K>(f, ws, chunk, dt, even, lanes, nst);
+            case 65536: return launch_staged_g<GS_64K>(f, ws, chunk, dt, even, lanes, nst);
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    if (f.rows <= chunk) return run(&st, 1);   // one chunk: the caller's stream only
+    // fork the two lanes off the caller's stream, join them back at the end
+    cudaError_t e = cudaEventRecord(sl.fork, st);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
+    if (e != cudaSuccess) return e;
+    const cudaError_t le = run(sl.lane, 2);
+    for (int i = 0; i < 2; ++i) {
+        // join even after a failed launch, so that the caller's stream never runs ahead of the lanes
+        e = cudaEventRecord(sl.join[i], sl.lane[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sl.join[i], 0);
+        if (e != cudaSuccess) return e;
     }
+    return le;
 }
 
 }  // namespace hyena

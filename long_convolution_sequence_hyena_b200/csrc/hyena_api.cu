@@ -37,6 +37,22 @@ std::vector<float2> twiddle_table(int64_t M) {
     return t;
 }
 
+// Destroy the staged path's streams and events (those that were created).
+bool release_lanes(hyena_plan_s *p) {
+    if (!p->has_lanes) return true;
+    bool ok = true;
+    for (int i = 0; i < 2; ++i) {
+        if (p->lane[i] && cudaStreamDestroy(p->lane[i]) != cudaSuccess) ok = false;
+        if (p->join[i] && cudaEventDestroy(p->join[i]) != cudaSuccess) ok = false;
+        p->lane[i] = nullptr;
+        p->join[i] = nullptr;
+    }
+    if (p->fork && cudaEventDestroy(p->fork) != cudaSuccess) ok = false;
+    p->fork = nullptr;
+    p->has_lanes = false;
+    return ok;
+}
+
 hyena_status_t check_device(const hyena_plan_s *p) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return HYENA_ERR_CUDA;
@@ -136,8 +152,22 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         cudaFree(p.tw);
         return HYENA_ERR_CUDA;
     }
+    if (p.path == HYENA_PATH_STAGED) {
+        bool ok = cudaStreamCreateWithFlags(&p.lane[0], cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&p.lane[1], cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.join[0], cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.join[1], cudaEventDisableTiming) == cudaSuccess;
+        p.has_lanes = true;
+        if (!ok) {
+            release_lanes(&p);
+            cudaFree(p.tw);
+            return HYENA_ERR_CUDA;
+        }
+    }
     hyena_plan_s *heap = new (std::nothrow) hyena_plan_s(p);
     if (!heap) {
+        release_lanes(&p);
         cudaFree(p.tw);
         return HYENA_ERR_NOMEM;
     }
@@ -149,6 +179,7 @@ hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     if (!plan) return HYENA_OK;
     hyena_status_t st = HYENA_OK;
     if (plan->tw && cudaFree(plan->tw) != cudaSuccess) st = HYENA_ERR_CUDA;
+    if (!release_lanes(plan)) st = HYENA_ERR_CUDA;
     delete plan;
     return st;
 }
@@ -164,9 +195,7 @@ hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spe
 size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch) {
     if (!plan || batch < 0) return 0;
     if (plan->path != HYENA_PATH_STAGED) return 0;
-    const int64_t rows = batch * plan->D;
-    const int64_t chunk = staged_chunk_rows(plan->MC);
-    return (size_t)(rows < chunk ? rows : chunk) * (size_t)plan->MC * sizeof(float2);
+    return (size_t)staged_workspace_rows(plan->MC, batch * plan->D) * (size_t)plan->MC * sizeof(float2);
 }
 
 hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_implicit_params_t *params, float *h_out,
@@ -266,10 +295,16 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     a.order = plan->order;
     const bool even = (plan->L % 2) == 0;
     cudaError_t e;
-    if (plan->path == HYENA_PATH_STAGED)
+    if (plan->path == HYENA_PATH_STAGED) {
+        StagedLanes lanes;
+        lanes.lane[0] = plan->lane[0];
+        lanes.lane[1] = plan->lane[1];
+        lanes.fork = plan->fork;
+        lanes.join[0] = plan->join[0];
+        lanes.join[1] = plan->join[1];
         e = launch_fwd_1d_staged(a, plan->MC, reinterpret_cast<float2 *>(workspace), plan->dtype, even,
-                                 (cudaStream_t)stream);
-    else if (plan->path == HYENA_PATH_CLUSTER)
+                                 (cudaStream_t)stream, lanes);
+    } else if (plan->path == HYENA_PATH_CLUSTER)
         e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     else if (pair_path_supported(plan->MC, batch))
         e = launch_fwd_1d_pair(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);

@@ -21,11 +21,17 @@ cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t 
 cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
                                    const c32 *tw, cudaStream_t st);
 // 1D, staged four-step through a workspace (MC in {32768, 65536}); chunks of
-// staged_chunk_rows(MC) rows, workspace chunk * MC complex64
+// staged_chunk_rows(MC) rows, two in flight on the plan's lanes; workspace
+// staged_workspace_rows(MC, rows) * MC complex64
+struct StagedLanes {
+    cudaStream_t lane[2];     // non-blocking streams owned by the plan
+    cudaEvent_t fork, join[2];
+};
 bool staged_path_supported(int64_t MC);
 int64_t staged_chunk_rows(int64_t MC);
+int64_t staged_workspace_rows(int64_t MC, int64_t rows);
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &a, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
-                                 cudaStream_t st);
+                                 cudaStream_t st, const StagedLanes &lanes);
 // 2D, one cluster per plane (H == W in {32, 64, 128, 256})
 struct Fwd2dArgs;
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);

@@ -26,4 +26,9 @@ struct hyena_plan_s {
     // device tables (owned)
     int64_t tw_len = 0;          // 1D: M; 2D: 2W
     float2 *tw = nullptr;        // W_tw_len^m, m in [0, tw_len), then W_1024^m, m in [0, 1024)
+    // staged path: two non-blocking streams and the events that fork them off
+    // and join them back to the caller's stream
+    bool has_lanes = false;
+    cudaStream_t lane[2] = {nullptr, nullptr};
+    cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
 };
