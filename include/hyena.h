@@ -65,7 +65,8 @@ typedef enum {
 typedef enum {
     HYENA_PATH_CTA = 0,          /* 1D, M <= 32768: one CTA per row, all orders fused */
     HYENA_PATH_CLUSTER = 1,      /* 1D, M = 262144: a thread-block cluster per row */
-    HYENA_PATH_2D = 2,           /* 2D grid */
+    HYENA_PATH_2D = 2,           /* 2D grid (H = W = 256: column and row kernels through a workspace;
+                                    smaller grids: a thread-block cluster per plane) */
     HYENA_PATH_STAGED = 3        /* 1D, M in {65536, 131072}: column and row kernels per order,
                                     the row's transform in a device workspace */
 } hyena_path_t;
@@ -124,9 +125,11 @@ HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);
 HYENA_API hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path);
 
 /*
- * Bytes of device workspace hyena_forward needs for `batch`: 0 except on
- * HYENA_PATH_STAGED, where rows run in chunks that keep their transforms in
- * L2, and the workspace holds one chunk: min(batch * D, chunk) * (M/2) * 8 bytes.
+ * Bytes of device workspace hyena_forward needs for `batch`. It is 0, except
+ * on HYENA_PATH_STAGED and on 2D plans with H = W = 256. There, rows (planes)
+ * run in chunks that keep their transforms in L2, with two chunks in flight.
+ * The workspace then holds min(rows, 2 * chunk) transforms: (M/2) * 8 bytes
+ * per 1D row, 2H * (W/2) * 8 bytes per plane.
  */
 HYENA_API size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch);
 
@@ -186,8 +189,7 @@ HYENA_API const char *hyena_status_string(hyena_status_t status);
  * staged path's scratch lives, not what is computed.
  *
  * Plans on HYENA_PATH_STAGED only (1D, M in {65536, 131072}); any other plan
- * returns HYENA_ERR_UNSUPPORTED (those paths need no workspace: call
- * hyena_forward with workspace NULL). The other arguments are those of
+ * returns HYENA_ERR_UNSUPPORTED. The other arguments are those of
  * hyena_forward, and so is the result.
  *
  * The scratch is one array of HYENA_STATIC_SCRATCH_BYTES in device memory,

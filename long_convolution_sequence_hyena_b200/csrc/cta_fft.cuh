@@ -33,14 +33,15 @@ namespace hyena {
 // NSW: the number of sequences a warp spans at a common i. With 16 or more,
 // each half-warp holds 16 sequences and XOR-ing the sequence index into i
 // puts them on distinct 8-byte bank pairs. With 8, each half-warp holds 8
-// sequences at two elements i, i' that differ in bit 0 or in bit 3 (every
-// Stockham pattern of radix-8 passes); XOR-ing 2s into bits 1..3 and bit 3
-// of i into bit 0 separates them.
+// sequences at two elements i, i' that differ in one bit among bits 0..4
+// (every Stockham pattern of radix-8 and radix-16 passes): XOR-ing 2s into
+// bits 1..3 and the parity of bits 1..4 of i into bit 0 separates them
+// (checked on the CPU for lengths 64..512).
 template <int LEN, int NSW = 32>
 __device__ __forceinline__ int maddr(int i, int s) {
     static_assert(NSW == 8 || NSW >= 16, "sequence-major layout needs 8 or at least 16 sequences per warp");
     if constexpr (NSW >= 16) return s * LEN + (i ^ (s & 31));
-    else return s * LEN + (i ^ (((2 * s) & 15) | ((i >> 3) & 1)));
+    else return s * LEN + (i ^ (((2 * s) & 15) | (__popc((i >> 1) & 15) & 1)));
 }
 
 // Shared-memory element of a value type in the sequence-major layout: one

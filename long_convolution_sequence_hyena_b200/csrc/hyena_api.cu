@@ -152,7 +152,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         cudaFree(p.tw);
         return HYENA_ERR_CUDA;
     }
-    if (p.path == HYENA_PATH_STAGED) {
+    if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
         bool ok = cudaStreamCreateWithFlags(&p.lane[0], cudaStreamNonBlocking) == cudaSuccess &&
                   cudaStreamCreateWithFlags(&p.lane[1], cudaStreamNonBlocking) == cudaSuccess &&
                   cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess &&
@@ -194,6 +194,9 @@ hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spe
 
 size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch) {
     if (!plan || batch < 0) return 0;
+    if (plan->path == HYENA_PATH_2D && staged2d_supported(plan->Ww))
+        return (size_t)staged2d_workspace_planes(plan->Ww, batch * plan->D) * (size_t)(2 * plan->Hh) *
+               (size_t)(plan->Ww / 2) * sizeof(float2);
     if (plan->path != HYENA_PATH_STAGED) return 0;
     return (size_t)staged_workspace_rows(plan->MC, batch * plan->D) * (size_t)plan->MC * sizeof(float2);
 }
@@ -278,7 +281,20 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
         a.C = plan->D;
         a.B = batch;
         a.order = plan->order;
-        return launch_fwd_2d(a, plan->Ww, plan->dtype, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+        cudaError_t e2;
+        if (staged2d_supported(plan->Ww)) {
+            StagedLanes lanes;
+            lanes.lane[0] = plan->lane[0];
+            lanes.lane[1] = plan->lane[1];
+            lanes.fork = plan->fork;
+            lanes.join[0] = plan->join[0];
+            lanes.join[1] = plan->join[1];
+            e2 = launch_fwd_2d_staged(a, plan->Ww, reinterpret_cast<float2 *>(workspace), plan->dtype,
+                                      (cudaStream_t)stream, lanes);
+        } else {
+            e2 = launch_fwd_2d(a, plan->Ww, plan->dtype, (cudaStream_t)stream);
+        }
+        return e2 == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
     }
     Fwd1dArgs a;
     std::memset(&a, 0, sizeof(a));

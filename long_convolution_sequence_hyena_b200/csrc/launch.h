@@ -32,6 +32,14 @@ int64_t staged_chunk_rows(int64_t MC);
 int64_t staged_workspace_rows(int64_t MC, int64_t rows);
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &a, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
                                  cudaStream_t st, const StagedLanes &lanes);
+// 2D staged (H = W = 256): chunks of staged2d_chunk_planes(W) planes, two in flight;
+// workspace staged2d_workspace_planes(W, planes) * 2H * W/2 complex64
+struct Fwd2dArgs;
+bool staged2d_supported(int64_t W);
+int64_t staged2d_chunk_planes(int64_t W);
+int64_t staged2d_workspace_planes(int64_t W, int64_t planes);
+cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyena_dtype_t dt, cudaStream_t st,
+                                 const StagedLanes &lanes);
 // 2D, one cluster per plane (H == W in {32, 64, 128, 256})
 struct Fwd2dArgs;
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);
