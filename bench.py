@@ -259,7 +259,8 @@ def run_ours(args, w, rank, world, dist):
 # ------------------------------------------------------------ oracle (CPU)
 def oracle_runner(w):
     """Prepare the fp64 oracle on rows (planes) of the workload's recipe.
-    Returns (run(rows) -> None, elements per row, threads)."""
+    Returns (run(rows) -> None, elements per row, threads, distinct rows); run(rows)
+    evaluates `rows` rows, cycling over the distinct rows drawn."""
     import numpy as np
 
     import oracle
@@ -302,7 +303,7 @@ def oracle_runner(w):
             idx = np.arange(rows) % small.D
             oracle.hyena_2d(v[idx], g[:, idx], k64, d, fidx=idx)
         unit = H * W
-    return run, unit, threads
+    return run, unit, threads, small.D
 
 
 def calibrate_rows(run, threads, seconds):
@@ -322,19 +323,21 @@ def calibrate_rows(run, threads, seconds):
 def oracle_sample(w, seconds):
     """Time the fp64 oracle on a bounded sample of the workload's rows (planes).
     Returns (elements/s, sample description, threads, seconds)."""
-    run, unit, threads = oracle_runner(w)
+    run, unit, threads, distinct = oracle_runner(w)
     rows = calibrate_rows(run, threads, seconds)
     t0 = time.perf_counter()
     run(rows)
     dt = time.perf_counter() - t0
-    return rows * unit / dt, "%d rows of the workload (%d elements each), direct fp64 sum" % (rows, unit), threads, dt
+    what = "%d row evaluations (cycling over %d rows drawn with the workload's recipe; %d elements each), " \
+           "direct fp64 sum" % (rows, distinct, unit)
+    return rows * unit / dt, what, threads, dt
 
 
 def run_reference(args, w):
     """The reference arm: the oracle as it stands, W warm-up and K timed steps,
     each step a bounded sample of the workload's rows (sized so the whole run
     takes about two minutes)."""
-    run, unit, threads = oracle_runner(w)
+    run, unit, threads, distinct = oracle_runner(w)
     per_step = max(0.5, 120.0 / (args.steps + args.warmup))
     rows = calibrate_rows(run, threads, per_step)
     for _ in range(args.warmup):
@@ -345,7 +348,8 @@ def run_reference(args, w):
         run(rows)
         times.append(time.perf_counter() - t0)
     value = rows * unit * len(times) / sum(times)
-    sample = "%d rows of the workload (%d elements each) per step, direct fp64 sum" % (rows, unit)
+    sample = "%d row evaluations per step (cycling over %d rows drawn with the workload's recipe; " \
+             "%d elements each), direct fp64 sum" % (rows, distinct, unit)
     return value, sample, threads
 
 
