@@ -248,12 +248,33 @@ def run_ours(args, w, rank, world, dist):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dist, dev)
+    # implicit filters: also time the filter network and its spectrum with the
+    # forward, per step (filters regenerated every step, as in training)
+    filt_ms = 0.0
+    if "implicit" in inp:
+        def filt_step():
+            plan.filter_spectrum(implicit=imp, out=H, stream=stream)
+            step()
+        for _ in range(args.warmup):
+            flush.zero_()
+            filt_step()
+        torch.cuda.synchronize()
+        fs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            fs[i].record(stream)
+            filt_step()
+            fe[i].record(stream)
+        torch.cuda.synchronize()
+        filt_ms = sum(a.elapsed_time(b) for a, b in zip(fs, fe)) / args.steps
+
+    ms, e2e_ms, filt_ms = max_over_ranks([ms, e2e_ms, filt_ms], dist, dev)
     io = 4 if w.dtype == "f32" else 2
     h2d = (w.order + 1) * w.elements * io
     d2h = w.elements * io
     plan.close()
-    return ms, step_ms, e2e_ms, h2d, d2h, clk, launches
+    return ms, step_ms, e2e_ms, h2d, d2h, clk, launches, filt_ms
 
 
 # ------------------------------------------------------------ oracle (CPU)
@@ -386,7 +407,7 @@ def main():
         import torch.distributed as dist_mod
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
-    ms, step_ms, e2e_ms, h2d, d2h, clk, launches = run_ours(args, w, rank, world, dist)
+    ms, step_ms, e2e_ms, h2d, d2h, clk, launches, filt_ms = run_ours(args, w, rank, world, dist)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
@@ -428,6 +449,11 @@ def main():
         "clocks": clk,
         "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
     }
+    if filt_ms > 0:
+        # the same metric with the implicit filter network and the filter spectra
+        # computed inside every step (the operator as used in training)
+        line["with_filter_generation"] = {"value": job_throughput(w.elements, world, filt_ms), "unit": "elems/s",
+                                          "ms_per_step": filt_ms}
     if world == 1 and not args.no_cpu_baseline:
         cv, sample, threads, _ = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": cv, "unit": "elems/s", "cores": threads, "kind": "oracle", "sample": sample}
