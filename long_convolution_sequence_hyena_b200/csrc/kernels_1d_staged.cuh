@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
 }
 
 template <typename G>
-__global__ void __launch_bounds__(G::RT, 3) hyena_staged_rows_x2(const StagedArgs a, int64_t nr) {
+__global__ void __launch_bounds__(G::RT, 4) hyena_staged_rows_x2(const StagedArgs a, int64_t nr) {
     static_assert(G::ROWS == 2, "lockstep geometry");
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, MC = G::MC, M = 2 * MC;
     constexpr int NROW = G::NROW, HROW = G::HROW, RT = G::RT;

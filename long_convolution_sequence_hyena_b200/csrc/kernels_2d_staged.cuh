@@ -58,7 +58,7 @@ __device__ __forceinline__ int64_t visit_plane(const Fwd2dArgs &f, int64_t o, in
 // MODE 0: load v, forward columns; 1: inverse columns, gate x^n, forward
 // columns; 2: inverse columns, gate x^n, store y.
 template <typename G, typename IO, int MODE>
-__global__ void __launch_bounds__(G::CT, 2) hyena_staged2d_cols(const Staged2dArgs a) {
+__global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dArgs a) {
     constexpr int E = G::E, M1 = G::M1, XW = G::XW, T1 = G::T1, Hh = G::Hh, Ww = G::Ww;
     extern __shared__ float smem[];
     const int64_t lp = blockIdx.x / G::CGROUPS;      // plane within the chunk
