@@ -9,11 +9,11 @@
 //   features of offset (oy, ox): (oy/H, ox/W), oy in [-H, H), ox in [-W, W)
 //   window: exp(-(py^2 + px^2) / (2 sigma[o]^2))
 //
-// One CTA per tile of IMP_TP positions and one slice of the outputs. The two
-// hidden layers of the tile are computed once into shared memory. The head
-// is a dense contraction out[o][p] = sum_j W3[o][j] a2[j][p]; it is computed
-// as a register-blocked tiled product (each thread a 4-output x 4-position
-// block), with the W3 tile staged in shared memory.
+// One CTA per tile of IMP_TP positions and one slice of the outputs. Every
+// layer is a dense contraction out[j][p] = sum_k W[j][k] in[k][p] over the
+// tile's positions, computed as a register-blocked tiled product: each thread
+// takes a 4-row x 4-position block of a 64 x 64 tile, with the weight tile in
+// shared memory and the activations stored [unit][position].
 #pragma once
 #include "hyena.h"
 
@@ -39,15 +39,10 @@ struct ImplicitArgs {
 };
 
 struct ImplicitSmem {
-    float a2[IMP_MAXW][IMP_TP];        // second hidden layer, [unit][position]
-    union {
-        struct {
-            float feat[IMP_TP][IMP_MAXF + 1];
-            float h1[IMP_TP][IMP_MAXW + 1];
-        } in;                           // dead once a2 is complete
-        float w3[IMP_OT][IMP_MAXW + 4];    // head weight tile, [output][unit]
-    } u;
+    float act[2][IMP_MAXW][IMP_TP];     // activations [unit][position]; act[1] first holds the features
+    float wt[IMP_OT][IMP_MAXW + 4];     // weight tile [row][input] (a layer's 64 rows at a time)
 };
+static_assert(IMP_MAXF <= IMP_MAXW, "features are staged in an activation buffer");
 
 // Defined in implicit_filter.cu (one translation unit).
 __global__ void hyena_implicit_filter_kernel(const ImplicitArgs a);
