@@ -181,7 +181,9 @@ def run_ours(args, w, rank, world, dist):
     launches = 1
     if ws_bytes:
         rows = w.B * w.D
-        ws_rows = ws_bytes // ((plan.fft_len // 2) * 8)
+        # one row's (plane's) transform: M/2 complex64 in 1D, 2H x W/2 complex64 in 2D
+        per_row = (plan.fft_len // 2) * 8 if w.ndim == 1 else (2 * w.shape[0]) * (w.shape[1] // 2) * 8
+        ws_rows = ws_bytes // per_row
         chunks = 1 if ws_rows >= rows else -(-rows // (ws_rows // 2))
         launches = chunks * (2 * w.order + 1)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)

@@ -142,7 +142,7 @@ def test_2d_spectrum_matches_dft(api, Hw):
 
 @pytest.mark.parametrize("Hw,B,C,N,dtype", [(32, 2, 3, 1, "f32"), (32, 1, 2, 2, "f32"), (64, 2, 2, 1, "f32"),
                                             (64, 1, 3, 2, "bf16"), (128, 1, 2, 1, "f32"), (128, 1, 2, 2, "bf16"),
-                                            (256, 1, 2, 1, "f32")])
+                                            (256, 1, 2, 1, "f32"), (256, 3, 1, 2, "bf16")])
 def test_2d_parity(api, Hw, B, C, N, dtype):
     w = explicit_case_2d(B, C, Hw, N, dtype, seed=900 + Hw + N)
     inp = make_inputs(w)
