@@ -29,11 +29,9 @@ namespace cg = cooperative_groups;
 
 // MINB: CTAs resident per SM (the launch bounds); with 2, one cluster's
 // barrier waits are covered by another cluster's work on the same SMs.
-// ROWS: rows per cluster, 1 (complex values) or 2 (two rows in lockstep as
-// c32x2: every shared element is 16 bytes).
-template <int MC_, int C_, int M1_, int E_, int MINB_ = 1, int ROWS_ = 1>
+template <int MC_, int C_, int M1_, int E_, int MINB_ = 1>
 struct ClusterGeom {
-    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_, MINB = MINB_, ROWS = ROWS_;
+    static constexpr int MC = MC_, C = C_, M1 = M1_, M2 = MC_ / M1_, E = E_, MINB = MINB_;
     static constexpr int NCOL = M2 / C;          // columns per CTA (column phase)
     static constexpr int NROW = M1 / C;          // rows per CTA (row phase), in mirror pairs
     static constexpr int HROW = NROW / 2;        // rows k1 < M1/2 per CTA
@@ -42,9 +40,8 @@ struct ClusterGeom {
     static constexpr int THREADS = NCOL * T1;
     static constexpr int PER_CTA = MC / C;       // complex elements per CTA per buffer
     // column buffer + row buffer + staging for one order's gates (E/2 element pairs per thread and row)
-    static constexpr size_t GATE_STAGE = (size_t)THREADS * (E / 2) * 8 * ROWS;
-    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8 * ROWS + GATE_STAGE;
-    static_assert(ROWS == 1 || ROWS == 2, "one row or a lockstep pair per cluster");
+    static constexpr size_t GATE_STAGE = (size_t)THREADS * (E / 2) * 8;
+    static constexpr size_t SMEM = 2 * (size_t)PER_CTA * 8 + GATE_STAGE;
     static_assert(THREADS == NROW * T2, "both phases must use the same thread count");
     static_assert(NCOL >= 16 && NROW >= 16, "warps must span at least 16 sequences");
     static_assert(M1 >= 32 && M2 >= 32, "sequence-major layouts need sequences of at least 32");
@@ -63,11 +60,6 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t local, int rank) {
 }
 __device__ __forceinline__ void dsmem_st(uint32_t addr, c32 v) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
-}
-__device__ __forceinline__ void dsmem_st(uint32_t addr, c32x2 v) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.re.x), "f"(v.re.y),
-                 "f"(v.im.x), "f"(v.im.y)
-                 : "memory");
 }
 // Cluster barrier that also orders shared::cluster memory (release / acquire).
 __device__ __forceinline__ void cluster_sync_mem() {
@@ -108,11 +100,11 @@ __device__ __forceinline__ void slot_of_row(int k1, int &c, int &r) {
 // sent, and the M2/2 data columns are spread over all C CTAs (NCOLP = NCOL/2
 // per CTA, twice the threads per column, E/2 values per thread), so that no
 // CTA idles through the column phase.
-template <typename G, bool TWID, bool HALFX, typename V = c32>
+template <typename G, bool TWID, bool HALFX>
 struct ClusterCtx {
-    using SE = selem<V>;
-    using ET = typename SE::T;
-    static_assert(sizeof(ET) == 8 * G::ROWS, "value type must match the geometry's rows per cluster");
+    using V = c32;
+    using SE = selem<c32>;
+    using ET = float2;
     static constexpr int NCOLP = HALFX ? G::NCOL / 2 : G::NCOL;   // columns per CTA, column phase
     static constexpr int T1P = G::THREADS / NCOLP;                // threads per column FFT
     static constexpr int E1 = G::M1 / T1P;                        // values per thread, column phase
