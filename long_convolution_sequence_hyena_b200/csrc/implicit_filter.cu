@@ -3,8 +3,9 @@
 
 namespace hyena {
 
-// Thread (ty, tx) accumulates rows 4 ty..4 ty+3 of the weight tile (leading
-// dimension IMP_MAXW + 4) against positions 4 tx..4 tx+3 of in[k][IMP_TP].
+// Thread (ty, tx) accumulates rows 4 ty..4 ty+3 of the weight tile (stored
+// [input][row]) against positions 4 tx..4 tx+3 of in[k][IMP_TP]: per input k,
+// one 16-byte load of weights and one of activations feed 16 FMAs.
 __device__ __forceinline__ void tile_product(const ImplicitSmem &S, const float (*in)[IMP_TP], int K, int tx, int ty,
                                              float (&acc)[4][4]) {
 #pragma unroll
@@ -14,13 +15,14 @@ __device__ __forceinline__ void tile_product(const ImplicitSmem &S, const float 
 #pragma unroll 4
     for (int k = 0; k < K; ++k) {
         const float4 b = *reinterpret_cast<const float4 *>(&in[k][4 * tx]);
+        const float4 w4 = *reinterpret_cast<const float4 *>(&S.wt[k][4 * ty]);
+        const float wr[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const float w = S.wt[4 * ty + r][k];
-            acc[r][0] = fmaf(w, b.x, acc[r][0]);
-            acc[r][1] = fmaf(w, b.y, acc[r][1]);
-            acc[r][2] = fmaf(w, b.z, acc[r][2]);
-            acc[r][3] = fmaf(w, b.w, acc[r][3]);
+            acc[r][0] = fmaf(wr[r], b.x, acc[r][0]);
+            acc[r][1] = fmaf(wr[r], b.y, acc[r][1]);
+            acc[r][2] = fmaf(wr[r], b.z, acc[r][2]);
+            acc[r][3] = fmaf(wr[r], b.w, acc[r][3]);
         }
     }
 }
@@ -29,8 +31,8 @@ __device__ __forceinline__ void tile_product(const ImplicitSmem &S, const float 
 __device__ __forceinline__ void load_weight_tile(ImplicitSmem &S, const float *__restrict__ W, int64_t j0, int64_t J,
                                                  int K, int tid) {
     for (int i = tid; i < IMP_OT * K; i += IMP_THREADS) {
-        const int r = i / K, k = i - r * K;
-        S.wt[r][k] = j0 + r < J ? __ldg(W + (j0 + r) * K + k) : 0.f;
+        const int r = i / K, k = i - r * K;   // coalesced reads along k
+        S.wt[k][r] = j0 + r < J ? __ldg(W + (j0 + r) * K + k) : 0.f;
     }
 }
 

@@ -40,7 +40,7 @@ struct ImplicitArgs {
 
 struct ImplicitSmem {
     float act[2][IMP_MAXW][IMP_TP];     // activations [unit][position]; act[1] first holds the features
-    float wt[IMP_OT][IMP_MAXW + 4];     // weight tile [row][input] (a layer's 64 rows at a time)
+    float wt[IMP_MAXW][IMP_OT + 4];     // weight tile, transposed: [input][row] (a layer's 64 rows at a time)
 };
 static_assert(IMP_MAXF <= IMP_MAXW, "features are staged in an activation buffer");
 
