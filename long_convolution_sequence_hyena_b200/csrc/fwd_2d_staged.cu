@@ -48,6 +48,53 @@ cudaError_t launch_staged2d_io(const Fwd2dArgs &f, float2 *ws, int64_t chunk, co
     return cudaSuccess;
 }
 
+int64_t staged2d_spec_chunk(int64_t W) { return W == 256 ? 16 : 0; }
+
+size_t staged2d_spec_scratch_bytes(int64_t W) {
+    return W == 256 ? (size_t)2 * staged2d_spec_chunk(W) * (2 * W) * W * sizeof(float2) : 0;
+}
+
+cudaError_t launch_spec_2d_staged(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W,
+                                  const c32 *tw, float2 *scratch, cudaStream_t st, const StagedLanes &sl) {
+    using G = GS2_256;
+    if (W != 256) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(hyena_staged2d_spec_rows_x2<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)G::RSMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t chunk = staged2d_spec_chunk(W);
+    const int64_t per = (int64_t)G::M1 * G::M2;
+    auto run = [&](const cudaStream_t *lanes, int nst) -> cudaError_t {
+        for (int64_t o0 = 0, c = 0; o0 < n; o0 += chunk, ++c) {
+            Spec2dArgs a;
+            a.K = K;
+            a.rs = rs;
+            a.cs = cs;
+            a.Kout = Kout;
+            a.tw = tw;
+            a.ws = scratch + (c % nst) * chunk * per;
+            a.o0 = o0;
+            a.nk = (n - o0) < chunk ? (n - o0) : chunk;
+            const cudaStream_t s = lanes[c % nst];
+            hyena_staged2d_spec_cols<G><<<(unsigned)(a.nk * (G::M2 / G::NCOL)), G::CT, G::CSMEM, s>>>(a);
+            hyena_staged2d_spec_rows_x2<G><<<(unsigned)((a.nk + 1) / 2 * G::RGROUPS), G::RT, G::RSMEM, s>>>(a);
+            const cudaError_t le = cudaGetLastError();
+            if (le != cudaSuccess) return le;
+        }
+        return cudaSuccess;
+    };
+    if (n <= chunk) return run(&st, 1);
+    e = cudaEventRecord(sl.fork, st);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
+    if (e != cudaSuccess) return e;
+    const cudaError_t le = run(sl.lane, 2);
+    for (int i = 0; i < 2; ++i) {
+        e = cudaEventRecord(sl.join[i], sl.lane[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sl.join[i], 0);
+        if (e != cudaSuccess) return e;
+    }
+    return le;
+}
+
 cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyena_dtype_t dt, cudaStream_t st,
                                  const StagedLanes &sl) {
     if (W != 256) return cudaErrorInvalidValue;

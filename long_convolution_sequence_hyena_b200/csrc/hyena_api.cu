@@ -165,9 +165,18 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
             return HYENA_ERR_CUDA;
         }
     }
+    if (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww)) {
+        if (cudaMalloc(&p.spec_ws, staged2d_spec_scratch_bytes(p.Ww)) != cudaSuccess) {
+            cudaGetLastError();
+            release_lanes(&p);
+            cudaFree(p.tw);
+            return HYENA_ERR_NOMEM;
+        }
+    }
     hyena_plan_s *heap = new (std::nothrow) hyena_plan_s(p);
     if (!heap) {
         release_lanes(&p);
+        if (p.spec_ws) cudaFree(p.spec_ws);
         cudaFree(p.tw);
         return HYENA_ERR_NOMEM;
     }
@@ -180,6 +189,7 @@ hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     hyena_status_t st = HYENA_OK;
     if (plan->tw && cudaFree(plan->tw) != cudaSuccess) st = HYENA_ERR_CUDA;
     if (!release_lanes(plan)) st = HYENA_ERR_CUDA;
+    if (plan->spec_ws && cudaFree(plan->spec_ws) != cudaSuccess) st = HYENA_ERR_CUDA;
     delete plan;
     return st;
 }
@@ -247,7 +257,17 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
             src = reinterpret_cast<const float *>(H_out);
         }
-        e = launch_spec_2d(src, rs, cs, Hc, nrows, plan->Ww, tw, st);
+        if (plan->spec_ws) {
+            StagedLanes lanes;
+            lanes.lane[0] = plan->lane[0];
+            lanes.lane[1] = plan->lane[1];
+            lanes.fork = plan->fork;
+            lanes.join[0] = plan->join[0];
+            lanes.join[1] = plan->join[1];
+            e = launch_spec_2d_staged(src, rs, cs, Hc, nrows, plan->Ww, tw, plan->spec_ws, st, lanes);
+        } else {
+            e = launch_spec_2d(src, rs, cs, Hc, nrows, plan->Ww, tw, st);
+        }
     }
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }

@@ -233,4 +233,112 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged2d_rows_x2(const Staged2
     }
 }
 
+// ---------------------------------------------------------------------------
+// 2D kernel spectra through the same two stages. The kernel on the offset grid
+// is placed cyclically (offset o at index o mod 2H, o mod 2W), packed along x
+// and transformed; every column and row carries data. The plan owns the
+// scratch ([M1][M2] complex64 per kernel), so the spectrum may be computed in
+// place: a chunk's column kernel reads all of its kernels before its row
+// kernel writes their spectra.
+
+struct Spec2dArgs {
+    const float *K;    // kernel (n, c) at K + o * cs; row iy at + iy * rs, 2W floats (ox = ix - W)
+    int64_t rs, cs;
+    c32 *Kout;         // [W + 1][2H] complex per kernel, bin (ky, kx) at kx * 2H + ky
+    const c32 *tw;     // W_{2W}, then W_1024
+    float2 *ws;        // chunk kernels x [M1][M2]
+    int64_t o0;        // first kernel of the chunk
+    int64_t nk;        // kernels in the chunk
+};
+
+template <typename G>
+__global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_spec_cols(const Spec2dArgs a) {
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T1 = G::T1, Hh = G::Hh, Ww = G::Ww;
+    constexpr int CG = M2 / G::NCOL;                   // column groups: every column carries data
+    extern __shared__ float smem[];
+    const int64_t lk = blockIdx.x / CG;
+    const int cgp = blockIdx.x % CG;
+    const int j = threadIdx.x % G::NCOL, t1 = threadIdx.x / G::NCOL;
+    const int xc = cgp * G::NCOL + j;
+    const float *Kp = a.K + (a.o0 + lk) * a.cs;
+    float2 *wp = a.ws + lk * (int64_t)M1 * M2;
+    const int ix = (2 * xc + Ww) & (2 * Ww - 1);      // cyclic column 2 x' -> offset-grid column
+    c32 v[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int iy = (t1 + q * T1 + Hh) & (M1 - 1);
+        const float *rowp = Kp + iy * a.rs;
+        v[q] = mk(rowp[ix], rowp[ix + 1]);
+    }
+    fft_cta<M1, E, -1, false, G::TWS, G::NCOL>(v, smem, nullptr, t1, a.tw + 2 * M2, j);
+    const uint64_t keep = l2_keep();
+#pragma unroll
+    for (int q = 0; q < E; ++q) st_pol(wp + (t1 + q * T1) * M2 + xc, make_float2(v[q].x, v[q].y), keep);
+}
+
+template <typename G>
+__global__ void __launch_bounds__(G::RT, 3) hyena_staged2d_spec_rows_x2(const Spec2dArgs a) {
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, RT = G::RT;
+    constexpr int NROW = G::NROW, HROW = G::HROW;
+    extern __shared__ float smem[];
+    float4 *rowb = reinterpret_cast<float4 *>(smem);
+    const int64_t lp = blockIdx.x / G::RGROUPS;      // kernel pair within the chunk
+    const int g = blockIdx.x % G::RGROUPS;
+    const int r = threadIdx.x % NROW, t2 = threadIdx.x / NROW;
+    const int ky = row_of_slot<G>(g, r);
+    const int rm = (ky == 0 || ky == M1 / 2) ? r : (r < HROW ? r + HROW : r - HROW);
+    const int kym = (M1 - ky) & (M1 - 1);
+    const bool has1 = 2 * lp + 1 < a.nk;
+    const float2 *w0 = a.ws + (2 * lp) * (int64_t)M1 * M2;
+    const float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * (int64_t)M1 * M2;
+    auto ld = [&](int ad) -> c32x2 {
+        const float4 f = rowb[ad];
+        return c32x2{f2(f.x, f.y), f2(f.z, f.w)};
+    };
+    const uint64_t stream = l2_stream();              // the scratch is read once
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl) {
+        const int64_t base = (int64_t)row_of_slot<G>(g, sl) * M2;
+#pragma unroll
+        for (int x = threadIdx.x; x < M2; x += RT) {
+            const float2 f0 = ld_pol(w0 + base + x, stream), f1 = ld_pol(w1 + base + x, stream);
+            rowb[maddr<M2>(x, sl)] = make_float4(f0.x, f1.x, f0.y, f1.y);
+        }
+    }
+    __syncthreads();
+    c32x2 v[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = ld(maddr<M2>(t2 + q * T2, r));
+    __syncthreads();
+    fft_cta<M2, E, -1, false, G::TWS, NROW>(v, smem, nullptr, t2, a.tw + 2 * M2, r);
+#pragma unroll
+    for (int q = 0; q < E; ++q) rowb[maddr<M2>(t2 + q * T2, r)] = make_float4(v[q].re.x, v[q].re.y, v[q].im.x, v[q].im.y);
+    __syncthreads();
+    // unpack along x: X(ky, kx) = E + W_{2 M2}^{kx} O with the mirror bin (-ky, -kx); bin
+    // (-ky, M2) (the Nyquist column) is conj(E - W O) of kx = 0
+    const c32 wb = ldg_c(a.tw + t2);
+    c32 *K0 = a.Kout + (a.o0 + 2 * lp) * (int64_t)M1 * (M2 + 1);
+    c32 *K1 = a.Kout + (a.o0 + 2 * lp + (has1 ? 1 : 0)) * (int64_t)M1 * (M2 + 1);
+    const int z0 = opaque_zero();
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int kx = t2 + q * T2;
+        const c32x2 Zk = v[q];
+        const c32x2 Zm = ld(maddr<M2>((M2 - kx) & (M2 - 1), rm));
+        const c32x2 E2{f2add(Zk.re, Zm.re), f2sub(Zk.im, Zm.im)};   // 2E
+        const c32x2 O2{f2add(Zk.im, Zm.im), f2sub(Zm.re, Zk.re)};   // 2O
+        const c32x2 wO = mul(O2, mul(wb, w2e<E>(q, z0)));
+        const c32x2 X{f2mul(f2add(E2.re, wO.re), f2(0.5f, 0.5f)), f2mul(f2add(E2.im, wO.im), f2(0.5f, 0.5f))};
+        const int64_t ak = (int64_t)kx * M1 + ky;
+        K0[ak] = mk(X.re.x, X.im.x);
+        if (has1) K1[ak] = mk(X.re.y, X.im.y);
+        if (kx == 0) {
+            const c32x2 N{f2mul(f2sub(E2.re, wO.re), f2(0.5f, 0.5f)), f2mul(f2sub(wO.im, E2.im), f2(0.5f, 0.5f))};
+            const int64_t an = (int64_t)M2 * M1 + kym;
+            K0[an] = mk(N.re.x, N.im.x);
+            if (has1) K1[an] = mk(N.re.y, N.im.y);
+        }
+    }
+}
+
 }  // namespace hyena

@@ -40,6 +40,11 @@ int64_t staged2d_chunk_planes(int64_t W);
 int64_t staged2d_workspace_planes(int64_t W, int64_t planes);
 cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyena_dtype_t dt, cudaStream_t st,
                                  const StagedLanes &lanes);
+// 2D kernel spectra through the staged kernels, with plan-owned scratch of
+// staged2d_spec_scratch_bytes(W) (two chunks of staged2d_spec_chunk(W) kernels)
+size_t staged2d_spec_scratch_bytes(int64_t W);
+cudaError_t launch_spec_2d_staged(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W,
+                                  const c32 *tw, float2 *scratch, cudaStream_t st, const StagedLanes &lanes);
 // 2D, one cluster per plane (H == W in {32, 64, 128, 256})
 struct Fwd2dArgs;
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);
