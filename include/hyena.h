@@ -155,8 +155,9 @@ HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_im
  *           full row axis and the non-negative half of the column axis,
  *           stored column-bin-major: bin (ky, kx) at [kx][ky].
  *           Unnormalised. Must not overlap h.
- * 2D plans with H = W = 256 transform the kernels in chunks through a
- * 32 MiB device buffer that the plan allocates at creation and owns.
+ * Plans on HYENA_PATH_STAGED (64 MiB) and 2D plans with H = W = 256 (32 MiB)
+ * transform the filters in chunks through a device buffer that the plan
+ * allocates at creation and owns.
  */
 HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
                                      void *H_out, void *stream);

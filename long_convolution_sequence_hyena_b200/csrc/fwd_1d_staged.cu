@@ -62,6 +62,62 @@ cudaError_t launch_staged_g(const Fwd1dArgs &f, float2 *ws, int64_t chunk, hyena
                 : launch_staged_io<G, __nv_bfloat16, false>(f, ws, chunk, lanes, nst);
 }
 
+// Filter spectra: two chunks of 32 MB of transforms in flight, in plan-owned scratch.
+int64_t staged_spec_chunk(int64_t MC) { return ((int64_t)32 << 20) / (MC * 8); }
+size_t staged_spec_scratch_bytes(int64_t MC) { return (size_t)2 * staged_spec_chunk(MC) * MC * sizeof(float2); }
+
+template <typename G>
+cudaError_t launch_spec_staged_g(const Spec1dArgs &base, int64_t nrows, const cudaStream_t *lanes, int nst) {
+    cudaError_t e = cudaFuncSetAttribute(hyena_staged_spec_rows_x2<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)G::RSMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t chunk = staged_spec_chunk(G::MC);
+    for (int64_t o0 = 0, c = 0; o0 < nrows; o0 += chunk, ++c) {
+        Spec1dArgs a = base;
+        a.ws = base.ws + (c % nst) * chunk * G::MC;
+        a.o0 = o0;
+        a.nr = (nrows - o0) < chunk ? (nrows - o0) : chunk;
+        const int64_t pairs = (a.nr + 1) / 2;
+        const cudaStream_t s = lanes[c % nst];
+        hyena_staged_spec_cols_x2<G><<<(unsigned)(pairs * G::CGROUPS), G::CT, G::CSMEM, s>>>(a);
+        hyena_staged_spec_rows_x2<G><<<(unsigned)(pairs * G::RGROUPS), G::RT, G::RSMEM, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_spec_1d_staged(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
+                                  const c32 *tw, float2 *scratch, cudaStream_t st, const StagedLanes &sl) {
+    Spec1dArgs a;
+    a.h = h;
+    a.h_stride = h_stride;
+    a.L = L;
+    a.Hout = Hout;
+    a.tw = tw;
+    a.ws = scratch;
+    a.o0 = 0;
+    a.nr = 0;
+    auto run = [&](const cudaStream_t *lanes, int nst) -> cudaError_t {
+        switch (MC) {
+            case 32768: return launch_spec_staged_g<GS_32K>(a, nrows, lanes, nst);
+            case 65536: return launch_spec_staged_g<GS_64K>(a, nrows, lanes, nst);
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    if (nrows <= staged_spec_chunk(MC)) return run(&st, 1);
+    cudaError_t e = cudaEventRecord(sl.fork, st);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
+    if (e != cudaSuccess) return e;
+    const cudaError_t le = run(sl.lane, 2);
+    for (int i = 0; i < 2; ++i) {
+        e = cudaEventRecord(sl.join[i], sl.lane[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sl.join[i], 0);
+        if (e != cudaSuccess) return e;
+    }
+    return le;
+}
+
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &f, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
                                  cudaStream_t st, const StagedLanes &sl) {
     const int64_t chunk = staged_chunk_rows(MC);

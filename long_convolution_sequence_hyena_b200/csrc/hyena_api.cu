@@ -165,8 +165,10 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
             return HYENA_ERR_CUDA;
         }
     }
-    if (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww)) {
-        if (cudaMalloc(&p.spec_ws, staged2d_spec_scratch_bytes(p.Ww)) != cudaSuccess) {
+    if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
+        const size_t sb = p.path == HYENA_PATH_STAGED ? staged_spec_scratch_bytes(p.MC)
+                                                      : staged2d_spec_scratch_bytes(p.Ww);
+        if (cudaMalloc(&p.spec_ws, sb) != cudaSuccess) {
             cudaGetLastError();
             release_lanes(&p);
             cudaFree(p.tw);
@@ -245,8 +247,19 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
             src = reinterpret_cast<const float *>(H_out);
         }
-        e = plan->path == HYENA_PATH_CTA ? launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st)
-                                         : launch_spec_1d_cluster(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st);
+        if (plan->path == HYENA_PATH_STAGED) {
+            StagedLanes lanes;
+            lanes.lane[0] = plan->lane[0];
+            lanes.lane[1] = plan->lane[1];
+            lanes.fork = plan->fork;
+            lanes.join[0] = plan->join[0];
+            lanes.join[1] = plan->join[1];
+            e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, plan->spec_ws, st, lanes);
+        } else {
+            e = plan->path == HYENA_PATH_CTA
+                    ? launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st)
+                    : launch_spec_1d_cluster(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st);
+        }
     } else {
         int64_t rs = 2 * plan->Ww, cs = 4 * plan->Hh * plan->Ww;
         if (!h) {

@@ -475,4 +475,126 @@ __global__ void __launch_bounds__(G::RT, 4) hyena_staged_rows_x2(const StagedArg
     }
 }
 
+// ---------------------------------------------------------------------------
+// Filter spectra of long rows through the same two stages, two filter rows in
+// lockstep: the column kernel reads the taps (fp32, zero past L) and runs the
+// forward column FFTs and twiddle; the row kernel runs the row FFTs and
+// unpacks the packed spectrum into H[k] = E[k] + W_M^k O[k] (natural order,
+// H[MC] = E[0] - O[0]). The scratch belongs to the plan, so the spectrum may
+// be computed in place: a chunk's column kernel reads all of its rows before
+// its row kernel writes their spectra.
+
+struct Spec1dArgs {
+    const float *h;    // filter row o at h + o * h_stride, L taps
+    int64_t h_stride;
+    int64_t L;
+    c32 *Hout;         // [rows][MC + 1]
+    const c32 *tw;     // W_M, then W_1024
+    float2 *ws;        // chunk rows x MC complex, each [k1][n2]
+    int64_t o0;        // first filter row of the chunk
+    int64_t nr;        // rows in the chunk
+};
+
+template <typename G>
+__global__ void __launch_bounds__(G::CT, 3) hyena_staged_spec_cols_x2(const Spec1dArgs a) {
+    static_assert(G::ROWS == 2, "lockstep geometry");
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T1 = G::T1, MC = G::MC, M = 2 * MC;
+    extern __shared__ float smem[];
+    const int64_t lp = blockIdx.x / G::CGROUPS;
+    const int cgp = blockIdx.x % G::CGROUPS;
+    const int j = threadIdx.x % G::NCOL, t1 = threadIdx.x / G::NCOL;
+    const int n2 = cgp * G::NCOL + j;
+    const bool has1 = 2 * lp + 1 < a.nr;
+    const float *h0 = a.h + (a.o0 + 2 * lp) * a.h_stride;
+    const float *h1 = a.h + (a.o0 + 2 * lp + (has1 ? 1 : 0)) * a.h_stride;
+    float2 *w0 = a.ws + (2 * lp) * MC;
+    float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
+    c32x2 v[E];
+#pragma unroll
+    for (int q = 0; q < E / 2; ++q) {
+        const int64_t pos = 2 * ((int64_t)M2 * (t1 + q * T1) + n2);
+        const float a0 = pos < a.L ? h0[pos] : 0.f, b0 = pos + 1 < a.L ? h0[pos + 1] : 0.f;
+        const float a1 = has1 && pos < a.L ? h1[pos] : 0.f, b1 = has1 && pos + 1 < a.L ? h1[pos + 1] : 0.f;
+        v[q] = c32x2{f2(a0, a1), f2(b0, b1)};
+    }
+#pragma unroll
+    for (int q = E / 2; q < E; ++q) v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
+    fft_cta<M1, E, -1, true, G::TWS, G::NCOL>(v, smem, nullptr, t1, a.tw + M, j);
+    const c32 base = ldg_c(a.tw + ((2 * (int64_t)n2 * t1) & (M - 1)));
+    const c32 step = ldg_c(a.tw + ((2 * (int64_t)n2 * T1) & (M - 1)));
+    twiddle_powers<E, 1, 0>(v, step);
+    const uint64_t keep = l2_keep();
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const c32x2 r = mul(v[q], base);
+        const int ad = (t1 + q * T1) * M2 + n2;
+        st_pol(w0 + ad, make_float2(r.re.x, r.im.x), keep);
+        if (has1) st_pol(w1 + ad, make_float2(r.re.y, r.im.y), keep);
+    }
+}
+
+template <typename G>
+__global__ void __launch_bounds__(G::RT, 4) hyena_staged_spec_rows_x2(const Spec1dArgs a) {
+    static_assert(G::ROWS == 2, "lockstep geometry");
+    constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, MC = G::MC, M = 2 * MC;
+    constexpr int NROW = G::NROW, HROW = G::HROW, RT = G::RT;
+    extern __shared__ float smem[];
+    float4 *rowb = reinterpret_cast<float4 *>(smem);
+    const int64_t lp = blockIdx.x / G::RGROUPS;
+    const int g = blockIdx.x % G::RGROUPS;
+    const int r = threadIdx.x % NROW, t2 = threadIdx.x / NROW;
+    const int k1 = row_of_slot<G>(g, r);
+    const int rm = (k1 == 0 || k1 == M1 / 2) ? r : (r < HROW ? r + HROW : r - HROW);
+    const bool has1 = 2 * lp + 1 < a.nr;
+    const float2 *w0 = a.ws + (2 * lp) * MC;
+    const float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
+    auto ld = [&](int ad) -> c32x2 {
+        const float4 f = rowb[ad];
+        return c32x2{f2(f.x, f.y), f2(f.z, f.w)};
+    };
+    const uint64_t once = l2_stream();               // the scratch is read once
+#pragma unroll
+    for (int sl = 0; sl < NROW; ++sl) {
+        const int64_t base = (int64_t)row_of_slot<G>(g, sl) * M2;
+#pragma unroll
+        for (int k2 = threadIdx.x; k2 < M2; k2 += RT) {
+            const float2 f0 = ld_pol(w0 + base + k2, once), f1 = ld_pol(w1 + base + k2, once);
+            rowb[maddr<M2>(k2, sl)] = make_float4(f0.x, f1.x, f0.y, f1.y);
+        }
+    }
+    __syncthreads();
+    c32x2 v[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) v[q] = ld(maddr<M2>(t2 + q * T2, r));
+    __syncthreads();
+    fft_cta<M2, E, -1, false, G::TWS, NROW>(v, smem, nullptr, t2, a.tw + M, r);
+#pragma unroll
+    for (int q = 0; q < E; ++q)
+        rowb[maddr<M2>(t2 + q * T2, r)] = make_float4(v[q].re.x, v[q].re.y, v[q].im.x, v[q].im.y);
+    __syncthreads();
+    const c32 wb = ldg_c(a.tw + k1 + M1 * t2);      // W_M^{k1 + M1 t2}
+    c32 *H0 = a.Hout + (a.o0 + 2 * lp) * (int64_t)(MC + 1);
+    c32 *H1 = a.Hout + (a.o0 + 2 * lp + (has1 ? 1 : 0)) * (int64_t)(MC + 1);
+    const int z0 = opaque_zero();
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+        const int k = k1 + M1 * (t2 + q * T2);
+        const int km = (MC - k) & (MC - 1);
+        const c32x2 Zk = v[q];
+        const c32x2 Zm = ld(maddr<M2>(km / M1, rm));
+        const c32x2 E2{f2add(Zk.re, Zm.re), f2sub(Zk.im, Zm.im)};   // 2E
+        const c32x2 O2{f2add(Zk.im, Zm.im), f2sub(Zm.re, Zk.re)};   // 2O
+        const c32x2 wO = mul(O2, mul(wb, w2e<E>(q, z0)));
+        const float2 half = f2(0.5f, 0.5f);
+        const c32x2 X{f2mul(f2add(E2.re, wO.re), half), f2mul(f2add(E2.im, wO.im), half)};
+        H0[k] = mk(X.re.x, X.im.x);
+        if (has1) H1[k] = mk(X.re.y, X.im.y);
+        if (k == 0) {                                  // Nyquist bin: E_0 - O_0, real
+            const float2 ny = f2mul(f2sub(E2.re, O2.re), half);
+            H0[MC] = mk(ny.x, 0.f);
+            if (has1) H1[MC] = mk(ny.y, 0.f);
+        }
+    }
+}
+
 }  // namespace hyena

@@ -32,6 +32,11 @@ int64_t staged_chunk_rows(int64_t MC);
 int64_t staged_workspace_rows(int64_t MC, int64_t rows);
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &a, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
                                  cudaStream_t st, const StagedLanes &lanes);
+// 1D filter spectra through the staged kernels, with plan-owned scratch of
+// staged_spec_scratch_bytes(MC)
+size_t staged_spec_scratch_bytes(int64_t MC);
+cudaError_t launch_spec_1d_staged(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
+                                  const c32 *tw, float2 *scratch, cudaStream_t st, const StagedLanes &lanes);
 // 2D staged (H = W = 256): chunks of staged2d_chunk_planes(W) planes, two in flight;
 // workspace staged2d_workspace_planes(W, planes) * 2H * W/2 complex64
 struct Fwd2dArgs;

@@ -31,6 +31,6 @@ struct hyena_plan_s {
     bool has_lanes = false;
     cudaStream_t lane[2] = {nullptr, nullptr};
     cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
-    // 2D staged spectra: scratch for two chunks of kernel transforms (owned)
+    // staged spectra (1D long rows, 2D 256x256): scratch for two chunks of transforms (owned)
     float2 *spec_ws = nullptr;
 };
