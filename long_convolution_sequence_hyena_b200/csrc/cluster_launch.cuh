@@ -4,13 +4,10 @@
 
 namespace hyena {
 
-using G1_32K = ClusterGeom<32768, 8, 128, 16, 2>;    // 1D, 32768 < M <= 65536
-using G1_64K = ClusterGeom<65536, 16, 256, 16, 2>;   // 1D, M = 131072 (16-CTA cluster)
 using G1_128K = ClusterGeom<131072, 16, 512, 16>; // 1D, M = 262144 (16-CTA cluster)
 using G2_32 = ClusterGeom<2048, 1, 64, 16>;       // 2D, 32 x 32 grid (64 x 64 padded)
 using G2_64 = ClusterGeom<8192, 2, 128, 16>;      // 2D, 64 x 64
 using G2_128 = ClusterGeom<32768, 4, 256, 16>;    // 2D, 128 x 128
-using G2_256 = ClusterGeom<131072, 16, 512, 16>;  // 2D, 256 x 256 (16-CTA cluster)
 
 template <typename G, typename Kern, typename... Args>
 inline cudaError_t launch_cluster(Kern kern, int64_t units, cudaStream_t st, Args... args) {

@@ -1,4 +1,5 @@
-// 1D cluster kernels: fused forward and filter spectrum instantiations.
+// 1D cluster kernels: fused forward and filter spectrum instantiations
+// (M = 262144; shorter long rows take the staged kernels).
 #include "launch.h"
 #include "cluster_launch.cuh"
 
@@ -16,8 +17,6 @@ cudaError_t launch_fwd_1d_cluster_g(const Fwd1dArgs &a, hyena_dtype_t dt, bool e
 
 cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
     switch (MC) {
-        case 32768: return launch_fwd_1d_cluster_g<G1_32K>(a, dt, even, st);
-        case 65536: return launch_fwd_1d_cluster_g<G1_64K>(a, dt, even, st);
         case 131072: return launch_fwd_1d_cluster_g<G1_128K>(a, dt, even, st);
         default: return cudaErrorInvalidValue;
     }
@@ -26,8 +25,6 @@ cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t 
 cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
                                    const c32 *tw, cudaStream_t st) {
     switch (MC) {
-        case 32768: return launch_cluster<G1_32K>(hyena_spectrum_1d_cluster<G1_32K>, nrows, st, h, h_stride, L, Hout, tw);
-        case 65536: return launch_cluster<G1_64K>(hyena_spectrum_1d_cluster<G1_64K>, nrows, st, h, h_stride, L, Hout, tw);
         case 131072:
             return launch_cluster<G1_128K>(hyena_spectrum_1d_cluster<G1_128K>, nrows, st, h, h_stride, L, Hout, tw);
         default: return cudaErrorInvalidValue;

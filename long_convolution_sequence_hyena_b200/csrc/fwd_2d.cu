@@ -16,7 +16,6 @@ cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaS
         case 32: return launch_fwd_2d_g<G2_32>(a, dt, st);
         case 64: return launch_fwd_2d_g<G2_64>(a, dt, st);
         case 128: return launch_fwd_2d_g<G2_128>(a, dt, st);
-        case 256: return launch_fwd_2d_g<G2_256>(a, dt, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -27,7 +26,6 @@ cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, in
         case 32: return launch_cluster<G2_32>(hyena_spectrum_2d_cluster<G2_32>, n, st, K, rs, cs, Kout, tw);
         case 64: return launch_cluster<G2_64>(hyena_spectrum_2d_cluster<G2_64>, n, st, K, rs, cs, Kout, tw);
         case 128: return launch_cluster<G2_128>(hyena_spectrum_2d_cluster<G2_128>, n, st, K, rs, cs, Kout, tw);
-        case 256: return launch_cluster<G2_256>(hyena_spectrum_2d_cluster<G2_256>, n, st, K, rs, cs, Kout, tw);
         default: return cudaErrorInvalidValue;
     }
 }

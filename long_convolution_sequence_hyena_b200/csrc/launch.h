@@ -16,7 +16,7 @@ cudaError_t launch_spec_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hou
 // 1D, two rows of one channel per thread group (B even, MC <= 8192)
 bool pair_path_supported(int64_t MC, int64_t B);
 cudaError_t launch_fwd_1d_pair(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
-// 1D, one cluster per row (MC in {32768, 65536, 131072})
+// 1D, one cluster per row (MC = 131072)
 cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
 cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
                                    const c32 *tw, cudaStream_t st);
@@ -50,7 +50,7 @@ cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyen
 size_t staged2d_spec_scratch_bytes(int64_t W);
 cudaError_t launch_spec_2d_staged(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W,
                                   const c32 *tw, float2 *scratch, cudaStream_t st, const StagedLanes &lanes);
-// 2D, one cluster per plane (H == W in {32, 64, 128, 256})
+// 2D, one cluster per plane (H == W in {32, 64, 128})
 struct Fwd2dArgs;
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);
 cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W, const c32 *tw,
