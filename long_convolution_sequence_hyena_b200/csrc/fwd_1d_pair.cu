@@ -9,7 +9,13 @@ template <int MC, typename IO, bool EVEN>
 cudaError_t launch_fwd_1d_pair_t(const Fwd1dArgs &a, cudaStream_t st) {
     constexpr int E = 16;
     constexpr int PPC = pair_pairs_per_cta(MC, E);
-    auto kern = hyena_fwd_1d_pair<MC, E, IO, EVEN>;
+    // With 256 threads and more (128 registers), order 2 runs the unrolled
+    // chain, which needs fewer registers than the loop (4.8 % faster at
+    // MC = 8192). With 128 threads the loop is faster (the unrolled chain at
+    // MC = 2048 was 19 % slower).
+    auto kern = hyena_fwd_1d_pair<MC, E, IO, EVEN, 0>;
+    if constexpr (pair_threads(MC, E) >= 256)
+        if (a.order == 2) kern = hyena_fwd_1d_pair<MC, E, IO, EVEN, 2>;
     const size_t sm = pair_smem_bytes<IO, EVEN>(MC, E);
     if (sm > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

@@ -177,8 +177,10 @@ constexpr size_t pair_smem_bytes(int MC, int E) {
 
 // Fused order-N forward, one group of MC/E threads per pair of rows
 // (b, d), (b+1, d); B must be even. Pairs are visited d-major so the B/2
-// pairs that read the same spectrum row run together.
-template <int MC, int E, typename IO, bool EVEN>
+// pairs that read the same spectrum row run together. NORD > 0 fixes the
+// order at compile time (the chain is unrolled); NORD = 0 reads it from the
+// arguments.
+template <int MC, int E, typename IO, bool EVEN, int NORD>
 __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
     hyena_fwd_1d_pair(const Fwd1dArgs a) {
     constexpr int T = MC / E;
@@ -220,7 +222,9 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
     constexpr int NT = pair_threads(MC, E);
     P *gst = reinterpret_cast<P *>(reinterpret_cast<unsigned char *>(smem4) + PPC * pair_smem_bytes_per_pair(MC)) +
              threadIdx.x;   // thread-private slots gst[(2 q + row) * NT]
-    for (int n = 0; n < a.order; ++n) {
+    const int norder = NORD > 0 ? NORD : a.order;
+#pragma unroll
+    for (int n = 0; n < norder; ++n) {   // unrolled only when the order is a constant
         const IO *g0 = reinterpret_cast<const IO *>(a.gates[n]) + row0 * L;
         const IO *g1 = reinterpret_cast<const IO *>(a.gates[n]) + row1 * L;
         P ga[GST ? 1 : E / 2], gb[GST ? 1 : E / 2];
@@ -249,9 +253,18 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
         for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);   // staged while the FFT runs
         cp_async_commit();
 
-        fft_cta_x2<MC, E, -1, true>(v, sre, sim, t, a.tw);
-        spectral_product_x2<MC, E>(v, sre, sim, t, Hs, dsk, wt);
-        fft_cta_x2<MC, E, +1, false>(v, sre, sim, t, a.tw);
+        // With 128 registers (256 threads and more), each stage takes its own
+        // opaque copy of the thread index, so that the compiler recomputes the
+        // stage's shared-memory addresses and twiddle indices instead of
+        // keeping them live across the whole chain (which spills; ptxas -v).
+        constexpr bool OPQ = pair_threads(MC, E) >= 256;
+        int tf = t, ts = t, ti = t;
+        if constexpr (OPQ) asm volatile("" : "+r"(tf));
+        fft_cta_x2<MC, E, -1, true>(v, sre, sim, tf, a.tw);
+        if constexpr (OPQ) asm volatile("" : "+r"(ts));
+        spectral_product_x2<MC, E>(v, sre, sim, ts, Hs, dsk, wt);
+        if constexpr (OPQ) asm volatile("" : "+r"(ti));
+        fft_cta_x2<MC, E, +1, false>(v, sre, sim, ti, a.tw);
 
         // gate; positions >= L are cleared so the next order sees a zero-padded row
 #pragma unroll
