@@ -212,6 +212,44 @@ HYENA_API hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batch
                                                 const void *const *gates, const void *H, const float *Dskip,
                                                 void *y, void *stream);
 
+/*
+ * hyena_forward on activations that live in HOST memory: the call copies the
+ * inputs to the device, runs the forward and copies y back, pipelined over
+ * the batch so that the host-to-device copies of one stage, the forward of
+ * the stage before and the device-to-host copy of the one before that
+ * overlap. The paper has no counterpart of this call: it moves data, and
+ * each stage computes exactly what hyena_forward computes on its rows.
+ *
+ *   batch       B >= 0 (B = 0 copies and launches nothing)
+ *   v_host      [B, D, L] or [B, C, H, W] io dtype, in PAGE-LOCKED host
+ *               memory (cudaHostAlloc / cudaMallocHost, or registered with
+ *               cudaHostRegister); pageable memory returns
+ *               HYENA_ERR_INVALID_ARG, because a copy from the device into
+ *               it would block the calling thread
+ *   gates_host  HOST array of N pointers x^1..x^N, each page-locked and
+ *               shaped like v_host
+ *   H, Dskip    DEVICE pointers, as for hyena_forward
+ *   y_host      output, page-locked host memory shaped like v_host; must not
+ *               overlap v_host or a gate
+ *   workspace   device scratch of at least
+ *               hyena_forward_host_workspace_bytes(plan, batch) bytes,
+ *               16-byte aligned: two stage buffers of inputs and outputs,
+ *               then the forward's own workspace for one stage
+ *
+ * Stages are whole batch elements: as many as make about 8 MiB of input, at
+ * most B; in 1D rounded up to an even count, so that two rows of one channel
+ * share a thread group. With B = 1 there is one stage and nothing overlaps. The copies run on two streams the call creates
+ * and releases (cudaStreamDestroy returns at once, and the streams are freed
+ * when their work is done). Every copy waits for the work enqueued on
+ * `stream` before the call, and work enqueued on `stream` after the call
+ * waits for all of them. The host buffers must stay valid, and y_host
+ * unread, until then. Concurrent calls need one workspace each.
+ */
+HYENA_API size_t hyena_forward_host_workspace_bytes(hyena_plan_t plan, int64_t batch);
+HYENA_API hyena_status_t hyena_forward_host(hyena_plan_t plan, int64_t batch, const void *v_host,
+                                            const void *const *gates_host, const void *H, const float *Dskip,
+                                            void *y_host, void *workspace, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

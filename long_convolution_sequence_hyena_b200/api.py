@@ -114,3 +114,22 @@ class Plan:
                                 0 if ws is None else ws.numel(), _stream(stream))
         _check(st, "hyena_forward")
         return out
+
+    def host_workspace_bytes(self, batch: int) -> int:
+        return capi.hyena_forward_host_workspace_bytes(self.handle, batch)
+
+    def forward_host(self, v_host, gates_host, H, dskip=None, out=None, workspace=None, stream=None):
+        """Forward on page-locked CPU tensors (``tensor.pin_memory()``): the library copies v and
+        the gates in and y out, pipelined over the batch, on ``stream``. H and dskip are device
+        tensors. Returns the page-locked output; it is complete once ``stream`` reaches the end of
+        the call (synchronize before reading it)."""
+        if out is None:
+            out = torch.empty_like(v_host).pin_memory()
+        ws = workspace
+        if ws is None:
+            ws = torch.empty(max(1, self.host_workspace_bytes(v_host.shape[0])), dtype=torch.uint8, device=H.device)
+        st = capi.hyena_forward_host(self.handle, v_host.shape[0], v_host.data_ptr(),
+                                     [g.data_ptr() for g in gates_host], H.data_ptr(), _ptr(dskip), out.data_ptr(),
+                                     ws.data_ptr(), ws.numel(), _stream(stream))
+        _check(st, "hyena_forward_host")
+        return out

@@ -30,7 +30,7 @@ STATUS_NAMES = {
 EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
-    "hyena_forward_no_alloc",
+    "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
 )
 
 
@@ -61,6 +61,8 @@ def _load():
         "hyena_forward": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_status_string": ([i32], ctypes.c_char_p),
         "hyena_forward_no_alloc": ([p, i64, p, ctypes.POINTER(p), p, p, p, p], i32),
+        "hyena_forward_host_workspace_bytes": ([p, i64], sz),
+        "hyena_forward_host": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -118,3 +120,15 @@ def hyena_forward_no_alloc(plan, batch: int, v: int, gates, H: int, Dskip, y: in
     own fixed device array (for callers that cannot allocate device memory)."""
     garr = None if gates is None else (ctypes.c_void_p * len(gates))(*gates)
     return lib.hyena_forward_no_alloc(plan, batch, v, garr, H, Dskip, y, stream)
+
+
+def hyena_forward_host_workspace_bytes(plan, batch: int) -> int:
+    return lib.hyena_forward_host_workspace_bytes(plan, batch)
+
+
+def hyena_forward_host(plan, batch: int, v_host: int, gates_host, H: int, Dskip, y_host: int, workspace,
+                       ws_bytes: int, stream: int = 0) -> int:
+    """hyena_forward on page-locked host activations (v, gates, y): the library copies them in
+    and out, pipelined over the batch."""
+    garr = None if gates_host is None else (ctypes.c_void_p * len(gates_host))(*gates_host)
+    return lib.hyena_forward_host(plan, batch, v_host, garr, H, Dskip, y_host, workspace, ws_bytes, stream)

@@ -63,3 +63,5 @@ def test_null_plan_rejected(capi):
     assert capi.hyena_forward(None, 1, 16, [16], 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
     assert capi.hyena_filter_spectrum(None, 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
     assert capi.hyena_implicit_filter(None, None, 16) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_forward_host_workspace_bytes(None, 4) == 0
+    assert capi.hyena_forward_host(None, 1, 16, [16], 16, None, 16, 16, 1 << 20) == capi.HYENA_ERR_INVALID_ARG
