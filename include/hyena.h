@@ -27,7 +27,9 @@
  *    that returns an error has launched nothing (HYENA_ERR_CUDA excepted: the
  *    launch itself failed). Nothing aborts the process.
  *  - Calls on one plan from several host threads are safe: a plan is read-only
- *    after creation.
+ *    after creation, apart from the staged paths' streams and spectrum
+ *    scratch, whose use every call orders on the GPU itself (each call forks
+ *    and joins those streams with events of its own).
  */
 #ifndef HYENA_H
 #define HYENA_H
@@ -54,7 +56,7 @@ typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype_t;
 typedef enum {
     HYENA_OK = 0,
     HYENA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
-    HYENA_ERR_UNSUPPORTED = 2,   /* valid but outside what this build implements */
+    HYENA_ERR_UNSUPPORTED = 2,   /* valid but outside what this library implements */
     HYENA_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
     HYENA_ERR_WORKSPACE = 4,     /* workspace missing or smaller than hyena_workspace_bytes */
     HYENA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
@@ -157,7 +159,9 @@ HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_im
  *           Unnormalised. Must not overlap h.
  * Plans on HYENA_PATH_STAGED (64 MiB) and 2D plans with H = W = 256 (32 MiB)
  * transform the filters in chunks through a device buffer that the plan
- * allocates at creation and owns.
+ * allocates at creation and owns. Those chunks run on the plan's own two
+ * streams, forked from `stream` and joined back to it, so calls on one such
+ * plan (from any stream or thread) run one after another on the GPU.
  */
 HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
                                      void *H_out, void *stream);
@@ -188,8 +192,9 @@ HYENA_API const char *hyena_status_string(hyena_status_t status);
  * no allocator of its own to hand out a workspace; a process whose device
  * memory belongs to a framework's caching allocator; a latency-bound loop in
  * which a cudaMalloc, which may synchronise the device, is not acceptable.
- * The paper has no counterpart of this call: it changes only where the
- * staged path's scratch lives, not what is computed.
+ * The pages cited at the top of this file have no counterpart of this call:
+ * it changes only where the staged path's scratch lives, not what is
+ * computed.
  *
  * Plans on HYENA_PATH_STAGED only (1D, M in {65536, 131072}); any other plan
  * returns HYENA_ERR_UNSUPPORTED. The other arguments are those of
@@ -217,8 +222,9 @@ HYENA_API hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batch
  * inputs to the device, runs the forward and copies y back, pipelined over
  * the batch so that the host-to-device copies of one stage, the forward of
  * the stage before and the device-to-host copy of the one before that
- * overlap. The paper has no counterpart of this call: it moves data, and
- * each stage computes exactly what hyena_forward computes on its rows.
+ * overlap. The pages cited at the top of this file have no counterpart of
+ * this call: it moves data, and each stage computes exactly what
+ * hyena_forward computes on its rows.
  *
  *   batch       B >= 0 (B = 0 copies and launches nothing)
  *   v_host      [B, D, L] or [B, C, H, W] io dtype, in PAGE-LOCKED host

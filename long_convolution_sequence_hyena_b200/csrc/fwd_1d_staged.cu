@@ -105,7 +105,7 @@ cudaError_t launch_spec_1d_staged(const float *h, int64_t h_stride, int64_t L, c
             default: return cudaErrorInvalidValue;
         }
     };
-    if (nrows <= staged_spec_chunk(MC)) return run(&st, 1);
+    // always on the plan's lanes, one chunk too: scratch slot i is used by lane i only
     cudaError_t e = cudaEventRecord(sl.fork, st);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
     if (e != cudaSuccess) return e;

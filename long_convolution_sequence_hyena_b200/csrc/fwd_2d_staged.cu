@@ -82,7 +82,7 @@ cudaError_t launch_spec_2d_staged(const float *K, int64_t rs, int64_t cs, c32 *K
         }
         return cudaSuccess;
     };
-    if (n <= chunk) return run(&st, 1);
+    // always on the plan's lanes, one chunk too: scratch slot i is used by lane i only
     e = cudaEventRecord(sl.fork, st);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
     if (e != cudaSuccess) return e;

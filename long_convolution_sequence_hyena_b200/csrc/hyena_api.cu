@@ -37,21 +37,42 @@ std::vector<float2> twiddle_table(int64_t M) {
     return t;
 }
 
-// Destroy the staged path's streams and events (those that were created).
+// Destroy the staged path's streams (those that were created).
 bool release_lanes(hyena_plan_s *p) {
     if (!p->has_lanes) return true;
     bool ok = true;
     for (int i = 0; i < 2; ++i) {
         if (p->lane[i] && cudaStreamDestroy(p->lane[i]) != cudaSuccess) ok = false;
-        if (p->join[i] && cudaEventDestroy(p->join[i]) != cudaSuccess) ok = false;
         p->lane[i] = nullptr;
-        p->join[i] = nullptr;
     }
-    if (p->fork && cudaEventDestroy(p->fork) != cudaSuccess) ok = false;
-    p->fork = nullptr;
     p->has_lanes = false;
     return ok;
 }
+
+// The plan's lanes with fork and join events that belong to one call, so
+// that calls on one plan from several threads never wait on each other's
+// event records. cudaEventDestroy returns at once; an event that a stream
+// still waits on is released when the wait is over.
+struct CallLanes {
+    StagedLanes l;
+    bool ok = false;
+    explicit CallLanes(const hyena_plan_s *p) {
+        l.lane[0] = p->lane[0];
+        l.lane[1] = p->lane[1];
+        l.fork = l.join[0] = l.join[1] = nullptr;
+        ok = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&l.join[0], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&l.join[1], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+    }
+    ~CallLanes() {
+        if (l.fork) cudaEventDestroy(l.fork);
+        for (int i = 0; i < 2; ++i)
+            if (l.join[i]) cudaEventDestroy(l.join[i]);
+    }
+    CallLanes(const CallLanes &) = delete;
+    CallLanes &operator=(const CallLanes &) = delete;
+};
 
 hyena_status_t check_device(const hyena_plan_s *p) {
     int dev = -1;
@@ -154,10 +175,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
     }
     if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
         bool ok = cudaStreamCreateWithFlags(&p.lane[0], cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&p.lane[1], cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&p.join[0], cudaEventDisableTiming) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&p.join[1], cudaEventDisableTiming) == cudaSuccess;
+                  cudaStreamCreateWithFlags(&p.lane[1], cudaStreamNonBlocking) == cudaSuccess;
         p.has_lanes = true;
         if (!ok) {
             release_lanes(&p);
@@ -174,11 +192,19 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
             cudaFree(p.tw);
             return HYENA_ERR_NOMEM;
         }
+        p.spec_mu = new (std::nothrow) std::mutex;
+        if (!p.spec_mu) {
+            cudaFree(p.spec_ws);
+            release_lanes(&p);
+            cudaFree(p.tw);
+            return HYENA_ERR_NOMEM;
+        }
     }
     hyena_plan_s *heap = new (std::nothrow) hyena_plan_s(p);
     if (!heap) {
         release_lanes(&p);
         if (p.spec_ws) cudaFree(p.spec_ws);
+        delete p.spec_mu;
         cudaFree(p.tw);
         return HYENA_ERR_NOMEM;
     }
@@ -192,6 +218,7 @@ hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     if (plan->tw && cudaFree(plan->tw) != cudaSuccess) st = HYENA_ERR_CUDA;
     if (!release_lanes(plan)) st = HYENA_ERR_CUDA;
     if (plan->spec_ws && cudaFree(plan->spec_ws) != cudaSuccess) st = HYENA_ERR_CUDA;
+    delete plan->spec_mu;
     delete plan;
     return st;
 }
@@ -248,13 +275,10 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             src = reinterpret_cast<const float *>(H_out);
         }
         if (plan->path == HYENA_PATH_STAGED) {
-            StagedLanes lanes;
-            lanes.lane[0] = plan->lane[0];
-            lanes.lane[1] = plan->lane[1];
-            lanes.fork = plan->fork;
-            lanes.join[0] = plan->join[0];
-            lanes.join[1] = plan->join[1];
-            e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, plan->spec_ws, st, lanes);
+            CallLanes cl(plan);
+            if (!cl.ok) return HYENA_ERR_CUDA;
+            std::lock_guard<std::mutex> hold(*plan->spec_mu);
+            e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, plan->spec_ws, st, cl.l);
         } else {
             e = plan->path == HYENA_PATH_CTA
                     ? launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st)
@@ -271,13 +295,10 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             src = reinterpret_cast<const float *>(H_out);
         }
         if (plan->spec_ws) {
-            StagedLanes lanes;
-            lanes.lane[0] = plan->lane[0];
-            lanes.lane[1] = plan->lane[1];
-            lanes.fork = plan->fork;
-            lanes.join[0] = plan->join[0];
-            lanes.join[1] = plan->join[1];
-            e = launch_spec_2d_staged(src, rs, cs, Hc, nrows, plan->Ww, tw, plan->spec_ws, st, lanes);
+            CallLanes cl(plan);
+            if (!cl.ok) return HYENA_ERR_CUDA;
+            std::lock_guard<std::mutex> hold(*plan->spec_mu);
+            e = launch_spec_2d_staged(src, rs, cs, Hc, nrows, plan->Ww, tw, plan->spec_ws, st, cl.l);
         } else {
             e = launch_spec_2d(src, rs, cs, Hc, nrows, plan->Ww, tw, st);
         }
@@ -316,14 +337,10 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
         a.order = plan->order;
         cudaError_t e2;
         if (staged2d_supported(plan->Ww)) {
-            StagedLanes lanes;
-            lanes.lane[0] = plan->lane[0];
-            lanes.lane[1] = plan->lane[1];
-            lanes.fork = plan->fork;
-            lanes.join[0] = plan->join[0];
-            lanes.join[1] = plan->join[1];
+            CallLanes cl(plan);
+            if (!cl.ok) return HYENA_ERR_CUDA;
             e2 = launch_fwd_2d_staged(a, plan->Ww, reinterpret_cast<float2 *>(workspace), plan->dtype,
-                                      (cudaStream_t)stream, lanes);
+                                      (cudaStream_t)stream, cl.l);
         } else {
             e2 = launch_fwd_2d(a, plan->Ww, plan->dtype, (cudaStream_t)stream);
         }
@@ -345,14 +362,10 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     const bool even = (plan->L % 2) == 0;
     cudaError_t e;
     if (plan->path == HYENA_PATH_STAGED) {
-        StagedLanes lanes;
-        lanes.lane[0] = plan->lane[0];
-        lanes.lane[1] = plan->lane[1];
-        lanes.fork = plan->fork;
-        lanes.join[0] = plan->join[0];
-        lanes.join[1] = plan->join[1];
+        CallLanes cl(plan);
+        if (!cl.ok) return HYENA_ERR_CUDA;
         e = launch_fwd_1d_staged(a, plan->MC, reinterpret_cast<float2 *>(workspace), plan->dtype, even,
-                                 (cudaStream_t)stream, lanes);
+                                 (cudaStream_t)stream, cl.l);
     } else if (plan->path == HYENA_PATH_CLUSTER)
         e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     else if (pair_path_supported(plan->MC, batch))

@@ -25,7 +25,7 @@ cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, 
 // staged_workspace_rows(MC, rows) * MC complex64
 struct StagedLanes {
     cudaStream_t lane[2];     // non-blocking streams owned by the plan
-    cudaEvent_t fork, join[2];
+    cudaEvent_t fork, join[2];   // events of the calling operation only
 };
 bool staged_path_supported(int64_t MC);
 int64_t staged_chunk_rows(int64_t MC);

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "hyena.h"
 
 #define HYENA_MAX_L_1D 131072    // longest 1D sequence (M = 262144)
@@ -26,11 +28,14 @@ struct hyena_plan_s {
     // device tables (owned)
     int64_t tw_len = 0;          // 1D: M; 2D: 2W
     float2 *tw = nullptr;        // W_tw_len^m, m in [0, tw_len), then W_1024^m, m in [0, 1024)
-    // staged path: two non-blocking streams and the events that fork them off
-    // and join them back to the caller's stream
+    // staged paths: two non-blocking streams; each call forks them off its
+    // stream and joins them back with events of its own
     bool has_lanes = false;
     cudaStream_t lane[2] = {nullptr, nullptr};
-    cudaEvent_t fork = nullptr, join[2] = {nullptr, nullptr};
-    // staged spectra (1D long rows, 2D 256x256): scratch for two chunks of transforms (owned)
+    // staged spectra (1D long rows, 2D 256x256): scratch for two chunks of
+    // transforms (owned). Chunk slot i is only ever used by lane i, and the
+    // mutex keeps each call's launch sequence together on the lanes, so calls
+    // from several threads run one after the other on the GPU.
     float2 *spec_ws = nullptr;
+    std::mutex *spec_mu = nullptr;
 };
