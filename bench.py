@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="reference arm: oracle time of the W + K steps together")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--channels", type=int, default=None,
                     help="override the workload's channel count (small cases for profiling)")
@@ -369,9 +371,9 @@ def oracle_sample(w, seconds):
 def run_reference(args, w):
     """The reference arm: the oracle as it stands, W warm-up and K timed steps,
     each step a bounded sample of the workload's rows (sized so the whole run
-    takes about two minutes)."""
+    takes about --ref-seconds, two minutes by default)."""
     run, unit, threads, distinct = oracle_runner(w)
-    per_step = max(0.5, 120.0 / (args.steps + args.warmup))
+    per_step = max(0.25, args.ref_seconds / (args.steps + args.warmup))
     rows = calibrate_rows(run, threads, per_step)
     for _ in range(args.warmup):
         run(rows)

@@ -1,0 +1,36 @@
+"""bench.py on a host without a GPU: the reference arm (the fp64 oracle) prints
+its JSON line with the contract's keys, and our arm fails loudly instead of
+falling back to anything that runs on the CPU."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(*args, timeout=300):
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True, text=True,
+                          timeout=timeout)
+
+
+def test_reference_arm_prints_its_line():
+    out = _bench("--impl", "reference", "--steps", "2", "--warmup", "1", "--ref-seconds", "3")
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads(out.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference"
+    assert d["unit"] == "elems/s" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "order2_bf16_b8_d768_l2048"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="checks the behaviour on a host without a GPU")
+def test_our_arm_fails_without_a_gpu():
+    out = _bench("--steps", "1", "--warmup", "1", "--no-cpu-baseline", timeout=120)
+    assert out.returncode != 0
+    assert not out.stdout.strip()
