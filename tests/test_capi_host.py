@@ -65,3 +65,45 @@ def test_null_plan_rejected(capi):
     assert capi.hyena_implicit_filter(None, None, 16) == capi.HYENA_ERR_INVALID_ARG
     assert capi.hyena_forward_host_workspace_bytes(None, 4) == 0
     assert capi.hyena_forward_host(None, 1, 16, [16], 16, None, 16, 16, 1 << 20) == capi.HYENA_ERR_INVALID_ARG
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "hyena.h"
+
+int main(void) {
+    int bad = 0;
+    for (int s = HYENA_OK; s <= HYENA_ERR_NOMEM; ++s) {
+        const char *name = hyena_status_string((hyena_status_t)s);
+        if (!name || !name[0]) bad = 1;
+    }
+    const void *gates[1] = {0};
+    if (hyena_plan_destroy(NULL) != HYENA_OK) bad = 2;
+    if (hyena_workspace_bytes(NULL, 4) != 0) bad = 3;
+    if (hyena_forward_host_workspace_bytes(NULL, 4) != 0) bad = 4;
+    if (hyena_forward(NULL, 1, 0, gates, 0, NULL, 0, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 5;
+    if (hyena_forward_host(NULL, 1, 0, gates, 0, NULL, 0, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 6;
+    if (hyena_forward_no_alloc(NULL, 1, 0, gates, 0, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 7;
+    if (hyena_filter_spectrum(NULL, NULL, NULL, NULL, NULL) != HYENA_ERR_INVALID_ARG) bad = 8;
+    printf("%s\n", bad ? "FAIL" : "OK");
+    return bad;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(capi, tmp_path):
+    """include/hyena.h is a plain C header: a C99 program includes it with warnings as
+    errors, links libhyena.so and calls the entry points that need no GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "prog.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "prog"
+    pkg = os.path.dirname(capi.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", str(exe), "-L", pkg, "-lhyena", "-Wl,-rpath," + pkg])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0 and out.stdout.strip() == "OK", (out.returncode, out.stdout, out.stderr)
