@@ -9,7 +9,12 @@ same workload on its own GPU with its own seed, with no collective on the data
 path (weak scaling); the reported value is all ranks' elements divided by the
 slowest rank's time.
 
-Prints one JSON line on rank 0. See the design doc for the roofline arithmetic.
+Prints one JSON line on rank 0. The roofline object divides the operator's
+flop convention (5 M log2 M per transform, two transforms per row and order)
+by the kernel time, against the FP32 peak of 148 SMs x 128 lanes x 2 x the
+maximum SM clock; it also reports the HBM fraction against the measured copy
+bandwidth. e2e is the same metric through hyena_forward_host (page-locked host
+buffers, copies inside the timed region).
 """
 from __future__ import annotations
 
