@@ -34,3 +34,21 @@ def test_our_arm_fails_without_a_gpu():
     out = _bench("--steps", "1", "--warmup", "1", "--no-cpu-baseline", timeout=120)
     assert out.returncode != 0
     assert not out.stdout.strip()
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the multi-GPU run is (torchrun, two ranks), the reference arm runs on rank 0 only:
+    exactly one JSON line, and every rank exits 0."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "1", "--ref-seconds", "2"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0
