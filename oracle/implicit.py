@@ -1,8 +1,11 @@
 """Implicit filters of the Hyena operator, fp64 numpy. TEST INFRASTRUCTURE.
 
-Parity of these two functions is pinned only by special cases in which the
-network reduces to a closed form (see the CPU test suite); the network itself
-is a reading of the pages, not something they print.
+Parity of these two functions is pinned by special cases in which the
+network reduces to a closed form (see the CPU test suite): one feature through
+one unit per layer, the window alone, a non-zero bias in each hidden layer
+(which fixes the bias inside the sine's frequency), and an off-diagonal hidden
+weight (which fixes W2's orientation). The network itself is a reading of the
+pages, not something they print.
 
 1D filter ("Hyena — Long Convolutions Math", "Implicit filters: an MLP over
 positions" and "The decay window, and why it is not optional";

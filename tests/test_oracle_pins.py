@@ -312,3 +312,122 @@ def test_implicit_2d_reduces_to_closed_form(axis):
         np.testing.assert_allclose(k[0, c], expect, rtol=1e-13, atol=1e-15)
     # offset (0, 0) sits at [H, W] and has window 1 and coordinate 0
     np.testing.assert_array_equal(k[0, :, H, W], 0.0)
+
+
+# Bias placement and hidden-weight orientation. The one-hot pins above run with
+# zero biases and a symmetric W2, so they cannot tell sin(w0 (W1 g + b1)) from
+# sin(w0 W1 g) + b1, nor a1 W2^T from a1 W2. The nets below can: a non-zero
+# bias in the first unit of each hidden layer, and a W2 whose only entry sits
+# off the diagonal (unit 0 of layer 1 feeds unit 1 of layer 2, which the head
+# reads). The reading is the sine-network convention: each bias is added to
+# the pre-activation and scaled by that layer's frequency together with it
+# ("Hyena — Long Convolutions Math", "Implicit filters: an MLP over positions";
+# "How HyenaND works", "1. An implicit filter").
+
+def _biased_net(width, fin, out, feat_index, a, b1_0, b2_0):
+    W1, b1, W2, b2, W3, b3 = _onehot_net(width, fin, out, feat_index, a)
+    b1[0], b2[0] = b1_0, b2_0
+    return W1, b1, W2, b2, W3, b3
+
+
+def _offdiag_net(width, fin, out, feat_index, a, c):
+    W1 = np.zeros((width, fin)); W1[0, feat_index] = a
+    W2 = np.zeros((width, width)); W2[1, 0] = c       # layer-2 unit 1 reads layer-1 unit 0
+    W3 = np.zeros((out, width)); W3[:, 1] = 1.0       # the head reads layer-2 unit 1
+    return W1, np.zeros(width), W2, np.zeros(width), W3, np.zeros(out)
+
+
+def _closed_biased(f, a, b1_0, b2_0, w0, wh):
+    return np.sin(wh * (np.sin(w0 * (a * f + b1_0)) + b2_0))
+
+
+def _closed_offdiag(f, a, c, w0, wh):
+    return np.sin(wh * c * np.sin(w0 * a * f))
+
+
+def _check_1d_bias(fn_1d):
+    L, N, D, K, width = 48, 1, 2, 3, 8
+    a, b1_0, b2_0, w0, wh = 1.3, 0.4, -0.7, 1.1, 0.8
+    alpha = np.array([[0.0, 0.05]])
+    h = fn_1d(L, N, D, *_biased_net(width, 1 + 2 * K, N * D, 0, a, b1_0, b2_0), alpha, K, w0, wh)
+    t = np.arange(L)
+    base = _closed_biased(t / L, a, b1_0, b2_0, w0, wh)
+    for d in range(D):
+        np.testing.assert_allclose(h[0, d], np.exp(-alpha[0, d] * t) * base, rtol=1e-13, atol=1e-15)
+
+
+def _check_1d_offdiag(fn_1d):
+    L, N, D, K, width = 48, 2, 1, 3, 8
+    a, c, w0, wh = 1.9, 1.6, 0.7, 1.2
+    alpha = np.array([[0.02], [0.0]])
+    h = fn_1d(L, N, D, *_offdiag_net(width, 1 + 2 * K, N * D, 4, a, c), alpha, K, w0, wh)
+    t = np.arange(L)
+    base = _closed_offdiag(np.sin(2 * np.pi * 2 * t / L), a, c, w0, wh)   # feature 4 = sin(2 pi 2 t / L)
+    for n in range(N):
+        np.testing.assert_allclose(h[n, 0], np.exp(-alpha[n, 0] * t) * base, rtol=1e-13, atol=1e-15)
+
+
+def _check_2d_bias_offdiag(fn_2d):
+    H, W, N, C, width = 4, 4, 1, 2, 8
+    a, b1_0, b2_0, c, w0, wh = 0.6, 0.3, 0.5, -1.4, 10.0, 1.0
+    sigma = np.array([[0.5, 0.8]])
+    oy = np.arange(-H, H) / H
+    ox = np.arange(-W, W) / W
+    py, px = np.meshgrid(oy, ox, indexing="ij")
+    win = [np.exp(-(py ** 2 + px ** 2) / (2 * sigma[0, ch] ** 2)) for ch in range(C)]
+    k = fn_2d(H, W, N, C, *_biased_net(width, 2, N * C, 1, a, b1_0, b2_0), sigma, w0, wh)
+    for ch in range(C):
+        np.testing.assert_allclose(k[0, ch], win[ch] * _closed_biased(px, a, b1_0, b2_0, w0, wh),
+                                   rtol=1e-12, atol=1e-14)
+    k = fn_2d(H, W, N, C, *_offdiag_net(width, 2, N * C, 0, a, c), sigma, w0, wh)
+    for ch in range(C):
+        np.testing.assert_allclose(k[0, ch], win[ch] * _closed_offdiag(py, a, c, w0, wh), rtol=1e-12, atol=1e-14)
+
+
+def test_implicit_1d_bias_inside_the_frequency():
+    """b1, b2 non-zero: h = window * sin(w_h (sin(w0 (a f + b1_0)) + b2_0))."""
+    _check_1d_bias(oracle.implicit_filter_1d)
+
+
+def test_implicit_1d_hidden_weight_orientation():
+    """W2[1, 0] = c, head on unit 1: h = window * sin(w_h c sin(w0 a f)); W2 transposed gives 0."""
+    _check_1d_offdiag(oracle.implicit_filter_1d)
+
+
+def test_implicit_2d_bias_and_hidden_weight_orientation():
+    _check_2d_bias_offdiag(oracle.implicit_filter_2d)
+
+
+# Planted mistakes, in a copy of the network on the CPU: each must fail a pin above.
+def _mlp_bias_outside(feat, W1, b1, W2, b2, W3, b3, omega0, omega_hidden):
+    a1 = np.sin(omega0 * (feat @ W1.T)) + b1
+    a2 = np.sin(omega_hidden * (a1 @ W2.T)) + b2
+    return a2 @ W3.T + b3
+
+
+def _mlp_w2_transposed(feat, W1, b1, W2, b2, W3, b3, omega0, omega_hidden):
+    a1 = np.sin(omega0 * (feat @ W1.T + b1))
+    a2 = np.sin(omega_hidden * (a1 @ W2 + b2))
+    return a2 @ W3.T + b3
+
+
+def _mlp_bias_unscaled(feat, W1, b1, W2, b2, W3, b3, omega0, omega_hidden):
+    a1 = np.sin(omega0 * (feat @ W1.T) + b1)
+    a2 = np.sin(omega_hidden * (a1 @ W2.T) + b2)
+    return a2 @ W3.T + b3
+
+
+@pytest.mark.parametrize("planted,check", [
+    (_mlp_bias_outside, _check_1d_bias),
+    (_mlp_bias_unscaled, _check_1d_bias),
+    (_mlp_w2_transposed, _check_1d_offdiag),
+    (_mlp_bias_outside, _check_2d_bias_offdiag),
+    (_mlp_bias_unscaled, _check_2d_bias_offdiag),
+    (_mlp_w2_transposed, _check_2d_bias_offdiag),
+])
+def test_implicit_pins_catch_planted_mistakes(monkeypatch, planted, check):
+    import oracle.implicit as imp
+    monkeypatch.setattr(imp, "_mlp", planted)
+    fn = imp.implicit_filter_1d if check is not _check_2d_bias_offdiag else imp.implicit_filter_2d
+    with pytest.raises(AssertionError):
+        check(fn)
