@@ -3,8 +3,14 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 One step = one hyena_forward over the whole batch of the workload (all N
-orders, every row), inputs resident in HBM. The default workload is the
-order-2 bf16 B=8 D=768 L=2048 case. With N>1 (torchrun) every rank runs the
+orders, every row), inputs resident in HBM. The default (headline) workload is
+the order-3 bf16 B=1 D=768 L=65536 case, the longest single-GPU configuration
+of the operator (padded transform M = 131072). The same line carries a
+``workloads`` object with the other bench configurations (order-2 bf16 L=2048;
+order-2 bf16 L=8192 with implicit filters; the 2D order-1 256x256 grid), each
+measured the same way: ms per step, throughput, roofline fraction, DRAM
+traffic record, e2e, and the step with filter generation where the filters
+are implicit. With N>1 (torchrun) every rank runs the
 same workload on its own GPU with its own seed, with no collective on the data
 path (weak scaling); the reported value is all ranks' elements divided by the
 slowest rank's time.
@@ -31,7 +37,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "order2_bf16_b8_d768_l2048"
+DEFAULT_WORKLOAD = "order3_bf16_b1_d768_l65536"
+SIDE_WORKLOADS = ("order2_bf16_b8_d768_l2048", "order2_bf16_b4_d1024_l8192_implicit",
+                  "order1_bf16_2d_b2_c256_256x256")
 FP32_LANES_PER_SM = 128          # FP32 FMA lanes per SM (4 sub-partitions x 32)
 SM_MAX_MHZ_FALLBACK = 1965.0
 HBM_NOMINAL_GBS = 8000.0         # the operator's roofline convention (8 TB/s)
@@ -52,6 +60,8 @@ def parse():
     ap.add_argument("--channels", type=int, default=None,
                     help="override the workload's channel count (small cases for profiling)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="measure the selected workload only (no side workloads in the line)")
     return ap.parse_args()
 
 
@@ -267,6 +277,26 @@ def run_ours(args, w, rank, world, dist):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
+    # the copy-bound figure of this box: the same input bytes copied host to
+    # device from page-locked memory, one cudaMemcpyAsync per tensor on one stream
+    dv = torch.empty_like(hv, device=dev)
+    dg = [torch.empty_like(g, device=dev) for g in hg]
+
+    def copy_in():
+        dv.copy_(hv, non_blocking=True)
+        for a, b in zip(dg, hg):
+            a.copy_(b, non_blocking=True)
+    copy_in()
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(3):
+        copy_in()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    h2d_ms = c0.elapsed_time(c1) / 3
+    del dv, dg
+
     # implicit filters: also time the filter network and its spectrum with the
     # forward, per step (filters regenerated every step, as in training)
     filt_ms = 0.0
@@ -288,12 +318,15 @@ def run_ours(args, w, rank, world, dist):
         torch.cuda.synchronize()
         filt_ms = sum(a.elapsed_time(b) for a, b in zip(fs, fe)) / args.steps
 
-    ms, e2e_ms, filt_ms = max_over_ranks([ms, e2e_ms, filt_ms], dist, dev)
+    ms, e2e_ms, filt_ms, h2d_ms = max_over_ranks([ms, e2e_ms, filt_ms, h2d_ms], dist, dev)
     io = 4 if w.dtype == "f32" else 2
     h2d = (w.order + 1) * w.elements * io
     d2h = w.elements * io
     plan.close()
-    return ms, step_ms, e2e_ms, h2d, d2h, clk, launches, filt_ms
+    del v, gates, y, ws, flush, hws
+    torch.cuda.empty_cache()
+    return {"ms": ms, "step_ms": step_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "clk": clk,
+            "launches": launches, "filt_ms": filt_ms, "h2d_ms": h2d_ms}
 
 
 # ------------------------------------------------------------ oracle (CPU)
@@ -393,6 +426,53 @@ def run_reference(args, w):
     return value, sample, threads
 
 
+def traffic_record(w):
+    """DRAM bytes per launch of the workload's dominant kernel from the committed ncu
+    record, or None when there is none or the kernels changed since it was taken."""
+    prof = os.path.join(ROOT, "profiles", "traffic_%s.json" % w.name)
+    try:
+        with open(prof) as f:
+            pj = json.load(f)
+        from long_convolution_sequence_hyena_b200.build import source_hash
+        if pj.get("source_hash") == source_hash():
+            return pj.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def summarize(w, r, world):
+    """The per-workload numbers of one measurement (see run_ours)."""
+    cost = cost_model(w)
+    peaks, peak_src = measured_peaks()
+    sm_max = peaks.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)
+    fp32_peak, sms = device_fp32_peak_tflops(sm_max)
+    sec = r["ms"] * 1e-3
+    achieved_tflops = cost["flops"] / sec / 1e12
+    achieved_gbs = cost["bytes"] / sec / 1e9
+    t_roof = max(cost["bytes"] / (HBM_NOMINAL_GBS * 1e9), cost["flops"] / (fp32_peak * 1e12))
+    roof = {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak, "unit": "TFLOP/s",
+            "frac": achieved_tflops / fp32_peak, "traffic": traffic_record(w),
+            "peak_source": "FP32 FMA lanes x2 x max SM clock (%d SMs, %.0f MHz)" % (sms, sm_max),
+            "flops_convention": "5 M log2 M per transform, 2 transforms per row per order (M=%d)" % cost["M"],
+            "algorithmic_bytes": cost["bytes"],
+            "hbm_achieved_gbs": achieved_gbs, "hbm_peak_gbs": peaks.get("hbm_gbs"),
+            "hbm_frac": achieved_gbs / peaks.get("hbm_gbs", 6650.0), "hbm_peak_source": peak_src,
+            "operator_roofline_frac": t_roof / sec}
+    e2e = {"value": w.elements * world / (r["e2e_ms"] * 1e-3), "unit": "elems/s", "ms_per_step": r["e2e_ms"],
+           "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+           # copy-bound context: the step's input bytes over this box's measured pinned H2D rate
+           "h2d_gbs_measured": r["h2d"] / (r["h2d_ms"] * 1e-3) / 1e9, "h2d_ms_measured": r["h2d_ms"]}
+    out = {"ms_per_step": r["ms"], "value": job_throughput(w.elements, world, r["ms"]), "unit": "elems/s",
+           "roofline": roof, "e2e": e2e, "gpu_launches_per_step": r["launches"]}
+    if r["filt_ms"] > 0:
+        # the same metric with the implicit filter network and the filter spectra
+        # computed inside every step (the operator as used in training)
+        out["with_filter_generation"] = {"value": job_throughput(w.elements, world, r["filt_ms"]),
+                                         "unit": "elems/s", "ms_per_step": r["filt_ms"]}
+    return out
+
+
 def main():
     args = parse()
     from long_convolution_sequence_hyena_b200.workloads import WORKLOADS
@@ -426,53 +506,36 @@ def main():
         import torch.distributed as dist_mod
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
-    ms, step_ms, e2e_ms, h2d, d2h, clk, launches, filt_ms = run_ours(args, w, rank, world, dist)
+    r = run_ours(args, w, rank, world, dist)
+    side = {}
+    if not args.no_workloads and args.channels is None and args.batch is None:
+        for name in SIDE_WORKLOADS:
+            if name != w.name:
+                side[name] = run_ours(args, WORKLOADS[name], rank, world, dist)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    cost = cost_model(w)
-    peaks, peak_src = measured_peaks()
-    sm_max = peaks.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK)
-    fp32_peak, sms = device_fp32_peak_tflops(sm_max)
-    sec = ms * 1e-3
-    achieved_tflops = cost["flops"] / sec / 1e12
-    achieved_gbs = cost["bytes"] / sec / 1e9
-    t_roof = max(cost["bytes"] / (HBM_NOMINAL_GBS * 1e9), cost["flops"] / (fp32_peak * 1e12))
-    value = job_throughput(w.elements, world, ms)
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic_%s.json" % w.name)
-    try:
-        with open(prof) as f:
-            pj = json.load(f)
-        from long_convolution_sequence_hyena_b200.build import source_hash
-        if pj.get("source_hash") == source_hash():
-            traffic = pj.get("dram_bytes_per_launch")
-    except Exception:
-        traffic = None
+    head = summarize(w, r, world)
     line = {
-        "metric": metric, "value": value, "unit": "elems/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "metric": metric, "value": head["value"], "unit": "elems/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic", "config": cfg,
-        "roofline": {"bound": "alu", "achieved": achieved_tflops, "peak": fp32_peak, "unit": "TFLOP/s",
-                     "frac": achieved_tflops / fp32_peak, "traffic": traffic,
-                     "peak_source": "FP32 FMA lanes x2 x max SM clock (%d SMs, %.0f MHz)" % (sms, sm_max),
-                     "flops_convention": "5 M log2 M per transform, 2 transforms per row per order (M=%d)" % cost["M"],
-                     "hbm_achieved_gbs": achieved_gbs, "hbm_peak_gbs": peaks.get("hbm_gbs"),
-                     "hbm_frac": achieved_gbs / peaks.get("hbm_gbs", 6650.0), "hbm_peak_source": peak_src,
-                     "operator_roofline_frac": t_roof / sec},
-        "e2e": {"value": w.elements * world / (e2e_ms * 1e-3), "unit": "elems/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches,
-        "clocks": clk,
-        "step_ms_min": min(step_ms), "step_ms_max": max(step_ms),
+        "roofline": head["roofline"], "e2e": head["e2e"],
+        "gpu_launches": args.steps * r["launches"],
+        "clocks": r["clk"],
+        "step_ms_min": min(r["step_ms"]), "step_ms_max": max(r["step_ms"]),
     }
-    if filt_ms > 0:
-        # the same metric with the implicit filter network and the filter spectra
-        # computed inside every step (the operator as used in training)
-        line["with_filter_generation"] = {"value": job_throughput(w.elements, world, filt_ms), "unit": "elems/s",
-                                          "ms_per_step": filt_ms}
+    if "with_filter_generation" in head:
+        line["with_filter_generation"] = head["with_filter_generation"]
+    if side:
+        line["workloads"] = {}
+        for name, rs in side.items():
+            sw = WORKLOADS[name]
+            line["workloads"][name] = dict(summarize(sw, rs, world), clocks=rs["clk"],
+                                           config={"batch": sw.B, "channels": sw.D, "shape": list(sw.shape),
+                                                   "order": sw.order, "dtype": sw.dtype, "filters": sw.filt})
     if world == 1 and not args.no_cpu_baseline:
         cv, sample, threads, _ = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": cv, "unit": "elems/s", "cores": threads, "kind": "oracle", "sample": sample}

@@ -203,12 +203,16 @@ HYENA_API const char *hyena_status_string(hyena_status_t status);
  * The scratch is one array of HYENA_STATIC_SCRATCH_BYTES in device memory,
  * per device, held from when the library is loaded until the process exits.
  * Rows run in chunks of HYENA_STATIC_SCRATCH_BYTES / (M/2 * 8) rows (32 rows
- * at M = 131072); a plan whose row transform would not fit returns
- * HYENA_ERR_WORKSPACE. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current): make that first
- * call before any stream capture. Nothing in the array has to start at zero
- * (a chunk's transforms are written before they are read), but every call on
- * a device uses the same array: calls whose kernels overlap on the GPU (on
+ * at M = 131072, 64 at M = 65536), one chunk after another on `stream`,
+ * through the same kernels as hyena_forward, so y equals hyena_forward's bit
+ * for bit; a plan whose two-row transform would not fit returns
+ * HYENA_ERR_WORKSPACE. The first call in a CUDA context on a device looks up
+ * the array's device address (cudaGetSymbolAddress, with that device
+ * current): make that first call before any stream capture. The address is
+ * kept with the context's id, so after a device reset (a new context) the
+ * next call looks it up again. Nothing in the array has to start at zero (a
+ * chunk's transforms are written before they are read), but every call on a
+ * device uses the same array: calls whose kernels overlap on the GPU (on
  * different streams, or from different host threads) race; order them on one
  * stream or with events. This call allocates no memory.
  */

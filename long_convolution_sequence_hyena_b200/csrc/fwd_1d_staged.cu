@@ -118,15 +118,20 @@ cudaError_t launch_spec_1d_staged(const float *h, int64_t h_stride, int64_t L, c
     return le;
 }
 
+cudaError_t launch_fwd_1d_staged_chunks(const Fwd1dArgs &f, int64_t MC, float2 *ws, int64_t chunk, hyena_dtype_t dt,
+                                        bool even, const cudaStream_t *lanes, int nst) {
+    switch (MC) {
+        case 32768: return launch_staged_g<GS_32K>(f, ws, chunk, dt, even, lanes, nst);
+        case 65536: return launch_staged_g<GS_64K>(f, ws, chunk, dt, even, lanes, nst);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &f, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
                                  cudaStream_t st, const StagedLanes &sl) {
     const int64_t chunk = staged_chunk_rows(MC);
     auto run = [&](const cudaStream_t *lanes, int nst) -> cudaError_t {
-        switch (MC) {
-            case 32768: return launch_staged_g<GS_32K>(f, ws, chunk, dt, even, lanes, nst);
-            case 65536: return launch_staged_g<GS_64K>(f, ws, chunk, dt, even, lanes, nst);
-            default: return cudaErrorInvalidValue;
-        }
+        return launch_fwd_1d_staged_chunks(f, MC, ws, chunk, dt, even, lanes, nst);
     };
     if (f.rows <= chunk) return run(&st, 1);   // one chunk: the caller's stream only
     // fork the two lanes off the caller's stream, join them back at the end

@@ -11,19 +11,22 @@
 //
 // The scratch is one file-scope array of HYENA_STATIC_SCRATCH_BYTES per
 // device; every device that loads the library holds it until the process
-// exits. Rows run in chunks of as many rows as the array holds, through the
-// same column and row kernels as hyena_forward on HYENA_PATH_STAGED.
+// exits. Rows run in chunks of as many rows as the array holds, one chunk
+// after another on the caller's stream, through the same column and row
+// kernels (and the same launch sequence per chunk) as hyena_forward on
+// HYENA_PATH_STAGED, so each row's result is the same bit for bit.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "hyena.h"
-#include "kernels_1d_staged.cuh"
+#include "launch.h"
 #include "plan.h"
 
 // The scratch array (complex64 elements). In host code `scratch` names a
 // host-side stand-in, not device memory; its device address is looked up
-// once per device, with that device current (scratch_address below).
+// with the device current (scratch_address below).
 static __device__ __align__(256) float2 scratch[HYENA_STATIC_SCRATCH_BYTES / sizeof(float2)];
 
 namespace {
@@ -32,51 +35,62 @@ using namespace hyena;
 
 constexpr size_t kScratchBytes = HYENA_STATIC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
-float2 *g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
 
+// The array's address is a property of the CUDA context the module was
+// loaded into. It is cached per device together with the id of that context,
+// and looked up again when the current context is another one (after a
+// device reset, or when the primary context was released and created anew).
+struct ScratchCache {
+    unsigned long long ctx_id = 0;
+    float2 *ptr = nullptr;
+};
+ScratchCache g_cache[kMaxDevices];
+std::mutex g_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// The current context's id through the driver entry points the runtime hands
+// out (the library links only the runtime). 0 when it cannot be had.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+        cudaGetLastError();
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of the array for device `dev` (current). The first call in a
+// context looks it up with cudaGetSymbolAddress; later calls in the same
+// context reuse it.
 cudaError_t scratch_address(int dev, float2 **out) {
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    ScratchCache &c = g_cache[dev];
+    const unsigned long long id = current_context_id();
+    if (!c.ptr || id == 0 || id != c.ctx_id) {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, scratch);
+        const cudaError_t e = cudaGetSymbolAddress(&p, scratch);   // makes the context current if needed
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<float2 *>(p);
+        c.ptr = static_cast<float2 *>(p);
+        c.ctx_id = current_context_id();
     }
-    *out = g_scratch_ptr[dev];
+    *out = c.ptr;
     return cudaSuccess;
-}
-
-template <typename G, typename IO, bool EVEN>
-cudaError_t run_chunks(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cudaStream_t st) {
-    for (int64_t o0 = 0; o0 < f.rows; o0 += chunk) {
-        const int64_t nr = (f.rows - o0) < chunk ? (f.rows - o0) : chunk;
-        StagedArgs a;
-        a.f = f;
-        a.ws = ws;
-        a.o0 = o0;
-        a.n = 0;
-        hyena_staged_cols<G, IO, EVEN, 0><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
-        for (int n = 0; n < f.order; ++n) {
-            a.n = n;
-            hyena_staged_rows<G><<<(unsigned)(nr * G::RGROUPS), G::RT, G::RSMEM, st>>>(a);
-            if (n + 1 < f.order)
-                hyena_staged_cols<G, IO, EVEN, 1><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
-            else
-                hyena_staged_cols<G, IO, EVEN, 2><<<(unsigned)(nr * G::CGROUPS), G::CT, G::CSMEM, st>>>(a);
-        }
-        const cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
-template <typename G>
-cudaError_t run_geom(const Fwd1dArgs &f, float2 *ws, int64_t chunk, hyena_dtype_t dt, bool even, cudaStream_t st) {
-    if (dt == HYENA_F32)
-        return even ? run_chunks<G, float, true>(f, ws, chunk, st) : run_chunks<G, float, false>(f, ws, chunk, st);
-    return even ? run_chunks<G, __nv_bfloat16, true>(f, ws, chunk, st)
-                : run_chunks<G, __nv_bfloat16, false>(f, ws, chunk, st);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -87,10 +101,10 @@ extern "C" hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batc
                                                  const void *const *gates, const void *H, const float *Dskip,
                                                  void *y, void *stream) {
     if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
-    if (plan->path != HYENA_PATH_STAGED || (plan->MC != 32768 && plan->MC != 65536)) return HYENA_ERR_UNSUPPORTED;
-    // one row's transform (MC complex64) must fit the array: M <= kScratchBytes / 4
+    if (plan->path != HYENA_PATH_STAGED || !staged_path_supported(plan->MC)) return HYENA_ERR_UNSUPPORTED;
+    // two rows' transforms (MC complex64 each) must fit the array: the kernels run rows in pairs
     const size_t row_bytes = (size_t)plan->MC * sizeof(float2);
-    if (row_bytes > kScratchBytes) return HYENA_ERR_WORKSPACE;
+    if (2 * row_bytes > kScratchBytes) return HYENA_ERR_WORKSPACE;
     if (batch == 0) return HYENA_OK;
     if (!v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
     for (int n = 0; n < plan->order; ++n)
@@ -116,12 +130,9 @@ extern "C" hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batc
     a.D = plan->D;
     a.B = batch;
     a.order = plan->order;
-    const int64_t chunk = (int64_t)(kScratchBytes / row_bytes);
-    const bool even = (plan->L % 2) == 0;
+    const int64_t chunk = (int64_t)(kScratchBytes / row_bytes) & ~(int64_t)1;   // whole row pairs
     cudaStream_t st = (cudaStream_t)stream;
     const cudaError_t e =
-        plan->MC == 32768
-            ? run_geom<StagedGeom<32768, 128, 32, 16>>(a, ws, chunk, plan->dtype, even, st)
-            : run_geom<StagedGeom<65536, 256, 16, 16>>(a, ws, chunk, plan->dtype, even, st);
+        launch_fwd_1d_staged_chunks(a, plan->MC, ws, chunk, plan->dtype, (plan->L % 2) == 0, &st, 1);
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }

@@ -32,6 +32,10 @@ int64_t staged_chunk_rows(int64_t MC);
 int64_t staged_workspace_rows(int64_t MC, int64_t rows);
 cudaError_t launch_fwd_1d_staged(const Fwd1dArgs &a, int64_t MC, float2 *ws, hyena_dtype_t dt, bool even,
                                  cudaStream_t st, const StagedLanes &lanes);
+// The same launch sequence with an explicit chunk (rows per workspace slot) and
+// lanes: chunk c runs on lanes[c % nst] in slot c % nst of ws (nst slots).
+cudaError_t launch_fwd_1d_staged_chunks(const Fwd1dArgs &f, int64_t MC, float2 *ws, int64_t chunk, hyena_dtype_t dt,
+                                        bool even, const cudaStream_t *lanes, int nst);
 // 1D filter spectra through the staged kernels, with plan-owned scratch of
 // staged_spec_scratch_bytes(MC)
 size_t staged_spec_scratch_bytes(int64_t MC);

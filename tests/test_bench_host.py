@@ -23,7 +23,7 @@ def test_reference_arm_prints_its_line():
     assert d["impl"] == "reference"
     assert d["unit"] == "elems/s" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
-    assert d["config"]["workload"] == "order2_bf16_b8_d768_l2048"
+    assert d["config"]["workload"] == "order3_bf16_b1_d768_l65536"   # the headline: longest single-GPU case
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "elems/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -2,12 +2,14 @@
 memory where they run the operator (a plain C host program without an
 allocator of its own, a process whose device memory belongs to a framework's
 allocator, a loop that must not call cudaMalloc). Its scratch is a fixed
-device array inside the library, so it takes no workspace. Its output must
-match hyena_forward's, call after call, because every call reuses the same
-array.
+device array inside the library, so it takes no workspace. It runs the same
+kernels as hyena_forward over smaller chunks, so its output must equal
+hyena_forward's, call after call, because every call reuses the same array;
+sampled rows are also checked against the fp64 oracle directly.
 
 This file is collected last, so that a failure here stops a run only after
 every other test has run."""
+import numpy as np
 import pytest
 import torch
 
@@ -22,8 +24,11 @@ def _rel_l2(a, b):
 @pytest.mark.parametrize("L,B,D,N,dtype,tol", [
     (32768, 1, 70, 2, torch.float32, 1e-5),    # 70 rows: two chunks of the 64 rows the array holds
     (65536, 2, 20, 3, torch.bfloat16, 2e-2),   # 40 rows: two chunks of 32
+    (16385, 3, 1, 2, torch.float32, 1e-5),     # odd length, odd row count (the last pair has one row)
+    (40001, 1, 35, 1, torch.bfloat16, 2e-2),   # odd length at M = 131072, two chunks, odd rows
 ])
 def test_no_alloc_matches_forward_twice(L, B, D, N, dtype, tol):
+    import oracle
     from long_convolution_sequence_hyena_b200 import api, capi
 
     plan = api.Plan((L,), D, N, dtype)
@@ -48,6 +53,17 @@ def test_no_alloc_matches_forward_twice(L, B, D, N, dtype, tol):
         assert torch.isfinite(y.float()).all()
         err = _rel_l2(y, y_ref)
         assert err <= tol, (call, err)
+        assert torch.equal(y, y_ref), call      # same kernels, same per-row arithmetic
+    # a few rows against the fp64 oracle (first, last, and one in the second chunk)
+    R = B * D
+    rows = sorted({0, R - 1, min(R - 1, 33)})
+    v64 = v.double().cpu().reshape(R, L).numpy()[rows]
+    g64 = np.stack([x.double().cpu().reshape(R, L).numpy()[rows] for x in gates])
+    ref = oracle.hyena_1d(v64, g64, h.double().cpu().numpy(), dskip.double().cpu().numpy(),
+                          fidx=np.array(rows) % D)
+    got = y.double().cpu().reshape(R, L).numpy()[rows]
+    err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert err <= tol, err
     plan.close()
 
 
