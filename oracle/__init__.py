@@ -12,6 +12,8 @@ Contents
   direct O((HW)^2) sum, in C.
 * ``implicit_filter_1d`` / ``implicit_filter_2d`` -- the implicit filters in
   numpy fp64 (``implicit.py``).
+* ``hyena_gated`` / ``silu`` -- the HyenaND gate sandwich (inner gate
+  q ⊙ SiLU(k), outer gates SiLU(x^n)) around the same chains (``gated.py``).
 
 All arrays are float64 numpy arrays; callers pass the exact values the GPU path
 receives (bf16 inputs are widened exactly before they get here).
@@ -24,6 +26,7 @@ import subprocess
 
 import numpy as np
 
+from .gated import hyena_gated, silu  # noqa: F401
 from .implicit import implicit_filter_1d, implicit_filter_2d, positional_features_1d  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

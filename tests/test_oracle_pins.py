@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import scipy.linalg
 import scipy.signal
+import scipy.special
 
 import oracle
 
@@ -431,3 +432,58 @@ def test_implicit_pins_catch_planted_mistakes(monkeypatch, planted, check):
     fn = imp.implicit_filter_1d if check is not _check_2d_bias_offdiag else imp.implicit_filter_2d
     with pytest.raises(AssertionError):
         check(fn)
+
+
+# ------------------------------------------------------------ gate sandwich --
+# "How HyenaND works", "Putting it together: the HyenaND operator":
+# Z = q ⊙ SiLU(k), H = K ∗ Z, O = H ⊙ SiLU(v).
+
+def test_silu_special_values():
+    s = oracle.silu(np.array([0.0, 1.0, -1.0, 40.0, -40.0, 800.0, -800.0]))
+    assert s[0] == 0.0
+    assert s[1] == pytest.approx(1.0 / (1.0 + np.exp(-1.0)), rel=1e-15)           # 0.7310585786300049
+    assert s[2] == pytest.approx(-1.0 / (1.0 + np.exp(1.0)), rel=1e-15)
+    assert s[3] == pytest.approx(40.0, rel=1e-15) and abs(s[4]) < 1e-15          # SiLU(x) -> x, -> 0
+    assert s[5] == 800.0 and s[6] == 0.0 and np.all(np.isfinite(s))              # no overflow
+    x = np.linspace(-12, 12, 2001)
+    np.testing.assert_allclose(oracle.silu(x), x * scipy.special.expit(x), rtol=1e-14, atol=1e-300)
+
+
+def test_gated_2d_delta_kernel_is_the_gates_alone():
+    """K = δ at offset 0: y = SiLU(x) · (1 + Dskip) · q · SiLU(k), element by element."""
+    rng = np.random.default_rng(41)
+    P, H, W = 3, 5, 4
+    q, k, x = rng.standard_normal((3, P, H, W))
+    kern = np.zeros((1, P, 2 * H, 2 * W)); kern[0, :, H, W] = 1.0
+    dsk = rng.standard_normal((1, P))
+    y = oracle.hyena_gated(q, k, x[None], kern, dsk)
+    sig = lambda a: a * scipy.special.expit(a)
+    np.testing.assert_allclose(y, sig(x) * (1.0 + dsk[0][:, None, None]) * q * sig(k), rtol=1e-13, atol=1e-14)
+
+
+def test_gated_2d_matches_scipy_with_both_gates():
+    """O = (K ∗ (q ⊙ SiLU(k))) ⊙ SiLU(v) with scipy's full 2D convolution cropped at offset 0."""
+    rng = np.random.default_rng(42)
+    P, H, W = 2, 6, 7
+    q, k, v = rng.standard_normal((3, P, H, W))
+    kern = rng.standard_normal((1, P, 2 * H, 2 * W))
+    y = oracle.hyena_gated(q, k, v[None], kern)
+    sig = lambda a: a * scipy.special.expit(a)
+    for p in range(P):
+        c = scipy.signal.convolve2d(q[p] * sig(k[p]), kern[0, p])[H:2 * H, W:2 * W]
+        np.testing.assert_allclose(y[p], c * sig(v[p]), rtol=1e-11, atol=1e-11)
+
+
+def test_gated_saturated_gates_reduce_to_the_plain_operator():
+    """k, x -> +inf make both SiLU gates the identity on k and x scaled out: with k = x = 50
+    the sandwich equals 50 · 50 · (plain chain on q with unit gates)."""
+    rng = np.random.default_rng(43)
+    R, L = 3, 40
+    q = rng.standard_normal((R, L))
+    h = rng.standard_normal((1, R, L)) * np.exp(-0.1 * np.arange(L))
+    y = oracle.hyena_gated(q, np.full((R, L), 50.0), np.full((1, R, L), 50.0), h)
+    plain = oracle.hyena_1d(q, np.ones((1, R, L)), h)
+    np.testing.assert_allclose(y, 2500.0 * plain, rtol=1e-13, atol=1e-13)
+    # and k -> -inf closes the inner gate: the output is zero
+    y0 = oracle.hyena_gated(q, np.full((R, L), -800.0), rng.standard_normal((1, R, L)), h)
+    assert np.all(y0 == 0.0)
