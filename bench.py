@@ -7,7 +7,8 @@ orders, every row), inputs resident in HBM. The default (headline) workload is
 the order-3 bf16 B=1 D=768 L=65536 case, the longest single-GPU configuration
 of the operator (padded transform M = 131072). The same line carries a
 ``workloads`` object with the other bench configurations (order-2 bf16 L=2048;
-order-2 bf16 L=8192 with implicit filters; the 2D order-1 256x256 grid), each
+order-2 bf16 L=8192 with implicit filters; the 2D order-1 256x256 grid, plain
+and through the HyenaND gate sandwich), each
 measured the same way: ms per step, throughput, roofline fraction, DRAM
 traffic record, e2e, and the step with filter generation where the filters
 are implicit. With N>1 (torchrun) every rank runs the
@@ -39,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "order3_bf16_b1_d768_l65536"
 SIDE_WORKLOADS = ("order2_bf16_b8_d768_l2048", "order2_bf16_b4_d1024_l8192_implicit",
-                  "order1_bf16_2d_b2_c256_256x256")
+                  "order1_bf16_2d_b2_c256_256x256", "gated_order1_bf16_2d_b2_c256_256x256")
 FP32_LANES_PER_SM = 128          # FP32 FMA lanes per SM (4 sub-partitions x 32)
 SM_MAX_MHZ_FALLBACK = 1965.0
 HBM_NOMINAL_GBS = 8000.0         # the operator's roofline convention (8 TB/s)
@@ -69,7 +70,8 @@ def parse():
 def cost_model(w):
     """Algorithmic flops and bytes of one step (whole batch), per the operator's
     roofline convention: 5 M log2 M flops per transform, two transforms per row
-    per order; bytes = v, N gates and y once each, plus every spectrum row once."""
+    per order; bytes = v (q and k for the gate sandwich), N gates and y once each, plus
+    every spectrum row once."""
     io = 4 if w.dtype == "f32" else 2
     N = w.order
     if w.ndim == 1:
@@ -84,7 +86,7 @@ def cost_model(w):
         transforms = 2 * N * w.B * w.D
         flops = transforms * 5.0 * M * math.log2(M)
         spec_bytes = N * w.D * (2 * H) * (W + 1) * 8
-    act_bytes = (N + 2) * w.elements * io
+    act_bytes = (N + 2 + (1 if w.gated else 0)) * w.elements * io   # the gate sandwich also reads k
     return {"flops": flops, "bytes": act_bytes + spec_bytes + N * w.D * 4, "M": M}
 
 
@@ -213,13 +215,21 @@ def run_ours(args, w, rank, world, dist):
     # enqueues its kernels with as little host work as possible
     import ctypes
     garr = (ctypes.c_void_p * len(gptrs))(*gptrs)
-    fwd_args = (plan.handle, w.B, v.data_ptr(), garr, H.data_ptr(), dskip.data_ptr(), y.data_ptr(),
-                ws.data_ptr() if ws_bytes else None, ws_bytes, sptr)
+    if w.gated:
+        # the gate sandwich: v is q, and the key k forms the inner gate q SiLU(k)
+        kdev = inp["k"].to(dev)
+        fwd_fn, fwd_name = capi.lib.hyena_forward_gated, "hyena_forward_gated"
+        fwd_args = (plan.handle, w.B, v.data_ptr(), kdev.data_ptr(), garr, H.data_ptr(), dskip.data_ptr(),
+                    y.data_ptr(), ws.data_ptr() if ws_bytes else None, ws_bytes, sptr)
+    else:
+        fwd_fn, fwd_name = capi.lib.hyena_forward, "hyena_forward"
+        fwd_args = (plan.handle, w.B, v.data_ptr(), garr, H.data_ptr(), dskip.data_ptr(), y.data_ptr(),
+                    ws.data_ptr() if ws_bytes else None, ws_bytes, sptr)
 
     def step():
-        st = capi.lib.hyena_forward(*fwd_args)
+        st = fwd_fn(*fwd_args)
         if st != capi.HYENA_OK:
-            raise RuntimeError("hyena_forward: " + capi.hyena_status_string(st))
+            raise RuntimeError(fwd_name + ": " + capi.hyena_status_string(st))
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -247,7 +257,11 @@ def run_ours(args, w, rank, world, dist):
     ms = sum(step_ms) / len(step_ms)
 
     # end to end through the C ABI with HOST buffers: hyena_forward_host copies the
-    # page-locked inputs in and the output back, pipelined over the batch
+    # page-locked inputs in and the output back, pipelined over the batch (the plain
+    # operator only: the gate sandwich has no host-buffer entry point)
+    if w.gated:
+        return finish_gated(args, w, dist, dev, plan, ms, step_ms, clk, launches, imp if "implicit" in inp else None,
+                            H, stream, step, flush)
     hv = inp["v"].pin_memory()
     hg = [g.pin_memory() for g in inp["gates"]]
     hy = torch.empty_like(hv).pin_memory()
@@ -327,6 +341,34 @@ def run_ours(args, w, rank, world, dist):
     torch.cuda.empty_cache()
     return {"ms": ms, "step_ms": step_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h, "clk": clk,
             "launches": launches, "filt_ms": filt_ms, "h2d_ms": h2d_ms}
+
+
+def finish_gated(args, w, dist, dev, plan, ms, step_ms, clk, launches, imp, H, stream, step, flush):
+    """The rest of run_ours for the gate sandwich: the step with filter generation (implicit
+    kernels), no host-buffer leg."""
+    import torch
+    filt_ms = 0.0
+    if imp is not None:
+        def filt_step():
+            plan.filter_spectrum(implicit=imp, out=H, stream=stream)
+            step()
+        for _ in range(args.warmup):
+            flush.zero_()
+            filt_step()
+        torch.cuda.synchronize()
+        fs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            fs[i].record(stream)
+            filt_step()
+            fe[i].record(stream)
+        torch.cuda.synchronize()
+        filt_ms = sum(a.elapsed_time(b) for a, b in zip(fs, fe)) / args.steps
+    ms, filt_ms = max_over_ranks([ms, filt_ms], dist, dev)
+    plan.close()
+    return {"ms": ms, "step_ms": step_ms, "e2e_ms": None, "h2d": 0, "d2h": 0, "clk": clk,
+            "launches": launches, "filt_ms": filt_ms, "h2d_ms": None}
 
 
 # ------------------------------------------------------------ oracle (CPU)
@@ -459,10 +501,12 @@ def summarize(w, r, world):
             "hbm_achieved_gbs": achieved_gbs, "hbm_peak_gbs": peaks.get("hbm_gbs"),
             "hbm_frac": achieved_gbs / peaks.get("hbm_gbs", 6650.0), "hbm_peak_source": peak_src,
             "operator_roofline_frac": t_roof / sec}
-    e2e = {"value": w.elements * world / (r["e2e_ms"] * 1e-3), "unit": "elems/s", "ms_per_step": r["e2e_ms"],
-           "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-           # copy-bound context: the step's input bytes over this box's measured pinned H2D rate
-           "h2d_gbs_measured": r["h2d"] / (r["h2d_ms"] * 1e-3) / 1e9, "h2d_ms_measured": r["h2d_ms"]}
+    e2e = None
+    if r["e2e_ms"] is not None:
+        e2e = {"value": w.elements * world / (r["e2e_ms"] * 1e-3), "unit": "elems/s", "ms_per_step": r["e2e_ms"],
+               "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+               # copy-bound context: the step's input bytes over this box's measured pinned H2D rate
+               "h2d_gbs_measured": r["h2d"] / (r["h2d_ms"] * 1e-3) / 1e9, "h2d_ms_measured": r["h2d_ms"]}
     out = {"ms_per_step": r["ms"], "value": job_throughput(w.elements, world, r["ms"]), "unit": "elems/s",
            "roofline": roof, "e2e": e2e, "gpu_launches_per_step": r["launches"]}
     if r["filt_ms"] > 0:

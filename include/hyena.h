@@ -183,6 +183,28 @@ HYENA_API hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const v
                              const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
                              void *stream);
 
+/*
+ * The gate sandwich of HyenaND ("How HyenaND works", "How HyenaND stays
+ * data-dependent: gating" and "Putting it together: the HyenaND operator"):
+ * the inner gate Z = q ⊙ SiLU(k) is the convolution's input and every outer
+ * gate passes through SiLU, SiLU(x) = x / (1 + e^{-x}):
+ *
+ *     z^0 = q ⊙ SiLU(k)
+ *     z^n = SiLU(x^n) ⊙ ( K^n ∗ z^{n-1}  +  Dskip^n ⊙ z^{n-1} )     n = 1..N
+ *     y   = z^N
+ *
+ * With one order, no Dskip and gates = {v} this is the page's
+ * O = (K ∗ (q ⊙ SiLU(k))) ⊙ SiLU(v). Both gates are formed inside the
+ * forward's first load and its gate multiplies (no extra pass over memory).
+ *   q, k   [B, C, H, W] io dtype (device), in place of hyena_forward's v
+ * The other arguments, the workspace and the aliasing rule (y may alias q, k
+ * or a gate) are those of hyena_forward. 2D plans only; 1D plans return
+ * HYENA_ERR_UNSUPPORTED.
+ */
+HYENA_API hyena_status_t hyena_forward_gated(hyena_plan_t plan, int64_t batch, const void *q, const void *k,
+                                             const void *const *gates, const void *H, const float *Dskip,
+                                             void *y, void *workspace, size_t ws_bytes, void *stream);
+
 /* Static, human-readable name of a status code. */
 HYENA_API const char *hyena_status_string(hyena_status_t status);
 

@@ -115,6 +115,21 @@ class Plan:
         _check(st, "hyena_forward")
         return out
 
+    def forward_gated(self, q, k, gates, H, dskip=None, out=None, workspace=None, stream=None):
+        """The HyenaND gate sandwich: y = SiLU(x^N) (K^N * (... SiLU(x^1) (K^1 * (q SiLU(k)))));
+        with one order, (K * (q SiLU(k))) SiLU(v) for gates = [v]."""
+        if out is None:
+            out = torch.empty_like(q)
+        ws = workspace
+        need = self.workspace_bytes(q.shape[0])
+        if ws is None and need:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        st = capi.hyena_forward_gated(self.handle, q.shape[0], q.data_ptr(), k.data_ptr(),
+                                      [g.data_ptr() for g in gates], H.data_ptr(), _ptr(dskip), out.data_ptr(),
+                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+        _check(st, "hyena_forward_gated")
+        return out
+
     def host_workspace_bytes(self, batch: int) -> int:
         return capi.hyena_forward_host_workspace_bytes(self.handle, batch)
 

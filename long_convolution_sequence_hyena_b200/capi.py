@@ -31,6 +31,7 @@ EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
+    "hyena_forward_gated",
 )
 
 
@@ -63,6 +64,7 @@ def _load():
         "hyena_forward_no_alloc": ([p, i64, p, ctypes.POINTER(p), p, p, p, p], i32),
         "hyena_forward_host_workspace_bytes": ([p, i64], sz),
         "hyena_forward_host": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
+        "hyena_forward_gated": ([p, i64, p, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -113,6 +115,13 @@ def hyena_forward(plan, batch: int, v: int, gates, H: int, Dskip, y: int, worksp
                   stream: int = 0) -> int:
     garr = None if gates is None else (ctypes.c_void_p * len(gates))(*gates)
     return lib.hyena_forward(plan, batch, v, garr, H, Dskip, y, workspace, ws_bytes, stream)
+
+
+def hyena_forward_gated(plan, batch: int, q: int, k: int, gates, H: int, Dskip, y: int, workspace=None,
+                        ws_bytes: int = 0, stream: int = 0) -> int:
+    """The gate sandwich: z^0 = q SiLU(k), z^n = SiLU(x^n) (K^n * z^{n-1} + Dskip^n z^{n-1})."""
+    garr = None if gates is None else (ctypes.c_void_p * len(gates))(*gates)
+    return lib.hyena_forward_gated(plan, batch, q, k, garr, H, Dskip, y, workspace, ws_bytes, stream)
 
 
 def hyena_forward_no_alloc(plan, batch: int, v: int, gates, H: int, Dskip, y: int, stream: int = 0) -> int:

@@ -7,8 +7,12 @@ namespace hyena {
 
 template <typename G>
 cudaError_t launch_fwd_2d_g(const Fwd2dArgs &a, hyena_dtype_t dt, cudaStream_t st) {
-    if (dt == HYENA_F32) return launch_cluster<G>(hyena_fwd_2d_cluster<G, float>, a.planes, st, a);
-    return launch_cluster<G>(hyena_fwd_2d_cluster<G, __nv_bfloat16>, a.planes, st, a);
+    const bool gated = a.k != nullptr;
+    if (dt == HYENA_F32)
+        return gated ? launch_cluster<G>(hyena_fwd_2d_cluster<G, float, true>, a.planes, st, a)
+                     : launch_cluster<G>(hyena_fwd_2d_cluster<G, float, false>, a.planes, st, a);
+    return gated ? launch_cluster<G>(hyena_fwd_2d_cluster<G, __nv_bfloat16, true>, a.planes, st, a)
+                 : launch_cluster<G>(hyena_fwd_2d_cluster<G, __nv_bfloat16, false>, a.planes, st, a);
 }
 
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st) {

@@ -19,7 +19,7 @@ int64_t staged2d_workspace_planes(int64_t W, int64_t planes) {
     return planes <= r ? planes : 2 * r;
 }
 
-template <typename G, typename IO>
+template <typename G, typename IO, bool GATED>
 cudaError_t launch_staged2d_io(const Fwd2dArgs &f, float2 *ws, int64_t chunk, const cudaStream_t *lanes, int nst) {
     cudaError_t e = cudaFuncSetAttribute(hyena_staged2d_rows_x2<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)G::RSMEM);
@@ -33,14 +33,14 @@ cudaError_t launch_staged2d_io(const Fwd2dArgs &f, float2 *ws, int64_t chunk, co
         a.o0 = o0;
         a.n = 0;
         const unsigned cgrid = (unsigned)(np * G::CGROUPS), rgrid = (unsigned)((np + 1) / 2 * G::RGROUPS);
-        hyena_staged2d_cols<G, IO, 0><<<cgrid, G::CT, G::CSMEM, st>>>(a);
+        hyena_staged2d_cols<G, IO, 0, GATED><<<cgrid, G::CT, G::CSMEM, st>>>(a);
         for (int n = 0; n < f.order; ++n) {
             a.n = n;
             hyena_staged2d_rows_x2<G><<<rgrid, G::RT, G::RSMEM, st>>>(a, np);
             if (n + 1 < f.order)
-                hyena_staged2d_cols<G, IO, 1><<<cgrid, G::CT, G::CSMEM, st>>>(a);
+                hyena_staged2d_cols<G, IO, 1, GATED><<<cgrid, G::CT, G::CSMEM, st>>>(a);
             else
-                hyena_staged2d_cols<G, IO, 2><<<cgrid, G::CT, G::CSMEM, st>>>(a);
+                hyena_staged2d_cols<G, IO, 2, GATED><<<cgrid, G::CT, G::CSMEM, st>>>(a);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -100,8 +100,11 @@ cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyen
     if (W != 256) return cudaErrorInvalidValue;
     const int64_t chunk = staged2d_chunk_planes(W);
     auto run = [&](const cudaStream_t *lanes, int nst) -> cudaError_t {
-        return dt == HYENA_F32 ? launch_staged2d_io<GS2_256, float>(f, ws, chunk, lanes, nst)
-                               : launch_staged2d_io<GS2_256, __nv_bfloat16>(f, ws, chunk, lanes, nst);
+        if (f.k)
+            return dt == HYENA_F32 ? launch_staged2d_io<GS2_256, float, true>(f, ws, chunk, lanes, nst)
+                                   : launch_staged2d_io<GS2_256, __nv_bfloat16, true>(f, ws, chunk, lanes, nst);
+        return dt == HYENA_F32 ? launch_staged2d_io<GS2_256, float, false>(f, ws, chunk, lanes, nst)
+                               : launch_staged2d_io<GS2_256, __nv_bfloat16, false>(f, ws, chunk, lanes, nst);
     };
     if (f.planes <= chunk) return run(&st, 1);
     cudaError_t e = cudaEventRecord(sl.fork, st);

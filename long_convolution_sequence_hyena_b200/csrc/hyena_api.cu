@@ -306,11 +306,17 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
-hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, const void *const *gates, const void *H,
-                             const float *Dskip, void *y, void *workspace, size_t ws_bytes, void *stream) {
-    if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
-    if (batch == 0) return HYENA_OK;  // nothing to read or write; pointers may be NULL
+}  // extern "C"
+
+namespace {
+
+// The forward of both entry points: k == nullptr is the plain operator, else
+// the gate sandwich (z^0 = v SiLU(k), SiLU of every gate).
+hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, const void *k, const void *const *gates,
+                            const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
+                            void *stream) {
     if (!v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
+    if (k && !aligned16(k)) return HYENA_ERR_ALIGNMENT;
     for (int n = 0; n < plan->order; ++n)
         if (!gates[n]) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(v) || !aligned16(H) || !aligned16(y) || (Dskip && !aligned4(Dskip))) return HYENA_ERR_ALIGNMENT;
@@ -326,6 +332,7 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
         Fwd2dArgs a;
         std::memset(&a, 0, sizeof(a));
         a.v = v;
+        a.k = k;
         for (int n = 0; n < plan->order; ++n) a.gates[n] = gates[n];
         a.K = reinterpret_cast<const c32 *>(H);
         a.dskip = Dskip;
@@ -373,6 +380,27 @@ hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, co
     else
         e = launch_fwd_1d(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+hyena_status_t hyena_forward(hyena_plan_t plan, int64_t batch, const void *v, const void *const *gates, const void *H,
+                             const float *Dskip, void *y, void *workspace, size_t ws_bytes, void *stream) {
+    if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
+    if (batch == 0) return HYENA_OK;  // nothing to read or write; pointers may be NULL
+    return forward_impl(plan, batch, v, nullptr, gates, H, Dskip, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_forward_gated(hyena_plan_t plan, int64_t batch, const void *q, const void *k,
+                                   const void *const *gates, const void *H, const float *Dskip, void *y,
+                                   void *workspace, size_t ws_bytes, void *stream) {
+    if (!plan || batch < 0) return HYENA_ERR_INVALID_ARG;
+    if (plan->ndim == 1) return HYENA_ERR_UNSUPPORTED;
+    if (batch == 0) return HYENA_OK;
+    if (!k) return HYENA_ERR_INVALID_ARG;
+    return forward_impl(plan, batch, q, k, gates, H, Dskip, y, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

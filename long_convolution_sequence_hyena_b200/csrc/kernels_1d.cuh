@@ -51,6 +51,13 @@ struct io<__nv_bfloat16> {
     __device__ __forceinline__ static pair_t zero() { return __floats2bfloat162_rn(0.f, 0.f); }
 };
 
+// SiLU(x) = x σ(x) = x / (1 + e^{-x}) for the gate sandwich of HyenaND
+// ("How HyenaND works", "Putting it together: the HyenaND operator"). For
+// x -> -inf, e^{-x} overflows to +inf and the quotient is -0; for x -> +inf it
+// is x.
+__device__ __forceinline__ float silu(float x) { return x / (1.f + expf(-x)); }
+__device__ __forceinline__ c32 silu(c32 a) { return mk(silu(a.x), silu(a.y)); }
+
 // Load positions (pos, pos+1) of a row of length L, zero beyond L.
 // EVEN: L is even, so the pair is either fully inside or fully outside and the
 // pair load is aligned.

@@ -19,7 +19,8 @@
 namespace hyena {
 
 struct Fwd2dArgs {
-    const void *v;
+    const void *v;        // the convolution input; with the gate sandwich, q
+    const void *k;        // gate sandwich only: the inner gate's key (z^0 = q SiLU(k))
     const void *gates[HYENA_MAX_ORDER];
     const c32 *K;         // [N, C, W + 1, 2H]: bin (ky, kx) at kx * 2H + ky
     const float *dskip;   // [N, C] or nullptr
@@ -31,8 +32,10 @@ struct Fwd2dArgs {
     int order;
 };
 
-// Fused order-N 2D forward (planes visited c-major, b-minor).
-template <typename G, typename IO>
+// Fused order-N 2D forward (planes visited c-major, b-minor). GATED: the
+// gate sandwich, z^0 = q SiLU(k) formed at the load and SiLU applied to every
+// gate x^n where it multiplies.
+template <typename G, typename IO, bool GATED>
 __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(const Fwd2dArgs a) {
     using Ctx = ClusterCtx<G, false, true>;
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2;
@@ -55,8 +58,15 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
     c32 v[E];
     {
         const IO *vp = reinterpret_cast<const IO *>(a.v) + plane * Hh * Ww;
+        const IO *kp = reinterpret_cast<const IO *>(a.k) + plane * Hh * Ww;
 #pragma unroll
-        for (int q = 0; q < E1 / 2; ++q) v[q] = load_pair<IO, true>(vp, pos_of(q), (int64_t)Hh * Ww);
+        for (int q = 0; q < E1 / 2; ++q) {
+            v[q] = load_pair<IO, true>(vp, pos_of(q), (int64_t)Hh * Ww);
+            if constexpr (GATED) {
+                const c32 kq = silu(load_pair<IO, true>(kp, pos_of(q), (int64_t)Hh * Ww));
+                v[q] = mk(v[q].x * kq.x, v[q].y * kq.y);
+            }
+        }
 #pragma unroll
         for (int q = E1 / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
@@ -124,7 +134,8 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_2d_cluster(cons
         cx.inverse(v, a.tw);
 #pragma unroll
         for (int q = 0; q < E1 / 2; ++q) {
-            const c32 gq = io<IO>::unpack(g[q]);
+            c32 gq = io<IO>::unpack(g[q]);
+            if constexpr (GATED) gq = silu(gq);
             v[q] = mk(gq.x * v[q].x, gq.y * v[q].y);
         }
 #pragma unroll

@@ -56,8 +56,9 @@ __device__ __forceinline__ int64_t visit_plane(const Fwd2dArgs &f, int64_t o, in
 }
 
 // MODE 0: load v, forward columns; 1: inverse columns, gate x^n, forward
-// columns; 2: inverse columns, gate x^n, store y.
-template <typename G, typename IO, int MODE>
+// columns; 2: inverse columns, gate x^n, store y. GATED: the gate sandwich
+// (z^0 = q SiLU(k) at the load, SiLU of every gate where it multiplies).
+template <typename G, typename IO, int MODE, bool GATED>
 __global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dArgs a) {
     constexpr int E = G::E, M1 = G::M1, XW = G::XW, T1 = G::T1, Hh = G::Hh, Ww = G::Ww;
     extern __shared__ float smem[];
@@ -76,8 +77,15 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dAr
     c32 v[E];
     if constexpr (MODE == 0) {
         const IO *vp = reinterpret_cast<const IO *>(a.f.v) + plane * plane_elems;
+        const IO *kp = reinterpret_cast<const IO *>(a.f.k) + plane * plane_elems;
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) v[q] = load_pair<IO, true>(vp, pos_of(q), plane_elems);
+        for (int q = 0; q < E / 2; ++q) {
+            v[q] = load_pair<IO, true>(vp, pos_of(q), plane_elems);
+            if constexpr (GATED) {
+                const c32 kq = silu(load_pair<IO, true>(kp, pos_of(q), plane_elems));
+                v[q] = mk(v[q].x * kq.x, v[q].y * kq.y);
+            }
+        }
     } else {
         using P = typename io<IO>::pair_t;
         const IO *gp = reinterpret_cast<const IO *>(a.f.gates[a.n]) + plane * plane_elems;
@@ -93,7 +101,8 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dAr
         fft_cta<M1, E, +1, false, G::TWS, G::NCOL>(v, smem, nullptr, t1, tws, j);
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
-            const c32 gq = io<IO>::unpack(g[q]);
+            c32 gq = io<IO>::unpack(g[q]);
+            if constexpr (GATED) gq = silu(gq);
             v[q] = mk(gq.x * v[q].x, gq.y * v[q].y);
         }
         if constexpr (MODE == 2) {

@@ -24,6 +24,9 @@ Named workloads (sizes as stated; activations v, x^n and Dskip ~ N(0, 1)):
   bf16, kernels from the 2D sine network on (y, x) in [-1, 1)^2 (first-layer
   frequency 10, hidden 1, width 64, weights ~ N(0, 1/64)) times a Gaussian
   window with sigma = 0.5.
+* ``gated_order1_bf16_2d_b2_c256_256x256`` -- the same grid, channels and
+  kernels through the HyenaND gate sandwich: q (drawn as v), k and the outer
+  gate v (drawn as x^1) ~ N(0, 1).
 """
 from __future__ import annotations
 
@@ -51,6 +54,7 @@ class Workload:
     omega_hidden: float = 1.0
     sigma: float = 0.5        # 2D Gaussian window
     seed: int = 0
+    gated: bool = False       # the gate sandwich: an inner-gate key k is drawn too
 
     @property
     def L(self) -> int:
@@ -82,6 +86,8 @@ WORKLOADS = {
                  alpha_lo=1e-4, alpha_hi=1e-2, seed=4),
         Workload("order1_bf16_2d_b2_c256_256x256", 2, 2, 256, (256, 256), 1, "bf16", "implicit2d",
                  width=64, omega0=10.0, omega_hidden=1.0, sigma=0.5, seed=5),
+        Workload("gated_order1_bf16_2d_b2_c256_256x256", 2, 2, 256, (256, 256), 1, "bf16", "implicit2d",
+                 width=64, omega0=10.0, omega_hidden=1.0, sigma=0.5, seed=6, gated=True),
     ]
 }
 
@@ -113,6 +119,7 @@ def make_inputs(w: Workload, seed=None) -> dict:
       implicit: dict of float32 weights W1 b1 W2 b2 W3 b3 and the window
                parameter (alpha [N, D] in 1D, sigma [N, D] in 2D), plus the
                scalars width, num_freqs, omega0, omega_hidden (implicit only)
+      k      [B, D, *shape]      activation dtype (gate sandwich only; v is then q)
     """
     g = _gen(w.seed if seed is None else seed)
     N, B, D = w.order, w.B, w.D
@@ -156,4 +163,6 @@ def make_inputs(w: Workload, seed=None) -> dict:
         p.update(width=w.width, num_freqs=w.num_freqs if w.filt == "implicit1d" else 0,
                  omega0=w.omega0, omega_hidden=w.omega_hidden)
         out["implicit"] = p
+    if w.gated:   # drawn last, so that the other tensors follow the plain recipe
+        out["k"] = torch.randn((B, D) + w.shape, generator=g, dtype=torch.float64).to(adt)
     return out

@@ -128,3 +128,32 @@ def compare_2d(w: Workload, inp, k64, y_gpu, planes=None, context=""):
         worst = (np.abs(got - ref) / (MAXABS_FACTOR * np.maximum(bound, 1e-300))[:, None, None]).max()
         assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
     return err
+
+
+# ------------------------------------------------------------- gate sandwich --
+
+def compare_gated_2d(w: Workload, inp, k64, y_gpu, planes=None, context=""):
+    """The gate sandwich (q = inp["v"], key inp["k"], SiLU of every gate) against the fp64 oracle."""
+    N, B, C = w.order, w.B, w.D
+    H, W = w.shape
+    P = B * C
+    planes = np.arange(P) if planes is None else np.asarray(planes)
+    q = inp["v"].double().reshape(P, H, W).numpy()[planes]
+    kk = inp["k"].double().reshape(P, H, W).numpy()[planes]
+    gates = inp["gates"].double().reshape(N, P, H, W).numpy()[:, planes]
+    dsk = inp["dskip"].double().numpy()
+    ref = oracle.hyena_gated(q, kk, gates, k64, dsk, fidx=planes % C)
+    got = y_gpu.detach().double().cpu().reshape(P, H, W).numpy()[planes]
+    assert np.all(np.isfinite(got)), context + ": non-finite output"
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err <= REL_L2[w.dtype], "%s: relative L2 error %.3e > %.1e" % (context, err, REL_L2[w.dtype])
+    if w.dtype == "f32":
+        c = planes % C
+        z0 = q * oracle.silu(kk)
+        bound = np.abs(z0).reshape(len(planes), -1).max(axis=1)
+        for n in range(N):
+            bound = bound * (np.abs(k64[n, c]).reshape(len(planes), -1).sum(axis=1) + np.abs(dsk[n, c])) \
+                * np.abs(oracle.silu(gates[n])).reshape(len(planes), -1).max(axis=1)
+        worst = (np.abs(got - ref) / (MAXABS_FACTOR * np.maximum(bound, 1e-300))[:, None, None]).max()
+        assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
+    return err

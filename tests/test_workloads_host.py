@@ -14,7 +14,21 @@ STATED = {   # name: (ndim, B, D, shape, order, dtype, filter kind)
     "order2_bf16_b4_d1024_l8192_implicit": (1, 4, 1024, (8192,), 2, "bf16", "implicit1d"),
     "order3_bf16_b1_d768_l65536": (1, 1, 768, (65536,), 3, "bf16", "explicit"),
     "order1_bf16_2d_b2_c256_256x256": (2, 2, 256, (256, 256), 1, "bf16", "implicit2d"),
+    "gated_order1_bf16_2d_b2_c256_256x256": (2, 2, 256, (256, 256), 1, "bf16", "implicit2d"),
 }
+
+
+def test_gated_workload_draws_k_last():
+    """The gate sandwich's key k is drawn after every other tensor: the other tensors follow
+    the plain recipe for the same seed, and k is N(0, 1) in the activation dtype."""
+    import dataclasses
+    w = WORKLOADS["gated_order1_bf16_2d_b2_c256_256x256"].scaled(B=1, D=4, shape=(16, 16))
+    plain = dataclasses.replace(w, gated=False)
+    a, b = make_inputs(w), make_inputs(plain)
+    assert "k" in a and "k" not in b
+    assert torch.equal(a["v"], b["v"]) and torch.equal(a["gates"], b["gates"])
+    assert a["k"].dtype == torch.bfloat16 and a["k"].shape == a["v"].shape
+    assert abs(a["k"].double().mean()) < 0.2 and 0.8 < a["k"].double().std() < 1.2
 
 
 def test_named_workloads_have_the_stated_sizes():
