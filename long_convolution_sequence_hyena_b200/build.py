@@ -36,9 +36,25 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
+def _object_stale(obj: str, dep: str, src: str, flags_file: str, flags: str) -> bool:
+    """Whether an object must be rebuilt: missing, built with other flags, or older than its
+    source or any file its dependency list (nvcc -MD) names."""
+    if not (os.path.exists(obj) and os.path.exists(dep) and os.path.exists(flags_file)):
+        return True
+    with open(flags_file) as f:
+        if f.read() != flags:
+            return True
+    t = os.path.getmtime(obj)
+    with open(dep) as f:
+        text = f.read().replace("\\\n", " ")
+    deps = text.split(":", 1)[1].split() if ":" in text else [src]
+    return any(not os.path.exists(d) or os.path.getmtime(d) > t for d in deps + [src])
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile every csrc/*.cu (in parallel, one object each) and link one shared library.
-    Skipped when the library is newer than every source."""
+    """Compile csrc/*.cu (in parallel, one object each; only the objects whose source or
+    included headers changed) and link one shared library. Skipped when the library is
+    newer than every source."""
     if not force and not needs_build():
         return LIB
     nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
@@ -46,14 +62,26 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     os.makedirs(objdir, exist_ok=True)
     procs = []
     objs = []
+    flags = " ".join([*NVCC_FLAGS, *extra_flags])
     for src in _sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+        dep, flags_file = obj[:-2] + ".d", obj[:-2] + ".flags"
         objs.append(obj)
-        cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        if not force and not _object_stale(obj, dep, src, flags_file, flags):
+            continue
+        if os.path.exists(flags_file):
+            os.remove(flags_file)            # written back only once the object is built
+        cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-MD", "-MF", dep, "-c", "-o", obj, src]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        procs.append((src, subprocess.Popen(cmd)))
-    failed = [src for src, p in procs if p.wait() != 0]
+        procs.append((src, flags_file, subprocess.Popen(cmd)))
+    failed = []
+    for src, flags_file, p in procs:
+        if p.wait() != 0:
+            failed.append(src)
+        else:
+            with open(flags_file, "w") as f:
+                f.write(flags)
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))
     tmp = LIB + ".tmp%d" % os.getpid()
