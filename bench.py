@@ -8,7 +8,8 @@ the order-3 bf16 B=1 D=768 L=65536 case, the longest single-GPU configuration
 of the operator (padded transform M = 131072). The same line carries a
 ``workloads`` object with the other bench configurations (order-2 bf16 L=2048;
 order-2 bf16 L=8192 with implicit filters; the 2D order-1 256x256 grid, plain
-and through the HyenaND gate sandwich), each
+and through the HyenaND gate sandwich; the L=65536 case with channels-last
+[B, L, D] activations), each
 measured the same way: ms per step, throughput, roofline fraction, DRAM
 traffic record, e2e, and the step with filter generation where the filters
 are implicit. With N>1 (torchrun) every rank runs the
@@ -40,7 +41,8 @@ sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "order3_bf16_b1_d768_l65536"
 SIDE_WORKLOADS = ("order2_bf16_b8_d768_l2048", "order2_bf16_b4_d1024_l8192_implicit",
-                  "order1_bf16_2d_b2_c256_256x256", "gated_order1_bf16_2d_b2_c256_256x256")
+                  "order1_bf16_2d_b2_c256_256x256", "gated_order1_bf16_2d_b2_c256_256x256",
+                  "order3_bf16_b1_d768_l65536_bld")
 FP32_LANES_PER_SM = 128          # FP32 FMA lanes per SM (4 sub-partitions x 32)
 SM_MAX_MHZ_FALLBACK = 1965.0
 HBM_NOMINAL_GBS = 8000.0         # the operator's roofline convention (8 TB/s)
@@ -186,7 +188,7 @@ def run_ours(args, w, rank, world, dist):
     v = inp["v"].to(dev)
     gates = [g.to(dev) for g in inp["gates"]]
     dskip = inp["dskip"].to(dev)
-    plan = Plan(w.shape, w.D, w.order, adt)
+    plan = Plan(w.shape, w.D, w.order, adt, layout=w.layout)
     if "h" in inp:
         H = plan.filter_spectrum(h=inp["h"].to(dev))
     else:

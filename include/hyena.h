@@ -73,6 +73,14 @@ typedef enum {
                                     the row's transform in a device workspace */
 } hyena_path_t;
 
+/* Activation layout of a 1D plan (hyena_plan_set_layout). */
+typedef enum {
+    HYENA_LAYOUT_BDL = 0,        /* [B, D, L]: each channel row contiguous (the default) */
+    HYENA_LAYOUT_BLD = 1         /* [B, L, D]: channels-last, the layout u ∈ R^{B×L×D} of the
+                                    operator's statement ("Hyena, Long Convolution, and Linear
+                                    Attention", "FFTConv: the O(L log L) primitive") */
+} hyena_layout_t;
+
 /*
  * Parameters of the implicit filter network, all DEVICE pointers to fp32.
  *
@@ -113,6 +121,19 @@ typedef struct {
  */
 HYENA_API hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *shape, int64_t channels,
                                  int order, hyena_dtype_t io_dtype, int causal);
+
+/*
+ * Select the activation layout of v, the gates and y for every later forward
+ * call on a 1D plan (hyena_forward, hyena_forward_host, hyena_forward_no_alloc).
+ * With HYENA_LAYOUT_BLD the kernels read and write the [B, L, D] tensors in
+ * place (no transpose pass): channel d of batch element b is the strided row
+ * at b L D + d with stride D. Filters, spectra and Dskip keep their layouts.
+ * 2D plans accept only HYENA_LAYOUT_BDL ([B, C, H, W]); another value returns
+ * HYENA_ERR_UNSUPPORTED, an unknown one HYENA_ERR_INVALID_ARG. Call it before
+ * the plan's first forward; it must not run concurrently with other calls on
+ * the plan.
+ */
+HYENA_API hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout);
 
 /* Free the plan's device tables (synchronises the device). NULL is accepted. */
 HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);

@@ -45,9 +45,11 @@ def implicit_params(p: dict) -> capi.hyena_implicit_params_t:
 
 
 class Plan:
-    """A plan for one geometry: shape (L,) or (H, W), channels, order, io dtype."""
+    """A plan for one geometry: shape (L,) or (H, W), channels, order, io dtype, and the
+    activation layout of 1D plans: "bdl" ([B, D, L], the default) or "bld" ([B, L, D],
+    channels-last, read and written in place)."""
 
-    def __init__(self, shape, channels: int, order: int, dtype=torch.bfloat16):
+    def __init__(self, shape, channels: int, order: int, dtype=torch.bfloat16, layout: str = "bdl"):
         shape = tuple(int(s) for s in shape)
         self.ndim = len(shape)
         self.shape = shape
@@ -60,6 +62,13 @@ class Plan:
         self.handle = h
         st, self.fft_len, self.spectrum_elems, self.path = capi.hyena_plan_info(h)
         _check(st, "hyena_plan_info")
+        self.layout = layout
+        if layout != "bdl":
+            lay = {"bld": capi.HYENA_LAYOUT_BLD}.get(layout)
+            if lay is None:
+                self.close()
+                raise ValueError("layout must be 'bdl' or 'bld'")
+            _check(capi.hyena_plan_set_layout(h, lay), "hyena_plan_set_layout")
 
     def close(self):
         if getattr(self, "handle", None):

@@ -18,6 +18,7 @@ HYENA_F32, HYENA_BF16 = 0, 1
 (HYENA_OK, HYENA_ERR_INVALID_ARG, HYENA_ERR_UNSUPPORTED, HYENA_ERR_ALIGNMENT,
  HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA, HYENA_ERR_NOMEM) = range(7)
 HYENA_PATH_CTA, HYENA_PATH_CLUSTER, HYENA_PATH_2D, HYENA_PATH_STAGED = 0, 1, 2, 3
+HYENA_LAYOUT_BDL, HYENA_LAYOUT_BLD = 0, 1
 
 STATUS_NAMES = {
     HYENA_OK: "HYENA_OK", HYENA_ERR_INVALID_ARG: "HYENA_ERR_INVALID_ARG",
@@ -31,7 +32,7 @@ EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
-    "hyena_forward_gated",
+    "hyena_forward_gated", "hyena_plan_set_layout",
 )
 
 
@@ -65,6 +66,7 @@ def _load():
         "hyena_forward_host_workspace_bytes": ([p, i64], sz),
         "hyena_forward_host": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_forward_gated": ([p, i64, p, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
+        "hyena_plan_set_layout": ([p, i32], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -90,6 +92,10 @@ def hyena_plan_create(ndim: int, shape, channels: int, order: int, io_dtype: int
 
 def hyena_plan_destroy(plan) -> int:
     return lib.hyena_plan_destroy(plan)
+
+
+def hyena_plan_set_layout(plan, layout: int) -> int:
+    return lib.hyena_plan_set_layout(plan, layout)
 
 
 def hyena_plan_info(plan):

@@ -223,6 +223,13 @@ hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     return st;
 }
 
+hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout) {
+    if (!plan || (layout != HYENA_LAYOUT_BDL && layout != HYENA_LAYOUT_BLD)) return HYENA_ERR_INVALID_ARG;
+    if (plan->ndim != 1 && layout != HYENA_LAYOUT_BDL) return HYENA_ERR_UNSUPPORTED;
+    plan->layout = layout;
+    return HYENA_OK;
+}
+
 hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path) {
     if (!plan) return HYENA_ERR_INVALID_ARG;
     if (fft_len) *fft_len = plan->ndim == 1 ? plan->M : 4 * plan->Hh * plan->Ww;
@@ -366,6 +373,7 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
     a.D = plan->D;
     a.B = batch;
     a.order = plan->order;
+    a.es = plan->layout == HYENA_LAYOUT_BLD ? plan->D : 1;
     const bool even = (plan->L % 2) == 0;
     cudaError_t e;
     if (plan->path == HYENA_PATH_STAGED) {
@@ -375,7 +383,7 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
                                  (cudaStream_t)stream, cl.l);
     } else if (plan->path == HYENA_PATH_CLUSTER)
         e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
-    else if (pair_path_supported(plan->MC, batch))
+    else if (a.es == 1 && pair_path_supported(plan->MC, batch))
         e = launch_fwd_1d_pair(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     else
         e = launch_fwd_1d(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);

@@ -20,7 +20,18 @@ struct Fwd1dArgs {
     int64_t D;
     int64_t B;
     int order;
+    // activation layout: es = 1 for [B, D, L] (a channel row is contiguous);
+    // es = D for channels-last [B, L, D] (consecutive positions of a row are D
+    // elements apart, and channel d of batch element b starts at b L D + d)
+    int64_t es;
 };
+
+// Offset (elements) of flat row b * D + d in an activation tensor.
+__device__ __forceinline__ int64_t act_row_off(const Fwd1dArgs &a, int64_t row) {
+    if (a.es == 1) return row * a.L;
+    const int64_t b = row / a.D;
+    return b * a.L * a.D + (row - b * a.D);
+}
 
 constexpr int rows_per_cta(int MC, int E) { return (MC / E) >= 128 ? 1 : 128 / (MC / E); }
 
@@ -52,10 +63,12 @@ struct io<__nv_bfloat16> {
 };
 
 // SiLU(x) = x σ(x) = x / (1 + e^{-x}) for the gate sandwich of HyenaND
-// ("How HyenaND works", "Putting it together: the HyenaND operator"). For
-// x -> -inf, e^{-x} overflows to +inf and the quotient is -0; for x -> +inf it
-// is x.
-__device__ __forceinline__ float silu(float x) { return x / (1.f + expf(-x)); }
+// ("How HyenaND works", "Putting it together: the HyenaND operator"), with the
+// fast exponential and divide (a few ulp, far inside the fp32 tolerance). The
+// exponent is clamped at 80 so that the divisor stays below 2^126, where the
+// fast divide is defined; below x = -80 the result is x / (1 + e^80), whose
+// magnitude is under 1e-32 (the exact value is smaller still).
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(fminf(-x, 80.f))); }
 __device__ __forceinline__ c32 silu(c32 a) { return mk(silu(a.x), silu(a.y)); }
 
 // Load positions (pos, pos+1) of a row of length L, zero beyond L.
@@ -94,6 +107,28 @@ __device__ __forceinline__ void store_pair(IO *__restrict__ row, int64_t pos, in
         if (pos < L) row[pos] = io<IO>::from_f(val.x);
         if (pos + 1 < L) row[pos + 1] = io<IO>::from_f(val.y);
     }
+}
+
+// The same accesses for a row whose consecutive positions are es elements
+// apart (es = 1: the contiguous forms above; channels-last: one element each).
+template <typename IO, bool EVEN>
+__device__ __forceinline__ c32 load_pair_s(const IO *__restrict__ row, int64_t pos, int64_t L, int64_t es) {
+    if (es == 1) return load_pair<IO, EVEN>(row, pos, L);
+    const float x0 = pos < L ? io<IO>::to_f(row[pos * es]) : 0.f;
+    const float x1 = pos + 1 < L ? io<IO>::to_f(row[(pos + 1) * es]) : 0.f;
+    return mk(x0, x1);
+}
+template <typename IO, bool EVEN>
+__device__ __forceinline__ typename io<IO>::pair_t load_pair_raw_s(const IO *__restrict__ row, int64_t pos, int64_t L,
+                                                                    int64_t es) {
+    if (es == 1) return load_pair_raw<IO, EVEN>(row, pos, L);
+    return io<IO>::pack(load_pair_s<IO, EVEN>(row, pos, L, es));
+}
+template <typename IO, bool EVEN>
+__device__ __forceinline__ void store_pair_s(IO *__restrict__ row, int64_t pos, int64_t L, int64_t es, c32 val) {
+    if (es == 1) return store_pair<IO, EVEN>(row, pos, L, val);
+    if (pos < L) row[pos * es] = io<IO>::from_f(val.x);
+    if (pos + 1 < L) row[(pos + 1) * es] = io<IO>::from_f(val.y);
 }
 
 __device__ __forceinline__ c32 ldg_c(const c32 *p) {
@@ -230,20 +265,20 @@ __global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
 
     c32 v[E];
     {
-        const IO *vrow = reinterpret_cast<const IO *>(a.v) + row * L;
+        const IO *vrow = reinterpret_cast<const IO *>(a.v) + act_row_off(a, row);
 #pragma unroll
         for (int q = 0; q < E / 2; ++q)
-            v[q] = active ? load_pair<IO, EVEN>(vrow, 2 * (int64_t)(t + q * T), L) : mk(0.f, 0.f);
+            v[q] = active ? load_pair_s<IO, EVEN>(vrow, 2 * (int64_t)(t + q * T), L, a.es) : mk(0.f, 0.f);
 #pragma unroll
         for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
     for (int n = 0; n < a.order; ++n) {
-        const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + row * L;
+        const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + act_row_off(a, row);
         typename io<IO>::pair_t g[E / 2];
 #pragma unroll
         for (int q = 0; q < E / 2; ++q)
-            g[q] = active ? load_pair_raw<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L) : io<IO>::zero();
+            g[q] = active ? load_pair_raw_s<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L, a.es) : io<IO>::zero();
         const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
         const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
         if constexpr (HS) {  // stage the spectrum row while the forward FFT runs
@@ -267,9 +302,9 @@ __global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
     }
 
     if (active) {
-        IO *yrow = reinterpret_cast<IO *>(a.y) + row * L;
+        IO *yrow = reinterpret_cast<IO *>(a.y) + act_row_off(a, row);
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) store_pair<IO, EVEN>(yrow, 2 * (int64_t)(t + q * T), L, v[q]);
+        for (int q = 0; q < E / 2; ++q) store_pair_s<IO, EVEN>(yrow, 2 * (int64_t)(t + q * T), L, a.es, v[q]);
     }
 }
 

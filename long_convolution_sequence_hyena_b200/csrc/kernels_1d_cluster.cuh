@@ -246,20 +246,22 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(cons
 
     c32 v[E];
     {
-        const IO *vrow = reinterpret_cast<const IO *>(a.v) + row * L;
+        const IO *vrow = reinterpret_cast<const IO *>(a.v) + act_row_off(a, row);
 #pragma unroll
-        for (int q = 0; q < E / 2; ++q) v[q] = load_pair<IO, EVEN>(vrow, 2 * cx.col_index(q), L);
+        for (int q = 0; q < E / 2; ++q) v[q] = load_pair_s<IO, EVEN>(vrow, 2 * cx.col_index(q), L, a.es);
 #pragma unroll
         for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
     // this order's gates are staged in shared memory (thread-private slots)
-    // while the transforms run, instead of occupying registers
+    // while the transforms run, instead of occupying registers (contiguous rows
+    // of even length; otherwise they are read where they multiply)
     using P = typename io<IO>::pair_t;
     P *gst = reinterpret_cast<P *>(smem + 4 * G::PER_CTA) + threadIdx.x;
+    const bool stage = EVEN && a.es == 1;
     for (int n = 0; n < a.order; ++n) {
-        const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + row * L;
-        if constexpr (EVEN) {
+        const IO *grow = reinterpret_cast<const IO *>(a.gates[n]) + act_row_off(a, row);
+        if (stage) {
 #pragma unroll
             for (int q = 0; q < E / 2; ++q) {
                 const int64_t pos = 2 * cx.col_index(q);
@@ -328,20 +330,20 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(cons
         cx.inverse(v, a.tw);
 
         // gate (registers q >= E/2 hold positions >= MC, i.e. padding)
-        if constexpr (EVEN) cp_async_wait_all();
+        if (stage) cp_async_wait_all();
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
             const int64_t pos = 2 * cx.col_index(q);
-            const c32 gq = EVEN ? io<IO>::unpack(gst[q * G::THREADS]) : load_pair<IO, false>(grow, pos, L);
+            const c32 gq = stage ? io<IO>::unpack(gst[q * G::THREADS]) : load_pair_s<IO, false>(grow, pos, L, a.es);
             v[q] = mk(pos < L ? gq.x * v[q].x : 0.f, pos + 1 < L ? gq.y * v[q].y : 0.f);
         }
 #pragma unroll
         for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);
     }
 
-    IO *yrow = reinterpret_cast<IO *>(a.y) + row * L;
+    IO *yrow = reinterpret_cast<IO *>(a.y) + act_row_off(a, row);
 #pragma unroll
-    for (int q = 0; q < E / 2; ++q) store_pair<IO, EVEN>(yrow, 2 * cx.col_index(q), L, v[q]);
+    for (int q = 0; q < E / 2; ++q) store_pair_s<IO, EVEN>(yrow, 2 * cx.col_index(q), L, a.es, v[q]);
 }
 
 // Spectrum of long causal filters (same layout as hyena_spectrum_1d), one

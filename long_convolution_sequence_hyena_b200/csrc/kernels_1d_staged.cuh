@@ -118,23 +118,23 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
 
     c32x2 v[E];
     if constexpr (MODE == 0) {
-        const IO *r0 = reinterpret_cast<const IO *>(a.f.v) + row0 * L;
-        const IO *r1 = reinterpret_cast<const IO *>(a.f.v) + row1 * L;
+        const IO *r0 = reinterpret_cast<const IO *>(a.f.v) + act_row_off(a.f, row0);
+        const IO *r1 = reinterpret_cast<const IO *>(a.f.v) + act_row_off(a.f, row1);
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
-            const c32 x0 = load_pair<IO, EVEN>(r0, pos_of(q), L);
-            const c32 x1 = has1 ? load_pair<IO, EVEN>(r1, pos_of(q), L) : mk(0.f, 0.f);
+            const c32 x0 = load_pair_s<IO, EVEN>(r0, pos_of(q), L, a.f.es);
+            const c32 x1 = has1 ? load_pair_s<IO, EVEN>(r1, pos_of(q), L, a.f.es) : mk(0.f, 0.f);
             v[q] = c32x2{f2(x0.x, x1.x), f2(x0.y, x1.y)};
         }
     } else {
         using P = typename io<IO>::pair_t;
-        const IO *g0 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + row0 * L;
-        const IO *g1 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + row1 * L;
+        const IO *g0 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + act_row_off(a.f, row0);
+        const IO *g1 = reinterpret_cast<const IO *>(a.f.gates[a.n]) + act_row_off(a.f, row1);
         P ga[E / 2], gb[E / 2];   // this order's gates, loaded while the inverse transform runs
 #pragma unroll
         for (int q = 0; q < E / 2; ++q) {
-            ga[q] = load_pair_raw<IO, EVEN>(g0, pos_of(q), L);
-            gb[q] = load_pair_raw<IO, EVEN>(g1, pos_of(q), L);
+            ga[q] = load_pair_raw_s<IO, EVEN>(g0, pos_of(q), L, a.f.es);
+            gb[q] = load_pair_raw_s<IO, EVEN>(g1, pos_of(q), L, a.f.es);
         }
         // the last read of the chunk's workspace releases it (evict_first)
         const uint64_t pol = MODE == 2 ? l2_stream() : l2_keep();
@@ -153,12 +153,12 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
                          pos + 1 < L ? f2mul(v[q].im, f2(ca.y, cb.y)) : f2(0.f, 0.f)};
         }
         if constexpr (MODE == 2) {
-            IO *y0 = reinterpret_cast<IO *>(a.f.y) + row0 * L;
-            IO *y1 = reinterpret_cast<IO *>(a.f.y) + row1 * L;
+            IO *y0 = reinterpret_cast<IO *>(a.f.y) + act_row_off(a.f, row0);
+            IO *y1 = reinterpret_cast<IO *>(a.f.y) + act_row_off(a.f, row1);
 #pragma unroll
             for (int q = 0; q < E / 2; ++q) {
-                store_pair<IO, EVEN>(y0, pos_of(q), L, mk(v[q].re.x, v[q].im.x));
-                if (has1) store_pair<IO, EVEN>(y1, pos_of(q), L, mk(v[q].re.y, v[q].im.y));
+                store_pair_s<IO, EVEN>(y0, pos_of(q), L, a.f.es, mk(v[q].re.x, v[q].im.x));
+                if (has1) store_pair_s<IO, EVEN>(y1, pos_of(q), L, a.f.es, mk(v[q].re.y, v[q].im.y));
             }
             return;
         }

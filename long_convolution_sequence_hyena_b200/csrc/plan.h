@@ -17,6 +17,7 @@ struct hyena_plan_s {
     int order = 0;
     hyena_dtype_t dtype = HYENA_F32;
     int path = HYENA_PATH_CTA;
+    int layout = HYENA_LAYOUT_BDL;   // activation layout (hyena_plan_set_layout)
     int device = 0;
     // 1D geometry
     int64_t L = 0;               // sequence length

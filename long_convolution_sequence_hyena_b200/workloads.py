@@ -27,6 +27,8 @@ Named workloads (sizes as stated; activations v, x^n and Dskip ~ N(0, 1)):
 * ``gated_order1_bf16_2d_b2_c256_256x256`` -- the same grid, channels and
   kernels through the HyenaND gate sandwich: q (drawn as v), k and the outer
   gate v (drawn as x^1) ~ N(0, 1).
+* ``order3_bf16_b1_d768_l65536_bld`` -- the L=65536 order-3 recipe with
+  channels-last activations [B, L, D] (drawn as [B, D, L], then transposed).
 """
 from __future__ import annotations
 
@@ -55,6 +57,7 @@ class Workload:
     sigma: float = 0.5        # 2D Gaussian window
     seed: int = 0
     gated: bool = False       # the gate sandwich: an inner-gate key k is drawn too
+    layout: str = "bdl"       # 1D activations [B, D, L] ("bdl") or channels-last [B, L, D] ("bld")
 
     @property
     def L(self) -> int:
@@ -88,6 +91,8 @@ WORKLOADS = {
                  width=64, omega0=10.0, omega_hidden=1.0, sigma=0.5, seed=5),
         Workload("gated_order1_bf16_2d_b2_c256_256x256", 2, 2, 256, (256, 256), 1, "bf16", "implicit2d",
                  width=64, omega0=10.0, omega_hidden=1.0, sigma=0.5, seed=6, gated=True),
+        Workload("order3_bf16_b1_d768_l65536_bld", 1, 1, 768, (65536,), 3, "bf16", "explicit",
+                 alpha_lo=1e-4, alpha_hi=1e-2, seed=7, layout="bld"),
     ]
 }
 
@@ -120,6 +125,7 @@ def make_inputs(w: Workload, seed=None) -> dict:
                parameter (alpha [N, D] in 1D, sigma [N, D] in 2D), plus the
                scalars width, num_freqs, omega0, omega_hidden (implicit only)
       k      [B, D, *shape]      activation dtype (gate sandwich only; v is then q)
+    With layout "bld" v and the gates are [B, L, D] and [N, B, L, D].
     """
     g = _gen(w.seed if seed is None else seed)
     N, B, D = w.order, w.B, w.D
@@ -165,4 +171,7 @@ def make_inputs(w: Workload, seed=None) -> dict:
         out["implicit"] = p
     if w.gated:   # drawn last, so that the other tensors follow the plain recipe
         out["k"] = torch.randn((B, D) + w.shape, generator=g, dtype=torch.float64).to(adt)
+    if w.layout == "bld":   # channels-last copies of the same values
+        out["v"] = out["v"].transpose(-1, -2).contiguous()
+        out["gates"] = out["gates"].transpose(-1, -2).contiguous()
     return out

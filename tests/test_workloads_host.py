@@ -15,7 +15,17 @@ STATED = {   # name: (ndim, B, D, shape, order, dtype, filter kind)
     "order3_bf16_b1_d768_l65536": (1, 1, 768, (65536,), 3, "bf16", "explicit"),
     "order1_bf16_2d_b2_c256_256x256": (2, 2, 256, (256, 256), 1, "bf16", "implicit2d"),
     "gated_order1_bf16_2d_b2_c256_256x256": (2, 2, 256, (256, 256), 1, "bf16", "implicit2d"),
+    "order3_bf16_b1_d768_l65536_bld": (1, 1, 768, (65536,), 3, "bf16", "explicit"),
 }
+
+
+def test_bld_workload_is_the_transposed_recipe():
+    import dataclasses
+    w = WORKLOADS["order3_bf16_b1_d768_l65536_bld"].scaled(B=2, D=3, shape=(64,))
+    a, b = make_inputs(w), make_inputs(dataclasses.replace(w, layout="bdl"))
+    assert a["v"].shape == (2, 64, 3) and a["gates"].shape == (3, 2, 64, 3)
+    assert torch.equal(a["v"], b["v"].transpose(1, 2)) and torch.equal(a["gates"], b["gates"].transpose(2, 3))
+    assert torch.equal(a["h"], b["h"])
 
 
 def test_gated_workload_draws_k_last():
@@ -50,7 +60,8 @@ def test_draws_are_reproducible_and_typed(name):
     assert torch.equal(a["v"], b["v"]) and not torch.equal(a["v"], c["v"])
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     assert a["v"].dtype == dt and a["gates"].dtype == dt and a["dskip"].dtype == torch.float32
-    assert a["gates"].shape == (w.order, 1, 8) + small.shape
+    expect = (w.order, 1, 8) + small.shape if w.layout == "bdl" else (w.order, 1) + small.shape + (8,)
+    assert a["gates"].shape == expect
 
 
 def test_activations_are_standard_normal():
