@@ -15,6 +15,8 @@ cudaError_t launch_fwd_1d_cluster_g(const Fwd1dArgs &a, hyena_dtype_t dt, bool e
                 : launch_cluster<G>(hyena_fwd_1d_cluster<G, __nv_bfloat16, false>, a.rows, st, a);
 }
 
+bool cluster_path_supported(int64_t MC) { return MC == 131072; }
+
 cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st) {
     switch (MC) {
         case 131072: return launch_fwd_1d_cluster_g<G1_128K>(a, dt, even, st);

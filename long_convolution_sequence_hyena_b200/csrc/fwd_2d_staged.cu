@@ -107,16 +107,7 @@ cudaError_t launch_fwd_2d_staged(const Fwd2dArgs &f, int64_t W, float2 *ws, hyen
                                : launch_staged2d_io<GS2_256, __nv_bfloat16, false>(f, ws, chunk, lanes, nst);
     };
     if (f.planes <= chunk) return run(&st, 1);
-    cudaError_t e = cudaEventRecord(sl.fork, st);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
-    if (e != cudaSuccess) return e;
-    const cudaError_t le = run(sl.lane, 2);
-    for (int i = 0; i < 2; ++i) {
-        e = cudaEventRecord(sl.join[i], sl.lane[i]);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sl.join[i], 0);
-        if (e != cudaSuccess) return e;
-    }
-    return le;
+    return run_on_lanes(st, sl, 2, run);
 }
 
 }  // namespace hyena

@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -41,7 +42,7 @@ std::vector<float2> twiddle_table(int64_t M) {
 bool release_lanes(hyena_plan_s *p) {
     if (!p->has_lanes) return true;
     bool ok = true;
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < HYENA_STAGED_LANES; ++i) {
         if (p->lane[i] && cudaStreamDestroy(p->lane[i]) != cudaSuccess) ok = false;
         p->lane[i] = nullptr;
     }
@@ -57,17 +58,19 @@ struct CallLanes {
     StagedLanes l;
     bool ok = false;
     explicit CallLanes(const hyena_plan_s *p) {
-        l.lane[0] = p->lane[0];
-        l.lane[1] = p->lane[1];
-        l.fork = l.join[0] = l.join[1] = nullptr;
-        ok = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&l.join[0], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&l.join[1], cudaEventDisableTiming) == cudaSuccess;
+        l.fork = nullptr;
+        for (int i = 0; i < HYENA_STAGED_LANES; ++i) {
+            l.lane[i] = p->lane[i];
+            l.join[i] = nullptr;
+        }
+        ok = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; i < HYENA_STAGED_LANES && ok; ++i)
+            ok = cudaEventCreateWithFlags(&l.join[i], cudaEventDisableTiming) == cudaSuccess;
         if (!ok) cudaGetLastError();
     }
     ~CallLanes() {
         if (l.fork) cudaEventDestroy(l.fork);
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < HYENA_STAGED_LANES; ++i)
             if (l.join[i]) cudaEventDestroy(l.join[i]);
     }
     CallLanes(const CallLanes &) = delete;
@@ -146,6 +149,23 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         p.MC = p.M / 2;
         p.path = p.M <= HYENA_MAX_M_CTA ? HYENA_PATH_CTA
                  : (staged_path_supported(p.MC) ? HYENA_PATH_STAGED : HYENA_PATH_CLUSTER);
+        // test and measurement override: HYENA_FORCE_PATH=cta|staged|cluster picks a
+        // kernel family that can run this length, or the plan is UNSUPPORTED
+        if (const char *fp = std::getenv("HYENA_FORCE_PATH")) {
+            if (!std::strcmp(fp, "cta")) {
+                if (p.M > HYENA_MAX_M_CTA) return HYENA_ERR_UNSUPPORTED;
+                p.path = HYENA_PATH_CTA;
+            } else if (!std::strcmp(fp, "staged")) {
+                if (!staged_path_supported(p.MC)) return HYENA_ERR_UNSUPPORTED;
+                p.path = HYENA_PATH_STAGED;
+            } else if (!std::strcmp(fp, "cluster")) {
+                if (!cluster_path_supported(p.MC)) return HYENA_ERR_UNSUPPORTED;
+                p.path = HYENA_PATH_CLUSTER;
+            } else if (*fp) {
+                return HYENA_ERR_INVALID_ARG;
+            }
+        }
+        if (p.path == HYENA_PATH_CLUSTER && !cluster_path_supported(p.MC)) return HYENA_ERR_UNSUPPORTED;
         p.spectrum_elems = p.MC + 1;
         p.tw_len = p.M;
     } else {
@@ -174,8 +194,9 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         return HYENA_ERR_CUDA;
     }
     if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
-        bool ok = cudaStreamCreateWithFlags(&p.lane[0], cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&p.lane[1], cudaStreamNonBlocking) == cudaSuccess;
+        bool ok = true;
+        for (int i = 0; i < HYENA_STAGED_LANES && ok; ++i)
+            ok = cudaStreamCreateWithFlags(&p.lane[i], cudaStreamNonBlocking) == cudaSuccess;
         p.has_lanes = true;
         if (!ok) {
             release_lanes(&p);

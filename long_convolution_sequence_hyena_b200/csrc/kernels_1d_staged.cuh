@@ -37,6 +37,10 @@ struct StagedGeom {
     static constexpr int TWS = 1024;                 // sub-transform twiddle table W_1024
     static constexpr size_t CSMEM = (size_t)NCOL * M1 * 8 * ROWS;
     static constexpr size_t RSMEM = (size_t)NROW * M2 * 8 * ROWS;
+    // resident CTAs per SM the register budget is sized for (128-thread CTAs: 3
+    // column / 4 row CTAs; larger CTAs: 128 registers per thread)
+    static constexpr int CMINB = CT <= 128 ? 3 : 512 / CT;
+    static constexpr int RMINB = RT <= 128 ? 4 : 512 / RT;
     static_assert(M2 % NCOL == 0 && M1 % NROW == 0 && NROW % 2 == 0, "groups must tile the row");
     static_assert((ROWS == 1 && NCOL >= 16 && NROW >= 16) || (ROWS == 2 && NCOL >= 8 && NROW >= 8),
                   "warps must span enough sequences for conflict-free exchanges");
@@ -98,7 +102,7 @@ __device__ __forceinline__ int64_t visit_row(const Fwd1dArgs &f, int64_t o, int6
 // gate x^n, forward columns); 2: last (inverse columns, gate x^n, store y).
 
 template <typename G, typename IO, bool EVEN, int MODE>
-__global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArgs a, int64_t nr) {
+__global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_cols_x2(const StagedArgs a, int64_t nr) {
     static_assert(G::ROWS == 2, "lockstep geometry");
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T1 = G::T1, MC = G::MC, M = 2 * MC;
     extern __shared__ float smem[];
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_cols_x2(const StagedArg
 }
 
 template <typename G>
-__global__ void __launch_bounds__(G::RT, 4) hyena_staged_rows_x2(const StagedArgs a, int64_t nr) {
+__global__ void __launch_bounds__(G::RT, G::RMINB) hyena_staged_rows_x2(const StagedArgs a, int64_t nr) {
     static_assert(G::ROWS == 2, "lockstep geometry");
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, MC = G::MC, M = 2 * MC;
     constexpr int NROW = G::NROW, HROW = G::HROW, RT = G::RT;
@@ -326,7 +330,7 @@ struct Spec1dArgs {
 };
 
 template <typename G>
-__global__ void __launch_bounds__(G::CT, 3) hyena_staged_spec_cols_x2(const Spec1dArgs a) {
+__global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_spec_cols_x2(const Spec1dArgs a) {
     static_assert(G::ROWS == 2, "lockstep geometry");
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T1 = G::T1, MC = G::MC, M = 2 * MC;
     extern __shared__ float smem[];
@@ -364,7 +368,7 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged_spec_cols_x2(const Spec
 }
 
 template <typename G>
-__global__ void __launch_bounds__(G::RT, 4) hyena_staged_spec_rows_x2(const Spec1dArgs a) {
+__global__ void __launch_bounds__(G::RT, G::RMINB) hyena_staged_spec_rows_x2(const Spec1dArgs a) {
     static_assert(G::ROWS == 2, "lockstep geometry");
     constexpr int E = G::E, M1 = G::M1, M2 = G::M2, T2 = G::T2, MC = G::MC, M = 2 * MC;
     constexpr int NROW = G::NROW, HROW = G::HROW, RT = G::RT;

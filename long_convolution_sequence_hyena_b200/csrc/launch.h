@@ -17,16 +17,42 @@ cudaError_t launch_spec_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hou
 bool pair_path_supported(int64_t MC, int64_t B);
 cudaError_t launch_fwd_1d_pair(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
 // 1D, one cluster per row (MC = 131072)
+bool cluster_path_supported(int64_t MC);
 cudaError_t launch_fwd_1d_cluster(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
 cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
                                    const c32 *tw, cudaStream_t st);
 // 1D, staged four-step through a workspace (MC in {32768, 65536}); chunks of
 // staged_chunk_rows(MC) rows, two in flight on the plan's lanes; workspace
 // staged_workspace_rows(MC, rows) * MC complex64
+// Lanes (plan-owned streams) of the staged paths: a staged 1D forward keeps
+// HYENA_STAGED_LANES chunks of HYENA_STAGED_CHUNK_MB of transforms in flight,
+// one per lane; spectra and the 2D path use the first two.
+#ifndef HYENA_STAGED_LANES
+#define HYENA_STAGED_LANES 2
+#endif
+#ifndef HYENA_STAGED_CHUNK_MB
+#define HYENA_STAGED_CHUNK_MB 32
+#endif
+static_assert(HYENA_STAGED_LANES >= 2 && HYENA_STAGED_LANES <= 8, "lane count");
 struct StagedLanes {
-    cudaStream_t lane[2];     // non-blocking streams owned by the plan
-    cudaEvent_t fork, join[2];   // events of the calling operation only
+    cudaStream_t lane[HYENA_STAGED_LANES];     // non-blocking streams owned by the plan
+    cudaEvent_t fork, join[HYENA_STAGED_LANES];   // events of the calling operation only
 };
+// Fork n lanes off `st`, run(lanes, n), join them back into `st` (also after a
+// failed launch, so that `st` never runs ahead of the lanes).
+template <typename F>
+cudaError_t run_on_lanes(cudaStream_t st, const StagedLanes &sl, int n, F &&run) {
+    cudaError_t e = cudaEventRecord(sl.fork, st);
+    for (int i = 0; i < n && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(sl.lane[i], sl.fork, 0);
+    if (e != cudaSuccess) return e;
+    const cudaError_t le = run(sl.lane, n);
+    for (int i = 0; i < n; ++i) {
+        e = cudaEventRecord(sl.join[i], sl.lane[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, sl.join[i], 0);
+        if (e != cudaSuccess) return e;
+    }
+    return le;
+}
 bool staged_path_supported(int64_t MC);
 int64_t staged_chunk_rows(int64_t MC);
 int64_t staged_workspace_rows(int64_t MC, int64_t rows);

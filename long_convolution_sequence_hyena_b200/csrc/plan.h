@@ -7,7 +7,7 @@
 
 #include "hyena.h"
 
-#define HYENA_MAX_L_1D 131072    // longest 1D sequence (M = 262144)
+#define HYENA_MAX_L_1D 524288    // longest 1D sequence (M = 1048576)
 #define HYENA_MAX_M_CTA 32768    // longest padded length the single-CTA path runs
 #define HYENA_SUB_TWIDDLES 1024  // W_1024 table appended to the main one (cluster sub-transforms)
 
@@ -32,7 +32,7 @@ struct hyena_plan_s {
     // staged paths: two non-blocking streams; each call forks them off its
     // stream and joins them back with events of its own
     bool has_lanes = false;
-    cudaStream_t lane[2] = {nullptr, nullptr};
+    cudaStream_t lane[8] = {};   // the first HYENA_STAGED_LANES are created
     // staged spectra (1D long rows, 2D 256x256): scratch for two chunks of
     // transforms (owned). Chunk slot i is only ever used by lane i, and the
     // mutex keeps each call's launch sequence together on the lanes, so calls

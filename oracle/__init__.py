@@ -8,6 +8,8 @@ Contents
 --------
 * ``hyena_1d``  -- the order-N causal chain, direct O(L^2) sum, in C
   (``hyena_oracle.c``); see that file for the definition and its citations.
+* ``hyena_1d_order1_at`` -- single order-1 outputs by their own direct sums,
+  for rows too long for the full chain.
 * ``hyena_2d``  -- the 2D gated global (non-causal, linear) convolution chain,
   direct O((HW)^2) sum, in C.
 * ``implicit_filter_1d`` / ``implicit_filter_2d`` -- the implicit filters in
@@ -96,6 +98,25 @@ def hyena_1d(v, gates, h, dskip=None, fidx=None, threads: int = 0):
     if rc != 0:
         raise RuntimeError("hyena_oracle_1d failed (%d)" % rc)
     return y
+
+
+def hyena_1d_order1_at(v, x, h, dskip=None, positions=()):
+    """Order-1 outputs at selected positions only, each by its own direct sum
+    (the causal sum of "Hyena — Long Convolutions Math", "The primitive", with
+    the feedthrough of "FFTConv"):  y[t] = x[t] (sum_{tau <= t} h[t - tau] v[tau] + dskip v[t]).
+
+    v, x, h  [L] one row, its gate and its filter;  dskip  scalar or None.
+    Returns fp64 [len(positions)]. O(t) per position, for rows too long for
+    the full O(L^2) chain.
+    """
+    v, x, h = _f64(v), _f64(x), _f64(h)
+    d = 0.0 if dskip is None else float(dskip)
+    out = np.empty(len(positions), dtype=np.float64)
+    for i, t in enumerate(positions):
+        t = int(t)
+        c = float(np.dot(h[t::-1], v[:t + 1]))        # h[t - tau] v[tau], tau = 0..t
+        out[i] = x[t] * (c + d * v[t])
+    return out
 
 
 def hyena_2d(v, gates, k, dskip=None, fidx=None, threads: int = 0):

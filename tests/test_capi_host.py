@@ -49,7 +49,7 @@ def test_status_strings(capi):
     ((3, [4, 4, 4], 4, 1, 1, 0), "HYENA_ERR_INVALID_ARG"),    # 3D
     ((1, [256], 4, 2, 1, 0), "HYENA_ERR_UNSUPPORTED"),        # non-causal 1D
     ((2, [64, 64], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # causal 2D
-    ((1, [262145], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # longer than the longest path
+    ((1, [524289], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # longer than the longest path (M = 2^20)
 ])
 def test_plan_create_rejects(capi, args, expect):
     st, h = capi.hyena_plan_create(*args)

@@ -487,3 +487,18 @@ def test_gated_saturated_gates_reduce_to_the_plain_operator():
     # and k -> -inf closes the inner gate: the output is zero
     y0 = oracle.hyena_gated(q, np.full((R, L), -800.0), rng.standard_normal((1, R, L)), h)
     assert np.all(y0 == 0.0)
+
+
+def test_order1_outputs_at_positions_match_the_chain_and_the_worked_example():
+    """Single outputs by their own direct sums equal the full order-1 chain, and reproduce the
+    worked example of 'Linear vs circular' (h = [1, .5, .25, .125], x = [1, 2, 0, 0])."""
+    rng = np.random.default_rng(51)
+    L = 300
+    v, x, h = rng.standard_normal((3, L))
+    d = 0.7
+    full = oracle.hyena_1d(v[None], x[None, None], h[None, None], np.array([[d]]))[0]
+    pos = [0, 1, 2, 150, 298, 299]
+    np.testing.assert_allclose(oracle.hyena_1d_order1_at(v, x, h, d, pos), full[pos], rtol=1e-12, atol=1e-12)
+    g = _read_golden("worked_example_causal_conv.txt")
+    y = oracle.hyena_1d_order1_at(g["x"], np.ones(4), g["h"], None, range(4))
+    np.testing.assert_array_equal(y, g["y_linear_causal"])
