@@ -8,6 +8,7 @@ Contents
 --------
 * ``hyena_1d``  -- the order-N causal chain, direct O(L^2) sum, in C
   (``hyena_oracle.c``); see that file for the definition and its citations.
+* ``hyena_3d``  -- the same chain on a 3D grid (volumes), direct sum, in C.
 * ``hyena_1d_order1_at`` -- single order-1 outputs by their own direct sums,
   for rows too long for the full chain.
 * ``hyena_2d``  -- the 2D gated global (non-causal, linear) convolution chain,
@@ -56,6 +57,8 @@ def _load():
         lib.hyena_oracle_1d.restype = ctypes.c_int
         lib.hyena_oracle_2d.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p, p, ctypes.c_int]
         lib.hyena_oracle_2d.restype = ctypes.c_int
+        lib.hyena_oracle_3d.argtypes = [i64, i64, i64, i64, i64, i64, p, p, p, p, p, p, ctypes.c_int]
+        lib.hyena_oracle_3d.restype = ctypes.c_int
         lib.hyena_oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -143,4 +146,32 @@ def hyena_2d(v, gates, k, dskip=None, fidx=None, threads: int = 0):
     rc = _load().hyena_oracle_2d(P, H, W, N, F, _ptr(v), _ptr(gates), _ptr(k), _ptr(dskip), _ptr(fidx), _ptr(y), threads)
     if rc != 0:
         raise RuntimeError("hyena_oracle_2d failed (%d)" % rc)
+    return y
+
+
+def hyena_3d(v, gates, k, dskip=None, fidx=None, threads: int = 0):
+    """3D gated global-convolution chain over P independent volumes.
+
+    v      [P, Dz, H, W]
+    gates  [N, P, Dz, H, W]
+    k      [N, F, 2Dz, 2H, 2W]  kernels on the offset grid: element (oz, oy, ox),
+                                oz in [-Dz, Dz) etc., at [oz + Dz, oy + H, ox + W]
+    dskip  [N, F] or None
+    fidx   [P] (default: volume p uses p % F)
+    Returns y [P, Dz, H, W] float64.
+    """
+    v, gates, k = _f64(v), _f64(gates), _f64(k)
+    P, Dz, H, W = v.shape
+    N, F, D2, H2, W2 = k.shape
+    if gates.shape != (N, P, Dz, H, W) or (D2, H2, W2) != (2 * Dz, 2 * H, 2 * W):
+        raise ValueError("shape mismatch: v %s gates %s k %s" % (v.shape, gates.shape, k.shape))
+    dskip = None if dskip is None else _f64(dskip)
+    if dskip is not None and dskip.shape != (N, F):
+        raise ValueError("dskip must be [N, F]")
+    fidx = np.arange(P, dtype=np.int64) % F if fidx is None else np.ascontiguousarray(fidx, dtype=np.int64)
+    y = np.zeros((P, Dz, H, W), dtype=np.float64)
+    rc = _load().hyena_oracle_3d(P, Dz, H, W, N, F, _ptr(v), _ptr(gates), _ptr(k), _ptr(dskip), _ptr(fidx),
+                                 _ptr(y), threads)
+    if rc != 0:
+        raise RuntimeError("hyena_oracle_3d failed (%d)" % rc)
     return y

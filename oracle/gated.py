@@ -44,4 +44,7 @@ def hyena_gated(q, k, gates, filters, dskip=None, fidx=None, threads: int = 0):
         return hyena_1d(z0, g, filters, dskip, fidx=fidx, threads=threads)
     if q.ndim == 3:
         return hyena_2d(z0, g, filters, dskip, fidx=fidx, threads=threads)
-    raise ValueError("q must be [R, L] or [P, H, W]")
+    if q.ndim == 4:
+        from . import hyena_3d
+        return hyena_3d(z0, g, filters, dskip, fidx=fidx, threads=threads)
+    raise ValueError("q must be [R, L], [P, H, W] or [P, Dz, H, W]")

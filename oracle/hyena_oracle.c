@@ -197,3 +197,93 @@ int hyena_oracle_2d(int64_t P, int64_t H, int64_t W, int64_t N, int64_t F,
     free(jobs);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ 3D
+ * The same gated global convolution on a 3D grid ("How HyenaND works", "2. The
+ * convolution theorem (FFT)": in N dimensions the convolution runs on the
+ * native grid, a 3D volume included). Kernel (n, f) lives on offsets
+ * oz in [-Dz, Dz), oy in [-H, H), ox in [-W, W), stored [2Dz, 2H, 2W] with
+ * offset (oz, oy, ox) at [oz + Dz, oy + H, ox + W]; the output at voxel
+ * (iz, iy, ix) sums K(iz - sz, iy - sy, ix - sx) z(sz, sy, sx) over the grid.
+ */
+typedef struct {
+    int64_t p_begin, p_end;
+    int64_t Dz, H, W, N, F, P;
+    const double *v, *x, *k, *dskip;
+    const int64_t *fidx;
+    double *y;
+} job3d_t;
+
+static void hyena_plane_3d(const job3d_t *j, int64_t p, double *z, double *znew) {
+    const int64_t Dz = j->Dz, H = j->H, W = j->W, V = Dz * H * W;
+    const int64_t f = j->fidx[p];
+    for (int64_t i = 0; i < V; ++i) z[i] = j->v[p * V + i];
+    for (int64_t n = 0; n < j->N; ++n) {
+        const double *K = j->k + (n * j->F + f) * (8 * V);   /* [2Dz, 2H, 2W] offset grid */
+        const double *xg = j->x + (n * j->P + p) * V;
+        const double d = j->dskip ? j->dskip[n * j->F + f] : 0.0;
+        for (int64_t iz = 0; iz < Dz; ++iz)
+            for (int64_t iy = 0; iy < H; ++iy)
+                for (int64_t ix = 0; ix < W; ++ix) {
+                    double c = 0.0;
+                    for (int64_t sz = 0; sz < Dz; ++sz)
+                        for (int64_t sy = 0; sy < H; ++sy)
+                            for (int64_t sx = 0; sx < W; ++sx) {
+                                const int64_t oz = iz - sz, oy = iy - sy, ox = ix - sx;
+                                c += K[((oz + Dz) * (2 * H) + (oy + H)) * (2 * W) + (ox + W)] *
+                                     z[(sz * H + sy) * W + sx];
+                            }
+                    const int64_t o = (iz * H + iy) * W + ix;
+                    znew[o] = xg[o] * (c + d * z[o]);
+                }
+        for (int64_t i = 0; i < V; ++i) z[i] = znew[i];
+    }
+    for (int64_t i = 0; i < V; ++i) j->y[p * V + i] = z[i];
+}
+
+static void *worker_3d(void *arg) {
+    const job3d_t *j = (const job3d_t *)arg;
+    const int64_t V = j->Dz * j->H * j->W;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(2 * V));
+    if (!z) return (void *)1;
+    for (int64_t p = j->p_begin; p < j->p_end; ++p) hyena_plane_3d(j, p, z, z + V);
+    free(z);
+    return NULL;
+}
+
+/*
+ * P volumes of Dz x H x W, order N.
+ *   v      [P, Dz, H, W]
+ *   x      [N, P, Dz, H, W]
+ *   k      [N, F, 2Dz, 2H, 2W]   kernels on the offset grid
+ *   dskip  [N, F] or NULL
+ *   fidx   [P]
+ *   y      [P, Dz, H, W]
+ */
+int hyena_oracle_3d(int64_t P, int64_t Dz, int64_t H, int64_t W, int64_t N, int64_t F,
+                    const double *v, const double *x, const double *k,
+                    const double *dskip, const int64_t *fidx, double *y, int threads) {
+    if (P < 0 || Dz < 0 || H < 0 || W < 0 || N < 1 || F < 1 || !v || !x || !k || !fidx || !y) return -1;
+    for (int64_t p = 0; p < P; ++p)
+        if (fidx[p] < 0 || fidx[p] >= F) return -1;
+    if (P == 0 || Dz == 0 || H == 0 || W == 0) return 0;
+    if (threads <= 0) threads = hyena_oracle_num_threads();
+    if (threads > P) threads = (int)P;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)threads);
+    job3d_t *jobs = (job3d_t *)malloc(sizeof(job3d_t) * (size_t)threads);
+    if (!tid || !jobs) { free(tid); free(jobs); return -1; }
+    int rc = 0;
+    for (int i = 0; i < threads; ++i) {
+        job3d_t j = {P * i / threads, P * (i + 1) / threads, Dz, H, W, N, F, P, v, x, k, dskip, fidx, y};
+        jobs[i] = j;
+        if (pthread_create(&tid[i], NULL, worker_3d, &jobs[i]) != 0) { threads = i; rc = -1; break; }
+    }
+    for (int i = 0; i < threads; ++i) {
+        void *ret = NULL;
+        pthread_join(tid[i], &ret);
+        if (ret) rc = -1;
+    }
+    free(tid);
+    free(jobs);
+    return rc;
+}

@@ -502,3 +502,61 @@ def test_order1_outputs_at_positions_match_the_chain_and_the_worked_example():
     g = _read_golden("worked_example_causal_conv.txt")
     y = oracle.hyena_1d_order1_at(g["x"], np.ones(4), g["h"], None, range(4))
     np.testing.assert_array_equal(y, g["y_linear_causal"])
+
+
+# ----------------------------------------------------------------- 3D chain --
+# "How HyenaND works", "2. The convolution theorem (FFT)": the convolution on
+# the native grid of a 3D volume.
+
+def test_3d_delta_kernel_is_identity():
+    rng = np.random.default_rng(61)
+    P, Dz, H, W = 2, 3, 4, 5
+    v = rng.standard_normal((P, Dz, H, W))
+    k = np.zeros((1, P, 2 * Dz, 2 * H, 2 * W)); k[0, :, Dz, H, W] = 1.0
+    np.testing.assert_array_equal(oracle.hyena_3d(v, _ones((1, P, Dz, H, W)), k), v)
+
+
+def test_3d_separable_kernel_is_three_1d_convolutions():
+    """k = a(oz) b(oy) c(ox): non-causal 1D convolutions along each axis (numpy.convolve)."""
+    rng = np.random.default_rng(62)
+    Dz, H, W = 4, 3, 5
+    v = rng.standard_normal((1, Dz, H, W))
+    a, b, c = rng.standard_normal(2 * Dz), rng.standard_normal(2 * H), rng.standard_normal(2 * W)
+    k = np.einsum("i,j,l->ijl", a, b, c)[None, None]
+    y = oracle.hyena_3d(v, _ones((1, 1, Dz, H, W)), k)
+    t = np.apply_along_axis(lambda r: np.convolve(r, c)[W:2 * W], 2, v[0])
+    t = np.apply_along_axis(lambda r: np.convolve(r, b)[H:2 * H], 1, t)
+    t = np.apply_along_axis(lambda r: np.convolve(r, a)[Dz:2 * Dz], 0, t)
+    np.testing.assert_allclose(y[0], t, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_3d_scipy_convolve_cross_check(N):
+    """Library routine: scipy.signal.convolve (N-D, direct, full) cropped at the zero offset, gated, chained."""
+    rng = np.random.default_rng(63 + N)
+    P, Dz, H, W = 2, 3, 4, 3
+    v = rng.standard_normal((P, Dz, H, W))
+    gates = rng.standard_normal((N, P, Dz, H, W))
+    k = rng.standard_normal((N, P, 2 * Dz, 2 * H, 2 * W))
+    dskip = rng.standard_normal((N, P))
+    y = oracle.hyena_3d(v, gates, k, dskip)
+    for p in range(P):
+        z = v[p]
+        for n in range(N):
+            full = scipy.signal.convolve(z, k[n, p], method="direct")
+            c = full[Dz:2 * Dz, H:2 * H, W:2 * W]
+            z = gates[n, p] * (c + dskip[n, p] * z)
+        np.testing.assert_allclose(y[p], z, rtol=1e-11, atol=1e-11)
+
+
+def test_3d_single_slice_reduces_to_2d():
+    """Dz = 1: only offset oz = 0 touches the output, and the chain is the 2D one on that slice."""
+    rng = np.random.default_rng(65)
+    P, H, W = 3, 5, 4
+    v = rng.standard_normal((P, 1, H, W))
+    gates = rng.standard_normal((2, P, 1, H, W))
+    k = rng.standard_normal((2, P, 2, 2 * H, 2 * W))
+    dskip = rng.standard_normal((2, P))
+    y3 = oracle.hyena_3d(v, gates, k, dskip)
+    y2 = oracle.hyena_2d(v[:, 0], gates[:, :, 0], k[:, :, 1], dskip)
+    np.testing.assert_allclose(y3[:, 0], y2, rtol=1e-13, atol=1e-13)
