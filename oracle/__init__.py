@@ -30,7 +30,7 @@ import subprocess
 import numpy as np
 
 from .gated import hyena_gated, silu  # noqa: F401
-from .implicit import implicit_filter_1d, implicit_filter_2d, positional_features_1d  # noqa: F401
+from .implicit import implicit_filter_1d, implicit_filter_2d, implicit_filter_3d, positional_features_1d  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hyena_oracle.c")
@@ -175,3 +175,22 @@ def hyena_3d(v, gates, k, dskip=None, fidx=None, threads: int = 0):
     if rc != 0:
         raise RuntimeError("hyena_oracle_3d failed (%d)" % rc)
     return y
+
+
+def hyena_3d_order1_at(v, x, k, dskip=None, voxels=()):
+    """Order-1 outputs of one volume at selected voxels only, each by its own direct sum:
+    y[i] = x[i] (sum_s K[i - s] v[s] + dskip v[i]), the kernel on the offset grid
+    [2Dz, 2H, 2W] (offset o at [o + extent]). O(Dz H W) per voxel.
+
+    v, x  [Dz, H, W];  k  [2Dz, 2H, 2W];  voxels: iterable of (iz, iy, ix).
+    """
+    v, x, k = _f64(v), _f64(x), _f64(k)
+    Dz, H, W = v.shape
+    d = 0.0 if dskip is None else float(dskip)
+    out = []
+    for iz, iy, ix in voxels:
+        # K[iz - sz + Dz, iy - sy + H, ix - sx + W] over sz < Dz, sy < H, sx < W: a reversed window
+        win = k[iz + 1:iz + Dz + 1, iy + 1:iy + H + 1, ix + 1:ix + W + 1][::-1, ::-1, ::-1]
+        c = float(np.sum(win * v))
+        out.append(x[iz, iy, ix] * (c + d * v[iz, iy, ix]))
+    return np.array(out)

@@ -72,3 +72,20 @@ def implicit_filter_2d(H, W, N, C, W1, b1, W2, b2, W3, b3, sigma, omega0=10.0, o
     r2 = (py ** 2 + px ** 2).ravel()
     window = np.exp(-r2[None, :] / (2.0 * sigma[:, None] ** 2))           # [N*C, 4HW]
     return (window * o.T).reshape(N, C, 2 * H, 2 * W)
+
+
+def implicit_filter_3d(Dz, H, W, N, C, W1, b1, W2, b2, W3, b3, sigma, omega0=10.0, omega_hidden=1.0):
+    """Returns K [N, C, 2Dz, 2H, 2W] fp64 on the offset grid: the 2D network on the
+    coordinates p = (oz / Dz, oy / H, ox / W) of a volume's offsets, with the Gaussian
+    window of |p|^2 ("How HyenaND works", "1. An implicit filter": the kernel as a
+    continuous function of the grid coordinates, here of a 3D grid)."""
+    oz = np.arange(-Dz, Dz, dtype=np.float64) / Dz
+    oy = np.arange(-H, H, dtype=np.float64) / H
+    ox = np.arange(-W, W, dtype=np.float64) / W
+    pz, py, px = np.meshgrid(oz, oy, ox, indexing="ij")
+    feat = np.stack([pz.ravel(), py.ravel(), px.ravel()], axis=1)         # [8 Dz H W, 3] as (z, y, x)
+    o = _mlp(feat, W1, b1, W2, b2, W3, b3, omega0, omega_hidden)          # [8 Dz H W, N*C]
+    sigma = np.asarray(sigma, dtype=np.float64).reshape(N * C)
+    r2 = (pz ** 2 + py ** 2 + px ** 2).ravel()
+    window = np.exp(-r2[None, :] / (2.0 * sigma[:, None] ** 2))
+    return (window * o.T).reshape(N, C, 2 * Dz, 2 * H, 2 * W)

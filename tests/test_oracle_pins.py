@@ -560,3 +560,29 @@ def test_3d_single_slice_reduces_to_2d():
     y3 = oracle.hyena_3d(v, gates, k, dskip)
     y2 = oracle.hyena_2d(v[:, 0], gates[:, :, 0], k[:, :, 1], dskip)
     np.testing.assert_allclose(y3[:, 0], y2, rtol=1e-13, atol=1e-13)
+
+
+def test_3d_order1_voxels_match_the_chain():
+    rng = np.random.default_rng(66)
+    Dz, H, W = 3, 4, 5
+    v, x = rng.standard_normal((2, Dz, H, W))
+    k = rng.standard_normal((2 * Dz, 2 * H, 2 * W))
+    full = oracle.hyena_3d(v[None], x[None, None], k[None, None], np.array([[0.4]]))[0]
+    vox = [(0, 0, 0), (2, 3, 4), (1, 2, 0), (0, 3, 2)]
+    got = oracle.hyena_3d_order1_at(v, x, k, 0.4, vox)
+    np.testing.assert_allclose(got, [full[i] for i in vox], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("axis", [0, 1, 2])
+def test_implicit_3d_reduces_to_closed_form(axis):
+    """One coordinate through one unit per layer: K = Gaussian(|p|) sin(w_h sin(w0 a p_axis))."""
+    Dz, H, W, N, C, width = 2, 3, 4, 1, 2, 8
+    a, w0, wh = 0.7, 10.0, 1.0
+    sigma = np.array([[0.5, 0.8]])
+    k = oracle.implicit_filter_3d(Dz, H, W, N, C, *_onehot_net(width, 3, N * C, axis, a), sigma, w0, wh)
+    pz, py, px = np.meshgrid(np.arange(-Dz, Dz) / Dz, np.arange(-H, H) / H, np.arange(-W, W) / W, indexing="ij")
+    coord = (pz, py, px)[axis]
+    for c in range(C):
+        expect = np.exp(-(pz ** 2 + py ** 2 + px ** 2) / (2 * sigma[0, c] ** 2)) * np.sin(wh * np.sin(w0 * a * coord))
+        np.testing.assert_allclose(k[0, c], expect, rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(k[0, :, Dz, H, W], 0.0)     # offset 0: coordinate 0, window 1
