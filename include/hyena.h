@@ -18,8 +18,9 @@
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
  *    and 16-byte aligned, unless a comment says "host".
- *  - Activation layout: 1D [B, D, L] (one channel row per (b, d));
- *    2D [B, C, H, W]. io dtype is the plan's (fp32 or bf16); filters, spectra
+ *  - Activation layout: 1D [B, D, L] (one channel row per (b, d); or [B, L, D],
+ *    see hyena_plan_set_layout); 2D [B, C, H, W]; 3D [B, C, Dz, H, W]. io
+ *    dtype is the plan's (fp32 or bf16); filters, spectra
  *    and Dskip are always fp32 / complex64 (interleaved re, im).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only
  *    enqueue work; none synchronises the host except plan create / destroy.
@@ -69,8 +70,10 @@ typedef enum {
     HYENA_PATH_CLUSTER = 1,      /* 1D, M = 262144: a thread-block cluster per row */
     HYENA_PATH_2D = 2,           /* 2D grid (H = W = 256: column and row kernels through a workspace;
                                     smaller grids: a thread-block cluster per plane) */
-    HYENA_PATH_STAGED = 3        /* 1D, M in {65536, 131072}: column and row kernels per order,
+    HYENA_PATH_STAGED = 3,       /* 1D, M from 65536 to 1048576: column and row kernels per order,
                                     the row's transform in a device workspace */
+    HYENA_PATH_3D = 4            /* 3D grid: one batched 1D transform stage per axis through a
+                                    device workspace */
 } hyena_path_t;
 
 /* Activation layout of a 1D plan (hyena_plan_set_layout). */
@@ -94,6 +97,8 @@ typedef enum {
  *   p = (oy / H, ox / W), oy in [-H, H), ox in [-W, W)  (in = 2, num_freqs ignored),
  *   same two sine layers and head, K[n, c, oy + H, ox + W] =
  *   exp(-|p|^2 / (2 window[n*C + c]^2)) * o[n*C + c]           (window = Gaussian σ > 0)
+ * 3D: p = (oz / Dz, oy / H, ox / W) (in = 3), K[n, c, oz + Dz, oy + H, ox + W]
+ *   with the same Gaussian window of |p|^2; width 64 only.
  * Shapes: W1 [width, in], b1 [width], W2 [width, width], b2 [width],
  * W3 [N*D, width], b3 [N*D], window [N*D]; row-major. width <= 128 and a
  * multiple of 4; num_freqs <= 32. W3 must be 16-byte aligned.
@@ -110,12 +115,13 @@ typedef struct {
 /*
  * Create a plan.
  *   ndim      1 (sequence) or 2 (grid)
- *   shape     host array of ndim sizes: {L} or {H, W}; each >= 1.
- *             1D: L <= 131072. 2D: H == W, one of 32, 64, 128, 256.
+ *   shape     host array of ndim sizes: {L}, {H, W} or {Dz, H, W}; each >= 1.
+ *             1D: L <= 524288. 2D: H == W, one of 32, 64, 128, 256.
+ *             3D: Dz, H, W each 16, 32 or 64.
  *   channels  D (1D) or C (2D), >= 1
  *   order     N, 1..HYENA_MAX_ORDER
  *   io_dtype  storage type of v, the gates and y
- *   causal    must be 1 for ndim 1 and 0 for ndim 2
+ *   causal    must be 1 for ndim 1 and 0 for ndim 2 and 3
  * Allocates the plan's device twiddle tables on the current device (the plan
  * may only be used on that device) and synchronises. *out is NULL on error.
  */
@@ -135,24 +141,38 @@ HYENA_API hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const in
  */
 HYENA_API hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout);
 
+/*
+ * Errors that kernels of this plan recorded on the device. A kernel that
+ * waits on a barrier of its own (the tensor-core implicit network) bounds
+ * every wait; when one runs out it records the event in a device word of the
+ * plan, abandons the remaining work of that call and still exits cleanly, so
+ * the context stays usable. This call copies that word to the host (it
+ * synchronises with the device: call it after the work to check), stores it
+ * in *flags if flags is not NULL, clears it when clear != 0, and returns
+ * HYENA_ERR_CUDA if an error was recorded, HYENA_OK otherwise.
+ */
+HYENA_API hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear);
+
 /* Free the plan's device tables (synchronises the device). NULL is accepted. */
 HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);
 
 /*
  * Geometry of a plan (any out-pointer may be NULL):
- *   fft_len        M (1D) or 2H * 2W (2D): the padded transform size
+ *   fft_len        M (1D), 2H * 2W (2D) or 2Dz * 2H * 2W (3D): the padded transform size
  *   spectrum_elems complex64 elements of one (order, channel) spectrum:
- *                  M/2 + 1 (1D) or 2H * (W + 1) (2D)
+ *                  M/2 + 1 (1D), 2H * (W + 1) (2D) or 2Dz * 2H * 2W (3D)
  *   path           a hyena_path_t
  */
 HYENA_API hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path);
 
 /*
  * Bytes of device workspace hyena_forward needs for `batch`. It is 0, except
- * on HYENA_PATH_STAGED and on 2D plans with H = W = 256. There, rows (planes)
- * run in chunks that keep their transforms in L2, with two chunks in flight.
- * The workspace then holds min(rows, 2 * chunk) transforms: (M/2) * 8 bytes
- * per 1D row, 2H * (W/2) * 8 bytes per plane.
+ * on HYENA_PATH_STAGED, on 2D plans with H = W = 256 and on 3D plans. There,
+ * rows (planes, volumes) run in chunks that keep their transforms in L2: 1D
+ * rows with three chunks of 16 MB in flight, 2D planes with two of 32 MB, 3D
+ * volumes one of 32 MB at a time. The workspace holds min(rows, lanes * chunk)
+ * transforms: (M/2) * 8 bytes per 1D row, 2H * (W/2) * 8 bytes per plane,
+ * Dz * 2H * 2W * 8 bytes per volume.
  */
 HYENA_API size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch);
 
@@ -172,11 +192,15 @@ HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_im
  *           May be NULL when params is given: the filters are then generated by
  *           the implicit network, inside H_out, with no other memory.
  *   params  implicit network, or NULL (then h must not be NULL)
+ *           3D: [N, C, 2Dz, 2H, 2W] kernel on the offset grid, element
+ *           (oz, oy, ox) at [oz + Dz, oy + H, ox + W]; h must not be NULL.
  *   H_out   1D: [N, D, M/2 + 1] complex64, bin k = sum_t h[t] e^{-2πi k t / M};
  *           2D: [N, C, W + 1, 2H] complex64, the 2D DFT of the kernel placed
  *           cyclically (offset o at index o mod 2H, o mod 2W), bins over the
  *           full row axis and the non-negative half of the column axis,
  *           stored column-bin-major: bin (ky, kx) at [kx][ky].
+ *           3D: [N, C, 2Dz, 2H, 2W] complex64, the full 3D DFT of the kernel
+ *           placed cyclically, bin (kz, ky, kx) at [kz][ky][kx].
  *           Unnormalised. Must not overlap h.
  * Plans on HYENA_PATH_STAGED (64 MiB) and 2D plans with H = W = 256 (32 MiB)
  * transform the filters in chunks through a device buffer that the plan

@@ -85,6 +85,8 @@ class Plan:
     def spectrum_shape(self):
         if self.ndim == 1:
             return (self.order, self.channels, self.spectrum_elems)
+        if self.ndim == 3:
+            return (self.order, self.channels) + tuple(2 * e for e in self.shape)   # bin (kz, ky, kx) natural order
         H, W = self.shape
         return (self.order, self.channels, W + 1, 2 * H)   # bin (ky, kx) at [kx][ky]
 
@@ -94,7 +96,7 @@ class Plan:
     def implicit_filter(self, params: dict, out=None, stream=None):
         if out is None:
             shp = ((self.order, self.channels, self.shape[0]) if self.ndim == 1 else
-                   (self.order, self.channels, 2 * self.shape[0], 2 * self.shape[1]))
+                   (self.order, self.channels) + tuple(2 * e for e in self.shape))
             out = torch.empty(shp, dtype=torch.float32, device="cuda")
         c = implicit_params(params)
         _check(capi.hyena_implicit_filter(self.handle, c, out.data_ptr(), _stream(stream)), "hyena_implicit_filter")

@@ -32,7 +32,7 @@ EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
-    "hyena_forward_gated", "hyena_plan_set_layout",
+    "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors",
 )
 
 
@@ -67,6 +67,7 @@ def _load():
         "hyena_forward_host": ([p, i64, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_forward_gated": ([p, i64, p, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_plan_set_layout": ([p, i32], i32),
+        "hyena_plan_device_errors": ([p, ctypes.POINTER(i32), i32], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -96,6 +97,13 @@ def hyena_plan_destroy(plan) -> int:
 
 def hyena_plan_set_layout(plan, layout: int) -> int:
     return lib.hyena_plan_set_layout(plan, layout)
+
+
+def hyena_plan_device_errors(plan, clear: bool = False):
+    """Returns (status, device error word); synchronises with the device."""
+    f = ctypes.c_int()
+    st = lib.hyena_plan_device_errors(plan, ctypes.byref(f), 1 if clear else 0)
+    return st, f.value
 
 
 def hyena_plan_info(plan):

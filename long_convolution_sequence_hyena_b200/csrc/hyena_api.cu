@@ -12,6 +12,7 @@
 
 #include "hyena.h"
 #include "kernels_2d.cuh"
+#include "kernels_3d.cuh"
 #include "launch.h"
 #include "plan.h"
 
@@ -87,6 +88,7 @@ hyena_status_t check_implicit(const hyena_plan_s *p, const hyena_implicit_params
     if (!ip->W1 || !ip->b1 || !ip->W2 || !ip->b2 || !ip->W3 || !ip->b3 || !ip->window) return HYENA_ERR_INVALID_ARG;
     if (ip->width < 4 || ip->width > IMP_MAXW || (ip->width & 3)) return HYENA_ERR_UNSUPPORTED;
     if (p->ndim == 1 && (ip->num_freqs < 0 || 1 + 2 * ip->num_freqs > IMP_MAXF)) return HYENA_ERR_UNSUPPORTED;
+    if (p->ndim == 3 && ip->width != 64) return HYENA_ERR_UNSUPPORTED;   // 3D coordinates: tensor-core network only
     if (!aligned16(ip->W3)) return HYENA_ERR_ALIGNMENT;
     if (!std::isfinite(ip->omega0) || !std::isfinite(ip->omega_hidden)) return HYENA_ERR_INVALID_ARG;
     return HYENA_OK;
@@ -100,7 +102,8 @@ ImplicitArgs implicit_args(const hyena_plan_s *p, const hyena_implicit_params_t 
     a.L = p->L;
     a.H = p->Hh;
     a.W = p->Ww;
-    a.npos = p->ndim == 1 ? p->L : 4 * p->Hh * p->Ww;
+    a.Dz = p->Dd;
+    a.npos = p->ndim == 1 ? p->L : (p->ndim == 2 ? 4 * p->Hh * p->Ww : 8 * p->Dd * p->Hh * p->Ww);
     a.nout = (int64_t)p->order * p->D;
     a.out = out;
     a.out_stride = out_stride;
@@ -131,10 +134,10 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
     *out = nullptr;
     if (!shape || channels < 1 || order < 1 || order > HYENA_MAX_ORDER) return HYENA_ERR_INVALID_ARG;
     if (io_dtype != HYENA_F32 && io_dtype != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
-    if (ndim != 1 && ndim != 2) return HYENA_ERR_INVALID_ARG;
+    if (ndim < 1 || ndim > 3) return HYENA_ERR_INVALID_ARG;
     for (int i = 0; i < ndim; ++i)
         if (shape[i] < 1) return HYENA_ERR_INVALID_ARG;
-    if ((ndim == 1 && causal != 1) || (ndim == 2 && causal != 0)) return HYENA_ERR_UNSUPPORTED;
+    if ((ndim == 1 && causal != 1) || (ndim >= 2 && causal != 0)) return HYENA_ERR_UNSUPPORTED;
 
     hyena_plan_s p;
     p.ndim = ndim;
@@ -168,6 +171,14 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         if (p.path == HYENA_PATH_CLUSTER && !cluster_path_supported(p.MC)) return HYENA_ERR_UNSUPPORTED;
         p.spectrum_elems = p.MC + 1;
         p.tw_len = p.M;
+    } else if (ndim == 3) {
+        p.Dd = shape[0];
+        p.Hh = shape[1];
+        p.Ww = shape[2];
+        if (!grid3d_supported(p.Dd, p.Hh, p.Ww)) return HYENA_ERR_UNSUPPORTED;
+        p.path = HYENA_PATH_3D;
+        p.spectrum_elems = 8 * p.Dd * p.Hh * p.Ww;
+        p.tw_len = 2 * p.Ww;
     } else {
         p.Hh = shape[0];
         p.Ww = shape[1];
@@ -193,6 +204,16 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         cudaFree(p.tw);
         return HYENA_ERR_CUDA;
     }
+    if (cudaMalloc(&p.dev_err, 4 * sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p.tw);
+        return HYENA_ERR_NOMEM;
+    }
+    if (cudaMemset(p.dev_err, 0, 4 * sizeof(int)) != cudaSuccess) {
+        cudaFree(p.dev_err);
+        cudaFree(p.tw);
+        return HYENA_ERR_CUDA;
+    }
     if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
         bool ok = true;
         for (int i = 0; i < HYENA_STAGED_LANES && ok; ++i)
@@ -200,6 +221,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         p.has_lanes = true;
         if (!ok) {
             release_lanes(&p);
+            cudaFree(p.dev_err);
             cudaFree(p.tw);
             return HYENA_ERR_CUDA;
         }
@@ -210,6 +232,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         if (cudaMalloc(&p.spec_ws, sb) != cudaSuccess) {
             cudaGetLastError();
             release_lanes(&p);
+            cudaFree(p.dev_err);
             cudaFree(p.tw);
             return HYENA_ERR_NOMEM;
         }
@@ -217,6 +240,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         if (!p.spec_mu) {
             cudaFree(p.spec_ws);
             release_lanes(&p);
+            cudaFree(p.dev_err);
             cudaFree(p.tw);
             return HYENA_ERR_NOMEM;
         }
@@ -226,6 +250,7 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         release_lanes(&p);
         if (p.spec_ws) cudaFree(p.spec_ws);
         delete p.spec_mu;
+        cudaFree(p.dev_err);
         cudaFree(p.tw);
         return HYENA_ERR_NOMEM;
     }
@@ -239,6 +264,7 @@ hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     if (plan->tw && cudaFree(plan->tw) != cudaSuccess) st = HYENA_ERR_CUDA;
     if (!release_lanes(plan)) st = HYENA_ERR_CUDA;
     if (plan->spec_ws && cudaFree(plan->spec_ws) != cudaSuccess) st = HYENA_ERR_CUDA;
+    if (plan->dev_err && cudaFree(plan->dev_err) != cudaSuccess) st = HYENA_ERR_CUDA;
     delete plan->spec_mu;
     delete plan;
     return st;
@@ -251,9 +277,20 @@ hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout) {
     return HYENA_OK;
 }
 
+hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear) {
+    if (!plan) return HYENA_ERR_INVALID_ARG;
+    int h[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(h, plan->dev_err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return HYENA_ERR_CUDA;
+    if (clear && cudaMemset(plan->dev_err, 0, sizeof(h)) != cudaSuccess) return HYENA_ERR_CUDA;
+    if (flags) flags[0] = h[0];
+    return h[0] ? HYENA_ERR_CUDA : HYENA_OK;
+}
+
 hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path) {
     if (!plan) return HYENA_ERR_INVALID_ARG;
-    if (fft_len) *fft_len = plan->ndim == 1 ? plan->M : 4 * plan->Hh * plan->Ww;
+    if (fft_len)
+        *fft_len = plan->ndim == 1 ? plan->M
+                                   : (plan->ndim == 2 ? 4 * plan->Hh * plan->Ww : 8 * plan->Dd * plan->Hh * plan->Ww);
     if (spectrum_elems) *spectrum_elems = plan->spectrum_elems;
     if (path) *path = plan->path;
     return HYENA_OK;
@@ -261,6 +298,10 @@ hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spe
 
 size_t hyena_workspace_bytes(hyena_plan_t plan, int64_t batch) {
     if (!plan || batch < 0) return 0;
+    if (plan->path == HYENA_PATH_3D) {
+        const int64_t c = grid3d_chunk_volumes(plan->Dd, plan->Hh, plan->Ww), vols = batch * plan->D;
+        return (size_t)(vols < c ? vols : c) * (size_t)(plan->Dd * 4 * plan->Hh * plan->Ww) * sizeof(float2);
+    }
     if (plan->path == HYENA_PATH_2D && staged2d_supported(plan->Ww))
         return (size_t)staged2d_workspace_planes(plan->Ww, batch * plan->D) * (size_t)(2 * plan->Hh) *
                (size_t)(plan->Ww / 2) * sizeof(float2);
@@ -275,9 +316,10 @@ hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_implicit_par
     if (s != HYENA_OK) return s;
     if (!aligned16(h_out)) return HYENA_ERR_ALIGNMENT;
     if ((s = check_device(plan)) != HYENA_OK) return s;
-    const int64_t stride = plan->ndim == 1 ? plan->L : 4 * plan->Hh * plan->Ww;
+    const int64_t stride = plan->ndim == 1 ? plan->L
+                           : (plan->ndim == 2 ? 4 * plan->Hh * plan->Ww : 8 * plan->Dd * plan->Hh * plan->Ww);
     ImplicitArgs a = implicit_args(plan, params, h_out, stride, 2 * plan->Ww);
-    return launch_implicit(a, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+    return launch_implicit(a, plan->dev_err, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
 hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
@@ -293,13 +335,20 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
     const c32 *tw = reinterpret_cast<const c32 *>(plan->tw);
     const float *src = h;
     cudaError_t e;
+    if (plan->ndim == 3) {
+        if (!h) return HYENA_ERR_UNSUPPORTED;   // 3D spectra from taps only (hyena_implicit_filter writes them)
+        if (!aligned16(h)) return HYENA_ERR_ALIGNMENT;
+        const int64_t V = plan->Dd * plan->Hh * plan->Ww;
+        e = launch_spec_3d(h, 8 * V, Hc, nrows, (int)plan->Dd, (int)plan->Hh, (int)plan->Ww, tw + plan->tw_len, st);
+        return e == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
+    }
     if (plan->ndim == 1) {
         int64_t src_stride = plan->L;
         if (!h) {
             // generate the taps inside each row's own output slot, then transform in place
             src_stride = 2 * (plan->MC + 1);
             ImplicitArgs a = implicit_args(plan, params, reinterpret_cast<float *>(H_out), src_stride, 0);
-            if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
+            if (launch_implicit(a, plan->dev_err, st) != cudaSuccess) return HYENA_ERR_CUDA;
             src = reinterpret_cast<const float *>(H_out);
         }
         if (plan->path == HYENA_PATH_STAGED) {
@@ -319,7 +368,7 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             rs = 2 * (plan->Ww + 1);
             cs = 2 * plan->Hh * rs;
             ImplicitArgs a = implicit_args(plan, params, reinterpret_cast<float *>(H_out), cs, rs);
-            if (launch_implicit(a, st) != cudaSuccess) return HYENA_ERR_CUDA;
+            if (launch_implicit(a, plan->dev_err, st) != cudaSuccess) return HYENA_ERR_CUDA;
             src = reinterpret_cast<const float *>(H_out);
         }
         if (plan->spec_ws) {
@@ -356,6 +405,26 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
     hyena_status_t s = check_device(plan);
     if (s != HYENA_OK) return s;
 
+    if (plan->ndim == 3) {
+        Fwd3dArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.v = v;
+        a.k = k;
+        for (int n = 0; n < plan->order; ++n) a.gates[n] = gates[n];
+        a.K = reinterpret_cast<const c32 *>(H);
+        a.dskip = Dskip;
+        a.y = y;
+        a.tws = reinterpret_cast<const c32 *>(plan->tw) + plan->tw_len;   // W_1024
+        a.ws = reinterpret_cast<float2 *>(workspace);
+        a.C = plan->D;
+        a.B = batch;
+        a.Dz = (int)plan->Dd;
+        a.H = (int)plan->Hh;
+        a.W = (int)plan->Ww;
+        a.order = plan->order;
+        return launch_fwd_3d(a, batch * plan->D, plan->dtype, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK
+                                                                                                  : HYENA_ERR_CUDA;
+    }
     if (plan->ndim == 2) {
         Fwd2dArgs a;
         std::memset(&a, 0, sizeof(a));

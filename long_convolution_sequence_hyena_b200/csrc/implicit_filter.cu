@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(IMP_THREADS) hyena_implicit_filter_kernel(cons
     }
 }
 
-cudaError_t launch_implicit(const ImplicitArgs &a, cudaStream_t st) {
+cudaError_t launch_implicit(const ImplicitArgs &a, int *err, cudaStream_t st) {
+    if (implicit_tc_supported(a)) return launch_implicit_tc(a, err, st);
     const size_t sm = sizeof(ImplicitSmem);
     cudaError_t e = cudaFuncSetAttribute(hyena_implicit_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;

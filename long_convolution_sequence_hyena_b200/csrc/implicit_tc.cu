@@ -1,0 +1,342 @@
+// Implicit filter network with the head on the 5th-generation tensor cores
+// (tcgen05.mma, accumulators in tensor memory), for networks of width 64.
+//
+// The network is the one of kernels_implicit.cuh ("Hyena — Long Convolutions
+// Math", "Implicit filters: an MLP over positions" and "The decay window";
+// "How HyenaND works", "1. An implicit filter"): positional features, two sine
+// layers of width 64, a linear head to N*D outputs, the window. The head is a
+// dense contraction o[p][j] = sum_k a2[p][k] W3[j][k] over every position p and
+// output j, and it holds almost all of the work (64 N D multiply-adds per
+// position against 64 (fin + 64) for the two hidden layers), so it runs on the
+// tensor cores; the hidden layers stay on the CUDA cores.
+//
+// Precision: the filters must match an fp64 evaluation to fp32 accuracy, which
+// one TF32 product (10-bit mantissa) cannot. Each operand is split as
+// x = hi + lo with hi = x rounded to TF32 and lo = x - hi (exact in fp32), and
+// the head accumulates hi*hi + hi*lo + lo*hi in fp32 (the dropped lo*lo term
+// and the TF32 rounding of lo are about 2^-21 of the product).
+//
+// One CTA (512 threads) per tile of 128 positions and one slice of the
+// outputs, one CTA per SM (about 160 KB of shared memory):
+//   1. thread (p, part) computes the features of position p, the 64 units of
+//      the first sine layer and units [16 part, 16 part + 16) of the second,
+//      and writes them, split, into the A tile (shared memory, the
+//      tensor core's K-major layout without swizzle: 8 x 16-byte core matrices);
+//   2. per slice of 128 outputs: the CTA converts W3's rows into the B tile;
+//      one thread issues 24 MMAs (M 128, N 128, K 8; eight K steps, three
+//      products) into one of two tensor-memory accumulators and commits them to
+//      an mbarrier; while they run, the 16 warps read the previous slice's
+//      accumulator (tcgen05.ld), add the bias, apply the window and store.
+// Every wait on the mbarrier is bounded: on a timeout the kernel records an
+// error in *err, skips the remaining MMAs and still frees its tensor memory.
+#include <cuda_runtime.h>
+
+#include "launch.h"
+
+namespace hyena {
+
+namespace {
+
+constexpr int TP = 128;            // positions per tile (the MMA's M)
+constexpr int NT = 128;            // outputs per slice (the MMA's N)
+constexpr int KW = 64;             // network width (the MMA's K over 8 steps)
+constexpr int THREADS = 512;
+constexpr int PARTS = THREADS / TP;      // threads per position (each takes KW / PARTS second-layer units)
+constexpr int LBO = 16 * 128;      // bytes between K-adjacent core matrices (16 row groups of 128 B)
+constexpr int SBO = 128;           // bytes between 8-row groups
+constexpr int TMEM_COLS = 2 * NT;      // two accumulators of 128 columns
+constexpr int SLICE_OUT = 512;         // outputs per CTA (grid.y covers the rest)
+
+struct alignas(128) TcSmem {
+    float a[2][TP * KW];           // A tile: hi, lo
+    float b[2][NT * KW];           // B tile: hi, lo
+    float w1t[IMP_MAXF][KW];       // first layer weights, transposed: [feature][unit]
+    float w2[KW][KW];              // second layer weights [unit][input]
+    float b1[KW], b2[KW];
+    unsigned long long mbar;
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// x rounded to TF32 (round to nearest, ties away), as an fp32 bit pattern whose low 13 bits are zero
+__device__ __forceinline__ float tf32_hi(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// Byte offset of element (row, k) in a K-major tile without swizzle: core matrices
+// of 8 rows x 4 elements (16 bytes per row), 8-row groups SBO apart, K chunks LBO apart.
+__device__ __forceinline__ int core_off(int row, int kc) { return kc * LBO + (row >> 3) * SBO + (row & 7) * 16; }
+
+// Shared-memory matrix descriptor (K-major, no swizzle): start address, leading
+// byte offset (between K-adjacent core matrices), stride byte offset (between
+// 8-row groups), descriptor version 1, layout type 0.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((LBO >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((SBO >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// Instruction descriptor: fp32 accumulator, TF32 A and B, both K-major, N = NT, M = TP.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TP >> 4) << 24);
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(unsigned long long *mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(mbar))
+                 : "memory");
+}
+
+// Bounded wait for the mbarrier's phase `parity` to complete; false on timeout.
+__device__ __forceinline__ bool mbar_wait(unsigned long long *mbar, uint32_t parity) {
+    for (int i = 0; i < (1 << 22); ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(saddr(mbar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
+    uint32_t u[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+          "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+          "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const ImplicitArgs a, int *err) {
+    extern __shared__ float4 tc_smem4[];
+    TcSmem &S = *reinterpret_cast<TcSmem *>(tc_smem4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int fin = a.ndim == 1 ? 1 + 2 * a.p.num_freqs : a.ndim;
+    const int64_t p0 = (int64_t)blockIdx.x * TP;
+
+    // weights of the hidden layers, and the barrier and tensor memory
+    for (int i = tid; i < KW * fin; i += THREADS) S.w1t[i % fin][i / fin] = __ldg(a.p.W1 + i);
+    for (int i = tid; i < KW * KW; i += THREADS) S.w2[i / KW][i % KW] = __ldg(a.p.W2 + i);
+    if (tid < KW) {
+        S.b1[tid] = __ldg(a.p.b1 + tid);
+        S.b2[tid] = __ldg(a.p.b2 + tid);
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.mbar)));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&S.tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+
+    // 1. features and hidden layers of position p; this thread writes units [16 part, 16 part + 16).
+    // The features are formed one at a time and folded into all 64 first-layer sums at once.
+    {
+        const int p = tid & (TP - 1), part = tid / TP;
+        const int64_t pos = p0 + p;
+        const bool in = pos < a.npos;
+        float a1[KW];
+#pragma unroll
+        for (int j = 0; j < KW; ++j) a1[j] = 0.f;
+#pragma unroll 1
+        for (int f = 0; f < fin; ++f) {
+            float fv = 0.f;
+            if (in) {
+                if (a.ndim == 1) {
+                    if (f == 0) {
+                        fv = (float)((double)pos / (double)a.L);
+                    } else {
+                        const int64_t k = (f + 1) / 2;
+                        const int64_t r = (k * pos) % a.L;   // angle 2 pi k t / L, reduced exactly first
+                        float sv, cv;
+                        sincospif((float)(2.0 * (double)r / (double)a.L), &sv, &cv);
+                        fv = (f & 1) ? cv : sv;
+                    }
+                } else if (a.ndim == 2) {
+                    const int64_t iy = pos / (2 * a.W), ix = pos - iy * (2 * a.W);
+                    fv = f == 0 ? (float)((double)(iy - a.H) / (double)a.H) : (float)((double)(ix - a.W) / (double)a.W);
+                } else {   // 3D: (oz / Dz, oy / H, ox / W) on the offset grid [2Dz][2H][2W]
+                    const int64_t hw = 4 * a.H * a.W;
+                    const int64_t iz = pos / hw, rem = pos - iz * hw;
+                    const int64_t iy = rem / (2 * a.W), ix = rem - iy * (2 * a.W);
+                    fv = f == 0 ? (float)((double)(iz - a.Dz) / (double)a.Dz)
+                                : (f == 1 ? (float)((double)(iy - a.H) / (double)a.H)
+                                          : (float)((double)(ix - a.W) / (double)a.W));
+                }
+            }
+            const float4 *wrow = reinterpret_cast<const float4 *>(S.w1t[f]);
+#pragma unroll
+            for (int j4 = 0; j4 < KW / 4; ++j4) {
+                const float4 w = wrow[j4];
+                a1[4 * j4] = fmaf(w.x, fv, a1[4 * j4]);
+                a1[4 * j4 + 1] = fmaf(w.y, fv, a1[4 * j4 + 1]);
+                a1[4 * j4 + 2] = fmaf(w.z, fv, a1[4 * j4 + 2]);
+                a1[4 * j4 + 3] = fmaf(w.w, fv, a1[4 * j4 + 3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KW; ++j) a1[j] = sinf(a.p.omega0 * (a1[j] + S.b1[j]));
+        unsigned char *ahi = reinterpret_cast<unsigned char *>(S.a[0]);
+        unsigned char *alo = reinterpret_cast<unsigned char *>(S.a[1]);
+#pragma unroll 1
+        for (int c = 0; c < KW / PARTS / 4; ++c) {   // 4 units per 16-byte core-matrix row
+            const int kc = (KW / PARTS / 4) * part + c;
+            float hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 4 * kc + u;
+                const float4 *wrow = reinterpret_cast<const float4 *>(S.w2[j]);
+                float acc = 0.f;
+#pragma unroll
+                for (int k4 = 0; k4 < KW / 4; ++k4) {
+                    const float4 w = wrow[k4];
+                    acc = fmaf(w.x, a1[4 * k4], acc);
+                    acc = fmaf(w.y, a1[4 * k4 + 1], acc);
+                    acc = fmaf(w.z, a1[4 * k4 + 2], acc);
+                    acc = fmaf(w.w, a1[4 * k4 + 3], acc);
+                }
+                const float v = in ? sinf(a.p.omega_hidden * (acc + S.b2[j])) : 0.f;
+                hi[u] = tf32_hi(v);
+                lo[u] = v - hi[u];
+            }
+            const int off = core_off(p, kc);
+            *reinterpret_cast<float4 *>(ahi + off) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<float4 *>(alo + off) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+
+    // 2. head slices
+    const int64_t o_begin = (int64_t)blockIdx.y * SLICE_OUT;
+    const int64_t o_end = o_begin + SLICE_OUT < a.nout ? o_begin + SLICE_OUT : a.nout;
+    const int nslices = (int)((o_end - o_begin + NT - 1) / NT);
+    const int q = warp & 3, cq = warp >> 2;            // TMEM lane quarter, column quarter
+    const int prow = 32 * q + lane;                    // this thread's position in the epilogue
+    const int64_t ppos = p0 + prow;
+    float we = 0.f;                                    // window exponent argument: t (1D) or |p|^2 (2D)
+    int64_t poff = ppos;
+    if (a.ndim == 1) {
+        we = (float)ppos;
+    } else if (a.ndim == 2 && ppos < a.npos) {
+        const int64_t iy = ppos / (2 * a.W), ix = ppos - iy * (2 * a.W);
+        const float py = (float)((double)(iy - a.H) / (double)a.H), px = (float)((double)(ix - a.W) / (double)a.W);
+        we = py * py + px * px;
+        poff = iy * a.out_row_stride + ix;
+    } else if (a.ndim == 3 && ppos < a.npos) {   // output [2Dz][2H][2W] contiguous per channel
+        const int64_t hw = 4 * a.H * a.W;
+        const int64_t iz = ppos / hw, rem = ppos - iz * hw;
+        const int64_t iy = rem / (2 * a.W), ix = rem - iy * (2 * a.W);
+        const float pz = (float)((double)(iz - a.Dz) / (double)a.Dz);
+        const float py = (float)((double)(iy - a.H) / (double)a.H), px = (float)((double)(ix - a.W) / (double)a.W);
+        we = pz * pz + py * py + px * px;
+    }
+    bool ok = true;
+    uint32_t phase = 0;
+    auto epilogue = [&](int s) {
+        float r[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((s & 1) * NT + 32 * cq), r);
+        if (ppos >= a.npos) return;
+#pragma unroll 4
+        for (int c = 0; c < 32; ++c) {
+            const int64_t o = o_begin + (int64_t)s * NT + 32 * cq + c;
+            if (o >= o_end) break;
+            const float wp = __ldg(a.p.window + o);
+            const float esc = a.ndim == 1 ? -wp : -1.f / (2.f * wp * wp);
+            a.out[o * a.out_stride + poff] = expf(esc * we) * (r[c] + __ldg(a.p.b3 + o));
+        }
+    };
+#pragma unroll 1
+    for (int s = 0; s < nslices; ++s) {
+        // B tile of slice s: rows o of W3 as 16-byte core-matrix rows, split
+        {
+            unsigned char *bhi = reinterpret_cast<unsigned char *>(S.b[0]);
+            unsigned char *blo = reinterpret_cast<unsigned char *>(S.b[1]);
+            const int o = tid & (NT - 1);
+            const int64_t og = o_begin + (int64_t)s * NT + o;
+#pragma unroll
+            for (int i = 0; i < KW / 4 / (THREADS / NT); ++i) {
+                const int kc = tid / NT + (THREADS / NT) * i;
+                float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (og < o_end) w = __ldg(reinterpret_cast<const float4 *>(a.p.W3 + og * KW) + kc);
+                const float4 h4 = make_float4(tf32_hi(w.x), tf32_hi(w.y), tf32_hi(w.z), tf32_hi(w.w));
+                const int off = core_off(o, kc);
+                *reinterpret_cast<float4 *>(bhi + off) = h4;
+                *reinterpret_cast<float4 *>(blo + off) = make_float4(w.x - h4.x, w.y - h4.y, w.z - h4.z, w.w - h4.w);
+            }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tensor core sees the tiles
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && ok) {
+            const uint32_t d = tmem + (uint32_t)((s & 1) * NT);
+            const uint32_t ah = saddr(S.a[0]), al = saddr(S.a[1]), bh = saddr(S.b[0]), bl = saddr(S.b[1]);
+#pragma unroll
+            for (int ks = 0; ks < KW / 8; ++ks) {   // K step of 8 = two core matrices along K
+                const uint32_t ko = (uint32_t)(2 * ks * LBO);
+                mma_tf32(d, smem_desc(ah + ko), smem_desc(bh + ko), ks > 0);
+                mma_tf32(d, smem_desc(ah + ko), smem_desc(bl + ko), 1);
+                mma_tf32(d, smem_desc(al + ko), smem_desc(bh + ko), 1);
+            }
+            mma_commit(&S.mbar);
+        }
+        if (s > 0) epilogue(s - 1);   // overlaps the MMAs of slice s
+        if (ok && !mbar_wait(&S.mbar, phase)) {
+            ok = false;
+            atomicExch(err, 1);
+        }
+        phase ^= 1;
+        tc_fence_after();
+        __syncthreads();   // slice s complete (or abandoned) before the B tile is rewritten
+    }
+    if (nslices > 0 && ok) epilogue(nslices - 1);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+}
+
+}  // namespace
+
+bool implicit_tc_supported(const ImplicitArgs &a) { return a.p.width == KW; }
+
+size_t implicit_tc_smem_bytes() { return sizeof(TcSmem) + 128; }
+
+cudaError_t launch_implicit_tc(const ImplicitArgs &a, int *err, cudaStream_t st) {
+    const int sm = (int)implicit_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(hyena_implicit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((a.npos + TP - 1) / TP), (unsigned)((a.nout + SLICE_OUT - 1) / SLICE_OUT));
+    hyena_implicit_tc_kernel<<<grid, THREADS, sm, st>>>(a, err);
+    return cudaGetLastError();
+}
+
+}  // namespace hyena

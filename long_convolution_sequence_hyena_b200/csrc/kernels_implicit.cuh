@@ -30,7 +30,8 @@ struct ImplicitArgs {
     hyena_implicit_params_t p;
     int ndim;
     int64_t L;                 // 1D length
-    int64_t H, W;              // 2D half-extents (grid is 2H x 2W offsets)
+    int64_t H, W;              // 2D / 3D half-extents (grid is 2H x 2W offsets)
+    int64_t Dz;                // 3D half-depth (grid is 2Dz x 2H x 2W offsets)
     int64_t npos;              // L or 4 H W
     int64_t nout;              // N * channels
     float *out;                // output base

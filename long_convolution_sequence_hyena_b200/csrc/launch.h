@@ -28,10 +28,10 @@ cudaError_t launch_spec_1d_cluster(const float *h, int64_t h_stride, int64_t L, 
 // HYENA_STAGED_LANES chunks of HYENA_STAGED_CHUNK_MB of transforms in flight,
 // one per lane; spectra and the 2D path use the first two.
 #ifndef HYENA_STAGED_LANES
-#define HYENA_STAGED_LANES 2
+#define HYENA_STAGED_LANES 3
 #endif
 #ifndef HYENA_STAGED_CHUNK_MB
-#define HYENA_STAGED_CHUNK_MB 32
+#define HYENA_STAGED_CHUNK_MB 16
 #endif
 static_assert(HYENA_STAGED_LANES >= 2 && HYENA_STAGED_LANES <= 8, "lane count");
 struct StagedLanes {
@@ -85,7 +85,19 @@ struct Fwd2dArgs;
 cudaError_t launch_fwd_2d(const Fwd2dArgs &a, int64_t W, hyena_dtype_t dt, cudaStream_t st);
 cudaError_t launch_spec_2d(const float *K, int64_t rs, int64_t cs, c32 *Kout, int64_t n, int64_t W, const c32 *tw,
                            cudaStream_t st);
-// implicit filter network
-cudaError_t launch_implicit(const ImplicitArgs &a, cudaStream_t st);
+// 3D grids (Dz, H, W each 16, 32 or 64): separable staged transforms through a
+// workspace of grid3d_chunk_volumes volumes of [Dz][2H][2W] complex64
+struct Fwd3dArgs;
+bool grid3d_supported(int64_t Dz, int64_t H, int64_t W);
+int64_t grid3d_chunk_volumes(int64_t Dz, int64_t H, int64_t W);
+cudaError_t launch_fwd_3d(const Fwd3dArgs &a, int64_t volumes, hyena_dtype_t dt, cudaStream_t st);
+cudaError_t launch_spec_3d(const float *K, int64_t cs, c32 *Kout, int64_t n, int Dz, int H, int W, const c32 *tws,
+                           cudaStream_t st);
+// implicit filter network: width 64 with the head on the tensor cores
+// (implicit_tc.cu), other widths on the CUDA cores; err: the plan's device
+// error word (bounded waits that time out set it)
+cudaError_t launch_implicit(const ImplicitArgs &a, int *err, cudaStream_t st);
+bool implicit_tc_supported(const ImplicitArgs &a);
+cudaError_t launch_implicit_tc(const ImplicitArgs &a, int *err, cudaStream_t st);
 
 }  // namespace hyena

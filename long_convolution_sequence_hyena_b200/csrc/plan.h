@@ -25,6 +25,7 @@ struct hyena_plan_s {
     int64_t MC = 0;              // M / 2: length of the packed complex FFT
     // 2D geometry
     int64_t Hh = 0, Ww = 0;      // grid extents (the transform is 2H x 2W)
+    int64_t Dd = 0;              // 3D: depth (the transform is 2Dz x 2H x 2W)
     int64_t spectrum_elems = 0;  // complex bins per (order, channel)
     // device tables (owned)
     int64_t tw_len = 0;          // 1D: M; 2D: 2W
@@ -39,4 +40,6 @@ struct hyena_plan_s {
     // from several threads run one after the other on the GPU.
     float2 *spec_ws = nullptr;
     std::mutex *spec_mu = nullptr;
+    // device error word (owned): set by a kernel whose bounded wait timed out
+    int *dev_err = nullptr;
 };

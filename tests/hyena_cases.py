@@ -157,3 +157,51 @@ def compare_gated_2d(w: Workload, inp, k64, y_gpu, planes=None, context=""):
         worst = (np.abs(got - ref) / (MAXABS_FACTOR * np.maximum(bound, 1e-300))[:, None, None]).max()
         assert worst <= 1.0, "%s: per-element error %.3f x the bound" % (context, worst)
     return err
+
+
+# ------------------------------------------------------------------------ 3D --
+
+def case_3d(B, C, shape, N, dtype="f32", seed=0, sigma=0.5):
+    """A 3D workload (shape (Dz, H, W)) with explicit kernels: Gaussian taps on the offset grid
+    under a Gaussian envelope of |p|^2, p = (oz / Dz, oy / H, ox / W)."""
+    return Workload("case3d_b%d_c%d_%dx%dx%d_n%d_%s" % ((B, C) + tuple(shape) + (N, dtype)), 3, B, C, tuple(shape), N,
+                    dtype, "explicit", sigma=sigma, seed=seed)
+
+
+def inputs_3d(w: Workload):
+    """Seeded inputs of a 3D case: v, gates ~ N(0, 1) in the io dtype, dskip ~ N(0, 1), kernels [N, C, 2Dz, 2H, 2W]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    Dz, H, W = w.shape
+    adt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    v = torch.randn((w.B, w.D, Dz, H, W), generator=g, dtype=torch.float64).to(adt)
+    gates = torch.randn((w.order, w.B, w.D, Dz, H, W), generator=g, dtype=torch.float64).to(adt)
+    dskip = torch.randn((w.order, w.D), generator=g, dtype=torch.float64).to(torch.float32)
+    oz = torch.arange(-Dz, Dz, dtype=torch.float64) / Dz
+    oy = torch.arange(-H, H, dtype=torch.float64) / H
+    ox = torch.arange(-W, W, dtype=torch.float64) / W
+    r2 = oz[:, None, None] ** 2 + oy[None, :, None] ** 2 + ox[None, None, :] ** 2
+    h = (torch.randn((w.order, w.D, 2 * Dz, 2 * H, 2 * W), generator=g, dtype=torch.float64)
+         * torch.exp(-r2 / (2 * w.sigma ** 2))).to(torch.float32)
+    k = torch.randn((w.B, w.D, Dz, H, W), generator=g, dtype=torch.float64).to(adt)
+    return {"v": v, "gates": gates, "dskip": dskip, "h": h, "k": k}
+
+
+def compare_3d(w: Workload, inp, k64, y_gpu, vols=None, gated=False, context=""):
+    N, B, C = w.order, w.B, w.D
+    Dz, H, W = w.shape
+    P = B * C
+    vols = np.arange(P) if vols is None else np.asarray(vols)
+    v = inp["v"].double().reshape(P, Dz, H, W).numpy()[vols]
+    gates = inp["gates"].double().reshape(N, P, Dz, H, W).numpy()[:, vols]
+    dsk = inp["dskip"].double().numpy()
+    if gated:
+        kk = inp["k"].double().reshape(P, Dz, H, W).numpy()[vols]
+        ref = oracle.hyena_gated(v, kk, gates, k64, dsk, fidx=vols % C)
+    else:
+        ref = oracle.hyena_3d(v, gates, k64, dsk, fidx=vols % C)
+    got = y_gpu.detach().double().cpu().reshape(P, Dz, H, W).numpy()[vols]
+    assert np.all(np.isfinite(got)), context + ": non-finite output"
+    err = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert err <= REL_L2[w.dtype], "%s: relative L2 error %.3e > %.1e" % (context, err, REL_L2[w.dtype])
+    return err

@@ -46,7 +46,9 @@ def test_status_strings(capi):
     ((1, [256], 4, 9, 1, 1), "HYENA_ERR_INVALID_ARG"),        # order above HYENA_MAX_ORDER
     ((1, [0], 4, 2, 1, 1), "HYENA_ERR_INVALID_ARG"),          # empty sequence
     ((1, [256], 4, 2, 7, 1), "HYENA_ERR_INVALID_ARG"),        # bad dtype
-    ((3, [4, 4, 4], 4, 1, 1, 0), "HYENA_ERR_INVALID_ARG"),    # 3D
+    ((4, [4, 4, 4, 4], 4, 1, 1, 0), "HYENA_ERR_INVALID_ARG"), # 4D
+    ((3, [4, 4, 4], 4, 1, 1, 0), "HYENA_ERR_UNSUPPORTED"),    # 3D extents outside 16, 32, 64
+    ((3, [16, 16, 16], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"), # causal 3D
     ((1, [256], 4, 2, 1, 0), "HYENA_ERR_UNSUPPORTED"),        # non-causal 1D
     ((2, [64, 64], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # causal 2D
     ((1, [524289], 4, 1, 1, 1), "HYENA_ERR_UNSUPPORTED"),     # longer than the longest path (M = 2^20)

@@ -34,7 +34,7 @@ def _plan(w, layout="bld"):
     (7, 2, 3, 1, "f32", 0),
     (65536, 1, 6, 3, "bf16", 3),     # staged long rows: lanes are adjacent channels
     (40001, 2, 3, 2, "f32", 3),      # staged, odd length
-    (100000, 1, 2, 1, "f32", 1),     # cluster
+    (100000, 1, 2, 1, "f32", 3),     # staged, M = 262144
 ])
 def test_bld_forward_matches_oracle(L, B, D, N, dtype, path):
     w = explicit_case(B, D, L, N, dtype, seed=2000 + L % 97 + D, alpha=(1e-4, 1e-2) if L > 16384 else (1e-3, 1e-1))

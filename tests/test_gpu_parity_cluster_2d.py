@@ -18,8 +18,9 @@ def api():
 
 
 def long_path(plan):
-    """Path the library takes for a 1D plan with M > 32768: staged up to M = 131072, else cluster."""
-    return 3 if plan.fft_len in (65536, 131072) else 1
+    """Path the library takes for a 1D plan with M > 32768: the staged four-step path (the
+    cluster kernel only when forced)."""
+    return 3
 
 
 def _run(api, w, inp):
@@ -69,14 +70,14 @@ def test_cluster_batches_and_channels(api, L, B, D, N, dtype):
 
 
 def test_staged_chunks(api):
-    """More rows than one workspace chunk holds (M = 65536: 128 rows per chunk, two chunks in
-    flight on two streams); rows on both sides of the chunk boundaries are checked."""
+    """More rows than one workspace chunk holds (M = 65536: 64 rows per 16 MB chunk, three
+    chunks in flight on three streams); rows on both sides of the chunk boundaries are checked."""
     w = explicit_case(2, 150, 16385, 2, "bf16", seed=1234, alpha=(1e-4, 1e-2))
     inp = make_inputs(w)
     plan, _, y = _run(api, w, inp)
-    assert plan.path == 3 and plan.workspace_bytes(2) == 256 * 32768 * 8
+    assert plan.path == 3 and plan.workspace_bytes(2) == 3 * 64 * 32768 * 8
     # visit order is d-major, b-minor: visit index o -> flat row (o % B) * D + o // B
-    visits = np.array([0, 1, 127, 128, 255, 256, 298, 299])
+    visits = np.array([0, 1, 63, 64, 127, 128, 191, 192, 255, 256, 298, 299])
     rows = (visits % 2) * 150 + visits // 2
     compare(w, inp, oracle_filters_1d(w, inp), y, rows=rows, context="staged chunks")
 
