@@ -153,6 +153,22 @@ HYENA_API hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout);
  */
 HYENA_API hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear);
 
+/*
+ * hyena_plan_create with options. flags is 0 (the same plan as
+ * hyena_plan_create) or HYENA_PLAN_RADIX3: a 1D plan then pads to the smallest
+ * M = 6 * 2^j >= 2L when that is below the power of two ("Hyena — Long
+ * Convolutions Math", "Linear vs circular": any transform of at least 2L
+ * points keeps the product causal; "Counting the cost": padding 2L up to a
+ * power of two can nearly double the work), e.g. 6144 points instead of 8192
+ * for L = 3000. Such plans (2^j from 16 to 4096, so L <= 12288) run one
+ * channel row per thread group through a radix-3 step and three
+ * power-of-two transforms; the spectrum has M/2 + 1 bins as for any 1D plan.
+ * Other plans ignore the flag. Unknown flags return HYENA_ERR_INVALID_ARG.
+ */
+#define HYENA_PLAN_RADIX3 1
+HYENA_API hyena_status_t hyena_plan_create_ex(hyena_plan_t *out, int ndim, const int64_t *shape, int64_t channels,
+                                              int order, hyena_dtype_t io_dtype, int causal, int flags);
+
 /* Free the plan's device tables (synchronises the device). NULL is accepted. */
 HYENA_API hyena_status_t hyena_plan_destroy(hyena_plan_t plan);
 

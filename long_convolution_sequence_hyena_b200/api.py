@@ -47,17 +47,19 @@ def implicit_params(p: dict) -> capi.hyena_implicit_params_t:
 class Plan:
     """A plan for one geometry: shape (L,) or (H, W), channels, order, io dtype, and the
     activation layout of 1D plans: "bdl" ([B, D, L], the default) or "bld" ([B, L, D],
-    channels-last, read and written in place)."""
+    channels-last, read and written in place). radix3: a 1D plan may pad to M = 6 * 2^j
+    when that is below the power of two."""
 
-    def __init__(self, shape, channels: int, order: int, dtype=torch.bfloat16, layout: str = "bdl"):
+    def __init__(self, shape, channels: int, order: int, dtype=torch.bfloat16, layout: str = "bdl",
+                 radix3: bool = False):
         shape = tuple(int(s) for s in shape)
         self.ndim = len(shape)
         self.shape = shape
         self.channels = int(channels)
         self.order = int(order)
         self.dtype = dtype
-        st, h = capi.hyena_plan_create(self.ndim, shape, self.channels, self.order, _DT[dtype],
-                                       1 if self.ndim == 1 else 0)
+        st, h = capi.hyena_plan_create_ex(self.ndim, shape, self.channels, self.order, _DT[dtype],
+                                          1 if self.ndim == 1 else 0, capi.HYENA_PLAN_RADIX3 if radix3 else 0)
         _check(st, "hyena_plan_create")
         self.handle = h
         st, self.fft_len, self.spectrum_elems, self.path = capi.hyena_plan_info(h)

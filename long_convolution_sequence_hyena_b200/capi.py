@@ -19,6 +19,7 @@ HYENA_F32, HYENA_BF16 = 0, 1
  HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA, HYENA_ERR_NOMEM) = range(7)
 HYENA_PATH_CTA, HYENA_PATH_CLUSTER, HYENA_PATH_2D, HYENA_PATH_STAGED = 0, 1, 2, 3
 HYENA_LAYOUT_BDL, HYENA_LAYOUT_BLD = 0, 1
+HYENA_PLAN_RADIX3 = 1
 
 STATUS_NAMES = {
     HYENA_OK: "HYENA_OK", HYENA_ERR_INVALID_ARG: "HYENA_ERR_INVALID_ARG",
@@ -32,7 +33,7 @@ EXPORTED = (
     "hyena_plan_create", "hyena_plan_destroy", "hyena_plan_info", "hyena_workspace_bytes",
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
-    "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors",
+    "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors", "hyena_plan_create_ex",
 )
 
 
@@ -68,6 +69,7 @@ def _load():
         "hyena_forward_gated": ([p, i64, p, p, ctypes.POINTER(p), p, p, p, p, sz, p], i32),
         "hyena_plan_set_layout": ([p, i32], i32),
         "hyena_plan_device_errors": ([p, ctypes.POINTER(i32), i32], i32),
+        "hyena_plan_create_ex": ([ctypes.POINTER(p), i32, ctypes.POINTER(i64), i64, i32, i32, i32, i32], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -88,6 +90,14 @@ def hyena_plan_create(ndim: int, shape, channels: int, order: int, io_dtype: int
     out = ctypes.c_void_p()
     arr = (ctypes.c_int64 * len(shape))(*shape)
     st = lib.hyena_plan_create(ctypes.byref(out), ndim, arr, channels, order, io_dtype, causal)
+    return st, out.value
+
+
+def hyena_plan_create_ex(ndim: int, shape, channels: int, order: int, io_dtype: int, causal: int, flags: int):
+    """Returns (status, plan handle as int or None)."""
+    out = ctypes.c_void_p()
+    arr = (ctypes.c_int64 * len(shape))(*shape)
+    st = lib.hyena_plan_create_ex(ctypes.byref(out), ndim, arr, channels, order, io_dtype, causal, flags)
     return st, out.value
 
 

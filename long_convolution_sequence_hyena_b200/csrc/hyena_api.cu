@@ -130,6 +130,12 @@ const char *hyena_status_string(hyena_status_t s) {
 
 hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *shape, int64_t channels, int order,
                                  hyena_dtype_t io_dtype, int causal) {
+    return hyena_plan_create_ex(out, ndim, shape, channels, order, io_dtype, causal, 0);
+}
+
+hyena_status_t hyena_plan_create_ex(hyena_plan_t *out, int ndim, const int64_t *shape, int64_t channels, int order,
+                                    hyena_dtype_t io_dtype, int causal, int flags) {
+    if (flags & ~HYENA_PLAN_RADIX3) return HYENA_ERR_INVALID_ARG;
     if (!out) return HYENA_ERR_INVALID_ARG;
     *out = nullptr;
     if (!shape || channels < 1 || order < 1 || order > HYENA_MAX_ORDER) return HYENA_ERR_INVALID_ARG;
@@ -149,12 +155,22 @@ hyena_status_t hyena_plan_create(hyena_plan_t *out, int ndim, const int64_t *sha
         if (p.L > HYENA_MAX_L_1D) return HYENA_ERR_UNSUPPORTED;
         p.M = next_pow2(2 * p.L);
         if (p.M < 32) p.M = 32;  // smallest FFT the kernels run (extra zero padding is exact)
+        if (flags & HYENA_PLAN_RADIX3) {
+            // the smallest M = 6 P >= 2L, when it is below the power of two
+            int64_t P = 16;
+            while (6 * P < 2 * p.L) P <<= 1;
+            if (6 * P < p.M && mr3_supported(P)) {
+                p.M = 6 * P;
+                p.P3 = P;
+            }
+        }
         p.MC = p.M / 2;
         p.path = p.M <= HYENA_MAX_M_CTA ? HYENA_PATH_CTA
                  : (staged_path_supported(p.MC) ? HYENA_PATH_STAGED : HYENA_PATH_CLUSTER);
+        if (p.P3) p.path = HYENA_PATH_CTA;
         // test and measurement override: HYENA_FORCE_PATH=cta|staged|cluster picks a
         // kernel family that can run this length, or the plan is UNSUPPORTED
-        if (const char *fp = std::getenv("HYENA_FORCE_PATH")) {
+        if (const char *fp = p.P3 ? nullptr : std::getenv("HYENA_FORCE_PATH")) {
             if (!std::strcmp(fp, "cta")) {
                 if (p.M > HYENA_MAX_M_CTA) return HYENA_ERR_UNSUPPORTED;
                 p.path = HYENA_PATH_CTA;
@@ -357,7 +373,8 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
             std::lock_guard<std::mutex> hold(*plan->spec_mu);
             e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, plan->spec_ws, st, cl.l);
         } else {
-            e = plan->path == HYENA_PATH_CTA
+            e = plan->P3 ? launch_spec_1d_mr3(src, src_stride, plan->L, Hc, nrows, plan->P3, tw, st)
+                : plan->path == HYENA_PATH_CTA
                     ? launch_spec_1d(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st)
                     : launch_spec_1d_cluster(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, st);
         }
@@ -471,6 +488,8 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
         if (!cl.ok) return HYENA_ERR_CUDA;
         e = launch_fwd_1d_staged(a, plan->MC, reinterpret_cast<float2 *>(workspace), plan->dtype, even,
                                  (cudaStream_t)stream, cl.l);
+    } else if (plan->P3) {
+        e = launch_fwd_1d_mr3(a, plan->P3, plan->dtype, even, (cudaStream_t)stream);
     } else if (plan->path == HYENA_PATH_CLUSTER)
         e = launch_fwd_1d_cluster(a, plan->MC, plan->dtype, even, (cudaStream_t)stream);
     else if (a.es == 1 && pair_path_supported(plan->MC, batch))

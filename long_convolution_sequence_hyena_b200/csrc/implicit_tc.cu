@@ -1,35 +1,41 @@
-// Implicit filter network with the head on the 5th-generation tensor cores
-// (tcgen05.mma, accumulators in tensor memory), for networks of width 64.
+// Implicit filter network on the 5th-generation tensor cores (tcgen05.mma,
+// accumulators in tensor memory), for networks of width 64.
 //
 // The network is the one of kernels_implicit.cuh ("Hyena — Long Convolutions
 // Math", "Implicit filters: an MLP over positions" and "The decay window";
 // "How HyenaND works", "1. An implicit filter"): positional features, two sine
-// layers of width 64, a linear head to N*D outputs, the window. The head is a
-// dense contraction o[p][j] = sum_k a2[p][k] W3[j][k] over every position p and
-// output j, and it holds almost all of the work (64 N D multiply-adds per
-// position against 64 (fin + 64) for the two hidden layers), so it runs on the
-// tensor cores; the hidden layers stay on the CUDA cores.
+// layers of width 64, a linear head to N*D outputs, the window. Two of its
+// three layers are dense contractions over every position p: the second sine
+// layer's pre-activation a1[p] W2^T (64 x 64) and the head a2[p] W3^T
+// (64 x N*D, almost all of the work); both run on the tensor cores. The
+// features and the first layer (1 + 2K or 2-3 inputs) stay on the CUDA cores.
 //
 // Precision: the filters must match an fp64 evaluation to fp32 accuracy, which
 // one TF32 product (10-bit mantissa) cannot. Each operand is split as
 // x = hi + lo with hi = x rounded to TF32 and lo = x - hi (exact in fp32), and
-// the head accumulates hi*hi + hi*lo + lo*hi in fp32 (the dropped lo*lo term
-// and the TF32 rounding of lo are about 2^-21 of the product).
+// each contraction accumulates hi*hi + hi*lo + lo*hi in fp32 (the dropped
+// lo*lo term and the TF32 rounding of lo are about 2^-21 of the product).
 //
-// One CTA (512 threads) per tile of 128 positions and one slice of the
-// outputs, one CTA per SM (about 160 KB of shared memory):
-//   1. thread (p, part) computes the features of position p, the 64 units of
-//      the first sine layer and units [16 part, 16 part + 16) of the second,
-//      and writes them, split, into the A tile (shared memory, the
-//      tensor core's K-major layout without swizzle: 8 x 16-byte core matrices);
-//   2. per slice of 128 outputs: the CTA converts W3's rows into the B tile;
-//      one thread issues 24 MMAs (M 128, N 128, K 8; eight K steps, three
-//      products) into one of two tensor-memory accumulators and commits them to
-//      an mbarrier; while they run, the 16 warps read the previous slice's
-//      accumulator (tcgen05.ld), add the bias, apply the window and store.
+// One CTA (256 threads, 8 warps) per tile of 128 positions and one slice of
+// the outputs, two CTAs per SM (about 100 KB of shared memory each):
+//   1. thread (p, part) forms the features of position p and units
+//      [16 part, 16 part + 16) of the first sine layer, and writes them, split,
+//      into the A tile (shared memory, the tensor core's K-major layout
+//      without swizzle: 8 x 16-byte core matrices); W2, split, is the B tile;
+//   2. one thread issues the 24 MMAs of the second layer (M 128, N 64, K 8:
+//      eight K steps, three products) into tensor memory; the warps read the
+//      pre-activations back (tcgen05.ld), add the bias, take the sine and
+//      write the split result over the A tile;
+//   3. per slice of 64 outputs: the CTA converts W3's rows into the B tile;
+//      one thread issues 24 MMAs (N 64) into one of two accumulators; while
+//      they run, the warps read the previous slice's accumulator, add the bias,
+//      apply the window (constants per output staged in shared memory) and
+//      store.
 // Every wait on the mbarrier is bounded: on a timeout the kernel records an
 // error in *err, skips the remaining MMAs and still frees its tensor memory.
 #include <cuda_runtime.h>
+
+#include <cstddef>
 
 #include "launch.h"
 
@@ -38,24 +44,28 @@ namespace hyena {
 namespace {
 
 constexpr int TP = 128;            // positions per tile (the MMA's M)
-constexpr int NT = 128;            // outputs per slice (the MMA's N)
+constexpr int NT = 64;             // outputs per slice (the MMA's N)
 constexpr int KW = 64;             // network width (the MMA's K over 8 steps)
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;
 constexpr int PARTS = THREADS / TP;      // threads per position (each takes KW / PARTS second-layer units)
 constexpr int LBO = 16 * 128;      // bytes between K-adjacent core matrices (16 row groups of 128 B)
 constexpr int SBO = 128;           // bytes between 8-row groups
-constexpr int TMEM_COLS = 2 * NT;      // two accumulators of 128 columns
+constexpr int TMEM_COLS = 256;         // two head accumulators of 64 columns, then the second layer's 64
+constexpr int L2COL = 2 * NT;          // first tensor-memory column of the second layer's accumulator
 constexpr int SLICE_OUT = 512;         // outputs per CTA (grid.y covers the rest)
 
 struct alignas(128) TcSmem {
     float a[2][TP * KW];           // A tile: hi, lo
-    float b[2][NT * KW];           // B tile: hi, lo
-    float w1t[IMP_MAXF][KW];       // first layer weights, transposed: [feature][unit]
-    float w2[KW][KW];              // second layer weights [unit][input]
+    float b[2][KW * KW];           // B tile: hi, lo (W2, then slices of W3: NT <= KW rows)
     float b1[KW], b2[KW];
+    float2 oc[NT];                 // per output of the slice: window exponent scale (log2 units), bias
     unsigned long long mbar;
     uint32_t tmem_base;
+    alignas(16) float w1t[1][KW];  // first layer weights, transposed: [feature][unit] (fin rows follow; read as float4)
 };
+static_assert(offsetof(TcSmem, w1t) % 16 == 0 && offsetof(TcSmem, a) % 16 == 0 && offsetof(TcSmem, b) % 16 == 0,
+              "16-byte accesses to the tiles and the first-layer weights");
+static_assert(NT <= KW, "the B tile holds W2 and the head slices");
 
 __device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -73,23 +83,38 @@ __device__ __forceinline__ int core_off(int row, int kc) { return kc * LBO + (ro
 // Shared-memory matrix descriptor (K-major, no swizzle): start address, leading
 // byte offset (between K-adjacent core matrices), stride byte offset (between
 // 8-row groups), descriptor version 1, layout type 0.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, int lbo = LBO) {
     uint64_t d = 0;
     d |= (uint64_t)((addr >> 4) & 0x3FFF);
-    d |= (uint64_t)((LBO >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
     d |= (uint64_t)((SBO >> 4) & 0x3FFF) << 32;
     d |= (uint64_t)1 << 46;
     return d;
 }
 
-// Instruction descriptor: fp32 accumulator, TF32 A and B, both K-major, N = NT, M = TP.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(TP >> 4) << 24);
+// Instruction descriptor: fp32 accumulator, TF32 A and B, both K-major, M = TP, N as given.
+constexpr uint32_t idesc_n(int n) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TP >> 4) << 24);
+}
 
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate));
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// The 24 MMAs of one contraction over K = 64: eight K steps (two core
+// matrices each), products hi*hi, hi*lo, lo*hi. Issued by one thread.
+__device__ __forceinline__ void mma_split_k64(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh, uint32_t bl,
+                                              int lbo_b, uint32_t idesc) {
+#pragma unroll
+    for (int ks = 0; ks < KW / 8; ++ks) {
+        const uint32_t ka = (uint32_t)(2 * ks * LBO), kb = (uint32_t)(2 * ks * lbo_b);
+        mma_tf32(d, smem_desc(ah + ka), smem_desc(bh + kb, lbo_b), idesc, ks > 0);
+        mma_tf32(d, smem_desc(ah + ka), smem_desc(bl + kb, lbo_b), idesc, 1);
+        mma_tf32(d, smem_desc(al + ka), smem_desc(bh + kb, lbo_b), idesc, 1);
+    }
 }
 
 __device__ __forceinline__ void mma_commit(unsigned long long *mbar) {
@@ -115,6 +140,23 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *mbar, uint32_t par
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Rows [o0, o0 + n) of a row-major [*][64] fp32 matrix as a split K-major B tile.
+__device__ __forceinline__ void load_b_tile(TcSmem &S, const float *__restrict__ Wm, int64_t o0, int n, int64_t oend,
+                                            int tid) {
+    unsigned char *bhi = reinterpret_cast<unsigned char *>(S.b[0]);
+    unsigned char *blo = reinterpret_cast<unsigned char *>(S.b[1]);
+    for (int i = tid; i < n * (KW / 4); i += THREADS) {
+        const int o = i % n, kc = i / n;          // consecutive threads: consecutive rows of one K chunk
+        const int64_t og = o0 + o;
+        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (og < oend) w = __ldg(reinterpret_cast<const float4 *>(Wm + og * KW) + kc);
+        const float4 h4 = make_float4(tf32_hi(w.x), tf32_hi(w.y), tf32_hi(w.z), tf32_hi(w.w));
+        const int off = kc * (n / 8) * SBO + (o >> 3) * SBO + (o & 7) * 16;   // K chunks n/8 row groups apart
+        *reinterpret_cast<float4 *>(bhi + off) = h4;
+        *reinterpret_cast<float4 *>(blo + off) = make_float4(w.x - h4.x, w.y - h4.y, w.z - h4.z, w.w - h4.w);
+    }
+}
+
 // 32 consecutive accumulator columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     uint32_t u[32];
@@ -131,20 +173,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const ImplicitArgs a, int *err) {
+__global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const ImplicitArgs a, int *err) {
     extern __shared__ float4 tc_smem4[];
     TcSmem &S = *reinterpret_cast<TcSmem *>(tc_smem4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int fin = a.ndim == 1 ? 1 + 2 * a.p.num_freqs : a.ndim;
     const int64_t p0 = (int64_t)blockIdx.x * TP;
 
-    // weights of the hidden layers, and the barrier and tensor memory
-    for (int i = tid; i < KW * fin; i += THREADS) S.w1t[i % fin][i / fin] = __ldg(a.p.W1 + i);
-    for (int i = tid; i < KW * KW; i += THREADS) S.w2[i / KW][i % KW] = __ldg(a.p.W2 + i);
+    // first-layer weights and biases, W2 as the B tile, the barrier and tensor memory
+    for (int i = tid; i < KW * fin; i += THREADS) S.w1t[0][(i % fin) * KW + i / fin] = __ldg(a.p.W1 + i);
     if (tid < KW) {
         S.b1[tid] = __ldg(a.p.b1 + tid);
         S.b2[tid] = __ldg(a.p.b2 + tid);
     }
+    load_b_tile(S, a.p.W2, 0, KW, KW, tid);
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(&S.mbar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -158,16 +200,28 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
+    unsigned char *ahi = reinterpret_cast<unsigned char *>(S.a[0]);
+    unsigned char *alo = reinterpret_cast<unsigned char *>(S.a[1]);
+    const uint32_t sah = saddr(S.a[0]), sal = saddr(S.a[1]), sbh = saddr(S.b[0]), sbl = saddr(S.b[1]);
+    bool ok = true;
+    uint32_t phase = 0;
+    auto wait_mma = [&]() {
+        if (ok && !mbar_wait(&S.mbar, phase)) {
+            ok = false;
+            atomicExch(err, 1);
+        }
+        phase ^= 1;
+        tc_fence_after();
+    };
 
-    // 1. features and hidden layers of position p; this thread writes units [16 part, 16 part + 16).
-    // The features are formed one at a time and folded into all 64 first-layer sums at once.
+    // 1. features and first-layer units [16 part, 16 part + 16) of position p, split into the A tile
     {
         const int p = tid & (TP - 1), part = tid / TP;
         const int64_t pos = p0 + p;
         const bool in = pos < a.npos;
-        float a1[KW];
+        float a1[KW / PARTS];
 #pragma unroll
-        for (int j = 0; j < KW; ++j) a1[j] = 0.f;
+        for (int j = 0; j < KW / PARTS; ++j) a1[j] = 0.f;
 #pragma unroll 1
         for (int f = 0; f < fin; ++f) {
             float fv = 0.f;
@@ -194,9 +248,9 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
                                           : (float)((double)(ix - a.W) / (double)a.W));
                 }
             }
-            const float4 *wrow = reinterpret_cast<const float4 *>(S.w1t[f]);
+            const float4 *wrow = reinterpret_cast<const float4 *>(S.w1t[0] + f * KW + (KW / PARTS) * part);
 #pragma unroll
-            for (int j4 = 0; j4 < KW / 4; ++j4) {
+            for (int j4 = 0; j4 < KW / PARTS / 4; ++j4) {
                 const float4 w = wrow[j4];
                 a1[4 * j4] = fmaf(w.x, fv, a1[4 * j4]);
                 a1[4 * j4 + 1] = fmaf(w.y, fv, a1[4 * j4 + 1]);
@@ -205,27 +259,45 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
             }
         }
 #pragma unroll
-        for (int j = 0; j < KW; ++j) a1[j] = sinf(a.p.omega0 * (a1[j] + S.b1[j]));
-        unsigned char *ahi = reinterpret_cast<unsigned char *>(S.a[0]);
-        unsigned char *alo = reinterpret_cast<unsigned char *>(S.a[1]);
-#pragma unroll 1
         for (int c = 0; c < KW / PARTS / 4; ++c) {   // 4 units per 16-byte core-matrix row
             const int kc = (KW / PARTS / 4) * part + c;
             float hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int j = 4 * kc + u;
-                const float4 *wrow = reinterpret_cast<const float4 *>(S.w2[j]);
-                float acc = 0.f;
+                const float v = in ? sinf(a.p.omega0 * (a1[4 * c + u] + S.b1[4 * kc + u])) : 0.f;
+                hi[u] = tf32_hi(v);
+                lo[u] = v - hi[u];
+            }
+            const int off = core_off(p, kc);
+            *reinterpret_cast<float4 *>(ahi + off) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<float4 *>(alo + off) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tensor core sees the tiles
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // 2. second layer on the tensor cores: pre-activations of 64 units -> tensor memory
+    if (tid == 0) {
+        mma_split_k64(tmem + L2COL, sah, sal, sbh, sbl, (KW / 8) * SBO, idesc_n(KW));
+        mma_commit(&S.mbar);
+    }
+    wait_mma();
+    {
+        constexpr int UPW = KW / (THREADS / 128);   // units per warp: 32
+        const int q = warp & 3, cq = warp >> 2;      // lane quarter (positions), unit group
+        const int p = 32 * q + lane;
+        float r[UPW];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(L2COL + UPW * cq), r);
+        const bool in = p0 + p < a.npos;
 #pragma unroll
-                for (int k4 = 0; k4 < KW / 4; ++k4) {
-                    const float4 w = wrow[k4];
-                    acc = fmaf(w.x, a1[4 * k4], acc);
-                    acc = fmaf(w.y, a1[4 * k4 + 1], acc);
-                    acc = fmaf(w.z, a1[4 * k4 + 2], acc);
-                    acc = fmaf(w.w, a1[4 * k4 + 3], acc);
-                }
-                const float v = in ? sinf(a.p.omega_hidden * (acc + S.b2[j])) : 0.f;
+        for (int c = 0; c < UPW / 4; ++c) {
+            const int kc = (UPW / 4) * cq + c;
+            float hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float v = in ? sinf(a.p.omega_hidden * (r[4 * c + u] + S.b2[4 * kc + u])) : 0.f;
                 hi[u] = tf32_hi(v);
                 lo[u] = v - hi[u];
             }
@@ -235,14 +307,14 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
         }
     }
 
-    // 2. head slices
+    // 3. head slices
     const int64_t o_begin = (int64_t)blockIdx.y * SLICE_OUT;
     const int64_t o_end = o_begin + SLICE_OUT < a.nout ? o_begin + SLICE_OUT : a.nout;
     const int nslices = (int)((o_end - o_begin + NT - 1) / NT);
     const int q = warp & 3, cq = warp >> 2;            // TMEM lane quarter, column quarter
     const int prow = 32 * q + lane;                    // this thread's position in the epilogue
     const int64_t ppos = p0 + prow;
-    float we = 0.f;                                    // window exponent argument: t (1D) or |p|^2 (2D)
+    float we = 0.f;                                    // window exponent argument: t (1D) or |p|^2 (2D, 3D)
     int64_t poff = ppos;
     if (a.ndim == 1) {
         we = (float)ppos;
@@ -259,64 +331,47 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
         const float py = (float)((double)(iy - a.H) / (double)a.H), px = (float)((double)(ix - a.W) / (double)a.W);
         we = pz * pz + py * py + px * px;
     }
-    bool ok = true;
-    uint32_t phase = 0;
+    static_assert(NT / (THREADS / 128) == 32, "each warp reads 32 accumulator columns");
     auto epilogue = [&](int s) {
         float r[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((s & 1) * NT + 32 * cq), r);
         if (ppos >= a.npos) return;
-#pragma unroll 4
+        const int64_t ob = o_begin + (int64_t)s * NT + 32 * cq;
+        float *dst = a.out + ob * a.out_stride + poff;
+#pragma unroll 8
         for (int c = 0; c < 32; ++c) {
-            const int64_t o = o_begin + (int64_t)s * NT + 32 * cq + c;
-            if (o >= o_end) break;
-            const float wp = __ldg(a.p.window + o);
-            const float esc = a.ndim == 1 ? -wp : -1.f / (2.f * wp * wp);
-            a.out[o * a.out_stride + poff] = expf(esc * we) * (r[c] + __ldg(a.p.b3 + o));
+            if (ob + c >= o_end) break;
+            const float2 k = S.oc[32 * cq + c];   // (window exponent scale in log2 units, bias)
+            *dst = exp2f(k.x * we) * (r[c] + k.y);
+            dst += a.out_stride;
         }
     };
 #pragma unroll 1
     for (int s = 0; s < nslices; ++s) {
-        // B tile of slice s: rows o of W3 as 16-byte core-matrix rows, split
-        {
-            unsigned char *bhi = reinterpret_cast<unsigned char *>(S.b[0]);
-            unsigned char *blo = reinterpret_cast<unsigned char *>(S.b[1]);
-            const int o = tid & (NT - 1);
-            const int64_t og = o_begin + (int64_t)s * NT + o;
-#pragma unroll
-            for (int i = 0; i < KW / 4 / (THREADS / NT); ++i) {
-                const int kc = tid / NT + (THREADS / NT) * i;
-                float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (og < o_end) w = __ldg(reinterpret_cast<const float4 *>(a.p.W3 + og * KW) + kc);
-                const float4 h4 = make_float4(tf32_hi(w.x), tf32_hi(w.y), tf32_hi(w.z), tf32_hi(w.w));
-                const int off = core_off(o, kc);
-                *reinterpret_cast<float4 *>(bhi + off) = h4;
-                *reinterpret_cast<float4 *>(blo + off) = make_float4(w.x - h4.x, w.y - h4.y, w.z - h4.z, w.w - h4.w);
-            }
+        // W3 rows of slice s as the B tile; their window scales and biases. The
+        // epilogue of slice s - 1 still reads S.oc: it runs after the barrier below.
+        const int64_t os = o_begin + (int64_t)s * NT;
+        load_b_tile(S, a.p.W3, os, NT, o_end, tid);
+        float2 oc_new = make_float2(0.f, 0.f);
+        if (tid < NT && os + tid < o_end) {
+            const float wp = __ldg(a.p.window + os + tid);
+            // exp(-alpha t) (1D) or exp(-|p|^2 / (2 sigma^2)) (2D, 3D), as 2^(scale * arg)
+            const float esc = a.ndim == 1 ? -wp : -1.f / (2.f * wp * wp);
+            oc_new = make_float2(esc * 1.4426950408889634f, __ldg(a.p.b3 + os + tid));
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the tensor core sees the tiles
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0 && ok) {
-            const uint32_t d = tmem + (uint32_t)((s & 1) * NT);
-            const uint32_t ah = saddr(S.a[0]), al = saddr(S.a[1]), bh = saddr(S.b[0]), bl = saddr(S.b[1]);
-#pragma unroll
-            for (int ks = 0; ks < KW / 8; ++ks) {   // K step of 8 = two core matrices along K
-                const uint32_t ko = (uint32_t)(2 * ks * LBO);
-                mma_tf32(d, smem_desc(ah + ko), smem_desc(bh + ko), ks > 0);
-                mma_tf32(d, smem_desc(ah + ko), smem_desc(bl + ko), 1);
-                mma_tf32(d, smem_desc(al + ko), smem_desc(bh + ko), 1);
-            }
+            mma_split_k64(tmem + (uint32_t)((s & 1) * NT), sah, sal, sbh, sbl, (NT / 8) * SBO, idesc_n(NT));
             mma_commit(&S.mbar);
         }
         if (s > 0) epilogue(s - 1);   // overlaps the MMAs of slice s
-        if (ok && !mbar_wait(&S.mbar, phase)) {
-            ok = false;
-            atomicExch(err, 1);
-        }
-        phase ^= 1;
-        tc_fence_after();
-        __syncthreads();   // slice s complete (or abandoned) before the B tile is rewritten
+        __syncthreads();              // every read of S.oc for slice s - 1 done
+        if (tid < NT) S.oc[tid] = oc_new;
+        wait_mma();
+        __syncthreads();              // slice s complete (or abandoned) and S.oc updated
     }
     if (nslices > 0 && ok) epilogue(nslices - 1);
     tc_fence_before();
@@ -328,10 +383,10 @@ __global__ void __launch_bounds__(THREADS, 1) hyena_implicit_tc_kernel(const Imp
 
 bool implicit_tc_supported(const ImplicitArgs &a) { return a.p.width == KW; }
 
-size_t implicit_tc_smem_bytes() { return sizeof(TcSmem) + 128; }
+size_t implicit_tc_smem_bytes(int fin) { return sizeof(TcSmem) + (size_t)(fin - 1) * KW * sizeof(float) + 128; }
 
 cudaError_t launch_implicit_tc(const ImplicitArgs &a, int *err, cudaStream_t st) {
-    const int sm = (int)implicit_tc_smem_bytes();
+    const int sm = (int)implicit_tc_smem_bytes(a.ndim == 1 ? 1 + 2 * a.p.num_freqs : a.ndim);
     cudaError_t e = cudaFuncSetAttribute(hyena_implicit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.npos + TP - 1) / TP), (unsigned)((a.nout + SLICE_OUT - 1) / SLICE_OUT));

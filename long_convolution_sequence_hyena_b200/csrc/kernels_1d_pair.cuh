@@ -293,3 +293,4 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
 }
 
 }  // namespace hyena
+

@@ -13,6 +13,11 @@ namespace hyena {
 cudaError_t launch_fwd_1d(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);
 cudaError_t launch_spec_1d(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t MC,
                            const c32 *tw, cudaStream_t st);
+// 1D, padded length M = 6 P (MC = 3 P, P a power of two, 16..4096): one row per thread group
+bool mr3_supported(int64_t P);
+cudaError_t launch_fwd_1d_mr3(const Fwd1dArgs &a, int64_t P, hyena_dtype_t dt, bool even, cudaStream_t st);
+cudaError_t launch_spec_1d_mr3(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows, int64_t P,
+                               const c32 *tw, cudaStream_t st);
 // 1D, two rows of one channel per thread group (B even, MC <= 8192)
 bool pair_path_supported(int64_t MC, int64_t B);
 cudaError_t launch_fwd_1d_pair(const Fwd1dArgs &a, int64_t MC, hyena_dtype_t dt, bool even, cudaStream_t st);

@@ -23,6 +23,7 @@ struct hyena_plan_s {
     int64_t L = 0;               // sequence length
     int64_t M = 0;               // padded real FFT length, next_pow2(2L) (at least 32)
     int64_t MC = 0;              // M / 2: length of the packed complex FFT
+    int64_t P3 = 0;              // M = 6 P3 (a radix-3 length, HYENA_PLAN_RADIX3), else 0
     // 2D geometry
     int64_t Hh = 0, Ww = 0;      // grid extents (the transform is 2H x 2W)
     int64_t Dd = 0;              // 3D: depth (the transform is 2Dz x 2H x 2W)

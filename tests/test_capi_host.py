@@ -109,3 +109,8 @@ def test_header_compiles_as_c_and_links(capi, tmp_path):
                            str(src), "-o", str(exe), "-L", pkg, "-lhyena", "-Wl,-rpath," + pkg])
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0 and out.stdout.strip() == "OK", (out.returncode, out.stdout, out.stderr)
+
+
+def test_plan_create_ex_rejects_unknown_flags(capi):
+    st, h = capi.hyena_plan_create_ex(1, [3000], 4, 2, capi.HYENA_F32, 1, 0x10)
+    assert st == capi.HYENA_ERR_INVALID_ARG and h is None
