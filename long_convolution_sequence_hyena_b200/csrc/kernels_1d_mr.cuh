@@ -36,6 +36,8 @@ struct MR3 {
     static constexpr int RPC = GT >= 96 ? 1 : 96 / GT;    // rows per CTA
     static constexpr int THREADS = RPC * GT;
     static constexpr int SMEM_FLOATS = 2 * MC;            // per row: the row (re, im planes) or three FFT exchanges
+    // resident CTAs per SM the register budget is sized for (about 170 registers per thread)
+    static constexpr int MINB = THREADS >= 384 ? 1 : 384 / THREADS;
     static_assert(P >= 16 && (P & (P - 1)) == 0, "P is a power of two of at least 16");
     static_assert(THREADS <= 1024, "P up to 4096");
 };
@@ -101,7 +103,7 @@ __device__ __forceinline__ void fft_mr3(c32 (&v)[MR3<P>::E], float *buf, int s, 
 }
 
 template <int P, typename IO, bool EVEN>
-__global__ void __launch_bounds__(MR3<P>::THREADS) hyena_fwd_1d_mr3(const Fwd1dArgs a) {
+__global__ void __launch_bounds__(MR3<P>::THREADS, MR3<P>::MINB) hyena_fwd_1d_mr3(const Fwd1dArgs a) {
     using G = MR3<P>;
     constexpr int E = G::E, T = G::T, MC = G::MC, RPC = G::RPC;
     extern __shared__ float smem[];
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(MR3<P>::THREADS) hyena_fwd_1d_mr3(const Fwd1dA
 
 // Filter spectra for M = 6 P: Hout[o, k] = sum_t h[o, t] e^{-2 pi i k t / M}, k in [0, MC].
 template <int P>
-__global__ void __launch_bounds__(MR3<P>::THREADS)
+__global__ void __launch_bounds__(MR3<P>::THREADS, MR3<P>::MINB)
     hyena_spectrum_1d_mr3(const float *h, int64_t h_stride, int64_t L, c32 *Hout, int64_t nrows,
                           const c32 *__restrict__ tw) {
     using G = MR3<P>;
