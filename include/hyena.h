@@ -154,6 +154,15 @@ HYENA_API hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout);
 HYENA_API hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear);
 
 /*
+ * The number of kernels this library has enqueued in the calling process
+ * since it was loaded, over all plans, threads and streams (a launch is
+ * counted when it is enqueued, whether or not it has run yet). Reading it
+ * before and after a call gives the kernels that call launched; it never
+ * touches the device. *count must not be NULL (HYENA_ERR_INVALID_ARG).
+ */
+HYENA_API hyena_status_t hyena_launch_count(int64_t *count);
+
+/*
  * hyena_plan_create with options. flags is 0 (the same plan as
  * hyena_plan_create) or HYENA_PLAN_RADIX3: a 1D plan then pads to the smallest
  * M = 6 * 2^j >= 2L when that is below the power of two ("Hyena — Long

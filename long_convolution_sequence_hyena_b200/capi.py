@@ -34,6 +34,7 @@ EXPORTED = (
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
     "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors", "hyena_plan_create_ex",
+    "hyena_launch_count",
 )
 
 
@@ -70,6 +71,7 @@ def _load():
         "hyena_plan_set_layout": ([p, i32], i32),
         "hyena_plan_device_errors": ([p, ctypes.POINTER(i32), i32], i32),
         "hyena_plan_create_ex": ([ctypes.POINTER(p), i32, ctypes.POINTER(i64), i64, i32, i32, i32, i32], i32),
+        "hyena_launch_count": ([ctypes.POINTER(i64)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -114,6 +116,15 @@ def hyena_plan_device_errors(plan, clear: bool = False):
     f = ctypes.c_int()
     st = lib.hyena_plan_device_errors(plan, ctypes.byref(f), 1 if clear else 0)
     return st, f.value
+
+
+def hyena_launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    n = ctypes.c_int64()
+    st = lib.hyena_launch_count(ctypes.byref(n))
+    if st != HYENA_OK:
+        raise RuntimeError("hyena_launch_count: %d" % st)
+    return n.value
 
 
 def hyena_plan_info(plan):

@@ -1,6 +1,7 @@
 #pragma once
 // Cluster geometries and the cluster launch helper.
 #include "kernels_1d_cluster.cuh"
+#include "launch_count.h"
 
 namespace hyena {
 
@@ -31,7 +32,7 @@ inline cudaError_t launch_cluster(Kern kern, int64_t units, cudaStream_t st, Arg
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, args...);
     if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace hyena

@@ -27,7 +27,7 @@ cudaError_t launch_fwd_1d_t(const Fwd1dArgs &a, cudaStream_t st) {
     }
     const int64_t grid = (a.rows + RPC - 1) / RPC;
     kern<<<(unsigned)grid, RPC * (MC / E), sm, st>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 template <int MC>
@@ -50,7 +50,7 @@ cudaError_t launch_spec_1d_mc(const float *h, int64_t h_stride, int64_t L, c32 *
     }
     const int64_t grid = (nrows + RPC - 1) / RPC;
     kern<<<(unsigned)grid, RPC * (MC / E), sm, st>>>(h, h_stride, L, Hout, nrows, tw);
-    return cudaGetLastError();
+    return launched();
 }
 
 #define HY_MC_SWITCH(MCV, CALL)     \

@@ -18,7 +18,7 @@ cudaError_t launch_t(const Fwd1dArgs &a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
     }
     kern<<<(unsigned)((a.rows + G::RPC - 1) / G::RPC), G::THREADS, sm, st>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 template <int P>
@@ -39,7 +39,7 @@ cudaError_t launch_spec_p(const float *h, int64_t hs, int64_t L, c32 *Hout, int6
     }
     hyena_spectrum_1d_mr3<P><<<(unsigned)((nrows + G::RPC - 1) / G::RPC), G::THREADS, sm, st>>>(h, hs, L, Hout,
                                                                                               nrows, tw);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace

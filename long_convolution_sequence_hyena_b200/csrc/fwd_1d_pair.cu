@@ -24,7 +24,7 @@ cudaError_t launch_fwd_1d_pair_t(const Fwd1dArgs &a, cudaStream_t st) {
     const int64_t npairs = a.rows / 2;
     const int64_t grid = (npairs + PPC - 1) / PPC;
     kern<<<(unsigned)grid, pair_threads(MC, E), sm, st>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 template <int MC>

@@ -72,6 +72,7 @@ cudaError_t launch_staged_io(const Fwd1dArgs &f, float2 *ws, int64_t chunk, cons
             else
                 hyena_staged_cols_x2<G, IO, EVEN, 2><<<cgrid, G::CT, G::CSMEM, st>>>(a, nr);
         }
+        note_launch(2 * f.order + 1);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -110,6 +111,7 @@ cudaError_t launch_spec_staged_g(const Spec1dArgs &base, int64_t nrows, const cu
         const cudaStream_t s = lanes[c % nst];
         hyena_staged_spec_cols_x2<G><<<(unsigned)(pairs * G::CGROUPS), G::CT, G::CSMEM, s>>>(a);
         hyena_staged_spec_rows_x2<G><<<(unsigned)(pairs * G::RGROUPS), G::RT, G::RSMEM, s>>>(a);
+        note_launch(2);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

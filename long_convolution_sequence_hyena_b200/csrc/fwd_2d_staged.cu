@@ -42,6 +42,7 @@ cudaError_t launch_staged2d_io(const Fwd2dArgs &f, float2 *ws, int64_t chunk, co
             else
                 hyena_staged2d_cols<G, IO, 2, GATED><<<cgrid, G::CT, G::CSMEM, st>>>(a);
         }
+        note_launch(2 * f.order + 1);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -77,6 +78,7 @@ cudaError_t launch_spec_2d_staged(const float *K, int64_t rs, int64_t cs, c32 *K
             const cudaStream_t s = lanes[c % nst];
             hyena_staged2d_spec_cols<G><<<(unsigned)(a.nk * (G::M2 / G::NCOL)), G::CT, G::CSMEM, s>>>(a);
             hyena_staged2d_spec_rows_x2<G><<<(unsigned)((a.nk + 1) / 2 * G::RGROUPS), G::RT, G::RSMEM, s>>>(a);
+            note_launch(2);
             const cudaError_t le = cudaGetLastError();
             if (le != cudaSuccess) return le;
         }

@@ -25,7 +25,7 @@ cudaError_t launch_x(const Fwd3dArgs &a, cudaStream_t st) {
     case LX:                                                                                                \
         hyena_3d_x<LX, IO, MODE, G><<<(unsigned)((rows + Stage3<LX>::NSEQ - 1) / Stage3<LX>::NSEQ),        \
                                       S3_THREADS, 0, st>>>(a);                                              \
-        return cudaGetLastError();
+        return launched();
         X_CASE(32) X_CASE(64) X_CASE(128)
 #undef X_CASE
         default: return cudaErrorInvalidValue;
@@ -40,7 +40,7 @@ cudaError_t launch_y(const Fwd3dArgs &a, cudaStream_t st) {
     case LY:                                                                                                \
         hyena_3d_y<LY, DIR><<<(unsigned)((cols + Stage3<LY>::NSEQ - 1) / Stage3<LY>::NSEQ), S3_THREADS, 0,  \
                               st>>>(a);                                                                     \
-        return cudaGetLastError();
+        return launched();
         Y_CASE(32) Y_CASE(64) Y_CASE(128)
 #undef Y_CASE
         default: return cudaErrorInvalidValue;
@@ -53,7 +53,7 @@ cudaError_t launch_z(const Fwd3dArgs &a, cudaStream_t st) {
 #define Z_CASE(LZ)                                                                                          \
     case LZ:                                                                                                \
         hyena_3d_z<LZ><<<(unsigned)((cols + Stage3<LZ>::NSEQ - 1) / Stage3<LZ>::NSEQ), S3_THREADS, 0, st>>>(a); \
-        return cudaGetLastError();
+        return launched();
         Z_CASE(32) Z_CASE(64) Z_CASE(128)
 #undef Z_CASE
         default: return cudaErrorInvalidValue;
@@ -109,19 +109,19 @@ cudaError_t launch_spec_3d(const float *K, int64_t cs, c32 *Kout, int64_t n, int
     a.W = W;
     const int64_t rows = n * 2 * Dz * 2 * H, ycols = n * 2 * Dz * 2 * W, zcols = n * 2 * H * 2 * W;
     switch (2 * W) {
-#define SX(LX) case LX: hyena_3d_spec_x<LX><<<(unsigned)((rows + Stage3<LX>::NSEQ - 1) / Stage3<LX>::NSEQ), S3_THREADS, 0, st>>>(a); break;
+#define SX(LX) case LX: hyena_3d_spec_x<LX><<<(unsigned)((rows + Stage3<LX>::NSEQ - 1) / Stage3<LX>::NSEQ), S3_THREADS, 0, st>>>(a); note_launch(); break;
         SX(32) SX(64) SX(128)
 #undef SX
         default: return cudaErrorInvalidValue;
     }
     switch (2 * H) {
-#define SY(LY) case LY: hyena_3d_spec_col<LY, 1><<<(unsigned)((ycols + Stage3<LY>::NSEQ - 1) / Stage3<LY>::NSEQ), S3_THREADS, 0, st>>>(a); break;
+#define SY(LY) case LY: hyena_3d_spec_col<LY, 1><<<(unsigned)((ycols + Stage3<LY>::NSEQ - 1) / Stage3<LY>::NSEQ), S3_THREADS, 0, st>>>(a); note_launch(); break;
         SY(32) SY(64) SY(128)
 #undef SY
         default: return cudaErrorInvalidValue;
     }
     switch (2 * Dz) {
-#define SZ(LZ) case LZ: hyena_3d_spec_col<LZ, 2><<<(unsigned)((zcols + Stage3<LZ>::NSEQ - 1) / Stage3<LZ>::NSEQ), S3_THREADS, 0, st>>>(a); break;
+#define SZ(LZ) case LZ: hyena_3d_spec_col<LZ, 2><<<(unsigned)((zcols + Stage3<LZ>::NSEQ - 1) / Stage3<LZ>::NSEQ), S3_THREADS, 0, st>>>(a); note_launch(); break;
         SZ(32) SZ(64) SZ(128)
 #undef SZ
         default: return cudaErrorInvalidValue;

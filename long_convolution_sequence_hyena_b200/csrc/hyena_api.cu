@@ -3,6 +3,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -112,6 +113,11 @@ ImplicitArgs implicit_args(const hyena_plan_s *p, const hyena_implicit_params_t 
 }
 
 }  // namespace
+
+namespace hyena {
+static std::atomic<int64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace hyena
 
 extern "C" {
 
@@ -300,6 +306,12 @@ hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear
     if (clear && cudaMemset(plan->dev_err, 0, sizeof(h)) != cudaSuccess) return HYENA_ERR_CUDA;
     if (flags) flags[0] = h[0];
     return h[0] ? HYENA_ERR_CUDA : HYENA_OK;
+}
+
+hyena_status_t hyena_launch_count(int64_t *count) {
+    if (!count) return HYENA_ERR_INVALID_ARG;
+    *count = hyena::g_launches.load(std::memory_order_relaxed);
+    return HYENA_OK;
 }
 
 hyena_status_t hyena_plan_info(hyena_plan_t plan, int64_t *fft_len, int64_t *spectrum_elems, int *path) {

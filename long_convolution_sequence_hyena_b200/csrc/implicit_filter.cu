@@ -147,7 +147,7 @@ cudaError_t launch_implicit(const ImplicitArgs &a, int *err, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.npos + IMP_TP - 1) / IMP_TP), (unsigned)((a.nout + IMP_OSPLIT - 1) / IMP_OSPLIT));
     hyena_implicit_filter_kernel<<<grid, IMP_THREADS, sm, st>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace hyena

@@ -391,7 +391,7 @@ cudaError_t launch_implicit_tc(const ImplicitArgs &a, int *err, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.npos + TP - 1) / TP), (unsigned)((a.nout + SLICE_OUT - 1) / SLICE_OUT));
     hyena_implicit_tc_kernel<<<grid, THREADS, sm, st>>>(a, err);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace hyena

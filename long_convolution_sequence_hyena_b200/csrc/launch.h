@@ -6,6 +6,7 @@
 #include "hyena.h"
 #include "kernels_1d.cuh"
 #include "kernels_implicit.cuh"
+#include "launch_count.h"
 
 namespace hyena {
 

@@ -88,6 +88,9 @@ int main(void) {
     if (hyena_forward_host(NULL, 1, 0, gates, 0, NULL, 0, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 6;
     if (hyena_forward_no_alloc(NULL, 1, 0, gates, 0, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 7;
     if (hyena_filter_spectrum(NULL, NULL, NULL, NULL, NULL) != HYENA_ERR_INVALID_ARG) bad = 8;
+    int64_t launches = -1;
+    if (hyena_launch_count(NULL) != HYENA_ERR_INVALID_ARG) bad = 9;
+    if (hyena_launch_count(&launches) != HYENA_OK || launches != 0) bad = 10;
     printf("%s\n", bad ? "FAIL" : "OK");
     return bad;
 }
@@ -114,3 +117,13 @@ def test_header_compiles_as_c_and_links(capi, tmp_path):
 def test_plan_create_ex_rejects_unknown_flags(capi):
     st, h = capi.hyena_plan_create_ex(1, [3000], 4, 2, capi.HYENA_F32, 1, 0x10)
     assert st == capi.HYENA_ERR_INVALID_ARG and h is None
+
+
+def test_launch_count_without_a_gpu(capi):
+    """The launch counter reads without touching the device; calls rejected before
+    any launch leave it unchanged."""
+    n0 = capi.hyena_launch_count()
+    assert n0 >= 0
+    assert capi.hyena_forward(None, 1, 16, [16], 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_launch_count() == n0
+    assert capi.lib.hyena_launch_count(None) == capi.HYENA_ERR_INVALID_ARG
