@@ -340,7 +340,13 @@ HYENA_API hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batch
  *
  * Stages are whole batch elements: as many as make about 8 MiB of input, at
  * most B; in 1D rounded up to an even count, so that two rows of one channel
- * share a thread group. With B = 1 there is one stage and nothing overlaps. The copies run on two streams the call creates
+ * share a thread group. On 1D plans of the staged and cluster paths (M of
+ * 65536 and more) in the [B, D, L] layout whose batch element holds more than
+ * 16 MiB of input, a stage is instead a range of channels of one batch
+ * element: about 16 MiB of input, a whole number of the staged path's chunks
+ * (32 rows at M = 131072), so that even B = 1 overlaps its copies with the
+ * forward. Each stage's rows equal hyena_forward's bit for bit either way.
+ * The copies run on two streams the call creates
  * and releases (cudaStreamDestroy returns at once, and the streams are freed
  * when their work is done). Every copy waits for the work enqueued on
  * `stream` before the call, and work enqueued on `stream` after the call

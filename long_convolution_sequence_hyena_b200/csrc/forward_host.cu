@@ -1,11 +1,15 @@
 // Forward on host-resident activations: the batch is cut into stages of whole
-// batch elements; a stage's inputs are copied to one of two device stage
-// buffers on a copy-in stream, the stage runs hyena_forward on the caller's
-// stream, and its output is copied back on a copy-out stream. Two buffers let
-// the copy-in of stage c+1, the forward of stage c and the copy-out of stage
-// c-1 overlap (host-to-device and device-to-host copies use separate copy
-// engines). The streams and events belong to the call, so that calls on one
-// plan from several threads stay independent.
+// batch elements, or, for long 1D rows in the [B, D, L] layout, of channel
+// ranges of one batch element (the operator is depthwise, so a channel range
+// is an independent forward; one batch element of such rows holds hundreds of
+// MB, and a stage per element would leave nothing to overlap at batch 1). A
+// stage's inputs are copied to one of two device stage buffers on a copy-in
+// stream, the stage runs the forward on the caller's stream, and its output
+// is copied back on a copy-out stream. Two buffers let the copy-in of stage
+// c+1, the forward of stage c and the copy-out of stage c-1 overlap
+// (host-to-device and device-to-host copies use separate copy engines). The
+// streams and events belong to the call, so that calls on one plan from
+// several threads stay independent.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -23,15 +27,33 @@ struct HostStages {
     int64_t per_b = 0;   // elements of one batch element: D * L (1D) or C * H * W (2D)
     size_t io = 0;       // bytes per element
     int64_t bc = 0;      // batch elements per stage
+    int64_t dc = 0;      // channels per stage: D (whole batch elements), or fewer
+                         // when every batch element is split into channel ranges (bc = 1)
     size_t tensor = 0;   // bytes of one stage tensor, rounded up to 256
-    size_t fwd_ws = 0;   // hyena_forward's workspace for one stage
+    size_t fwd_ws = 0;   // the forward's workspace for one stage
 };
 
 HostStages host_stages(hyena_plan_s *p, int64_t batch) {
     HostStages s;
     s.per_b = p->D * (p->ndim == 1 ? p->L : p->Hh * p->Ww);
     s.io = p->dtype == HYENA_F32 ? 4 : 2;
+    s.dc = p->D;
     const size_t in_per_b = (size_t)(p->order + 1) * (size_t)s.per_b * s.io;
+    // long rows: stages of about 16 MB of inputs, in whole chunks of the staged path
+    const size_t split_target = (size_t)16 << 20;
+    if (p->ndim == 1 && p->layout == HYENA_LAYOUT_BDL &&
+        (p->path == HYENA_PATH_STAGED || p->path == HYENA_PATH_CLUSTER) && in_per_b > split_target) {
+        const size_t in_per_ch = (size_t)(p->order + 1) * (size_t)p->L * s.io;
+        const int64_t q = p->path == HYENA_PATH_STAGED ? hyena::staged_chunk_rows(p->MC) : 1;
+        int64_t dc = (int64_t)(split_target / in_per_ch) / q * q;
+        if (dc < q) dc = q;
+        if (dc > p->D) dc = p->D;
+        s.bc = 1;
+        s.dc = dc;
+        s.tensor = align256((size_t)dc * (size_t)p->L * s.io);
+        s.fwd_ws = align256(hyena::workspace_bytes_1d(p, dc));
+        return s;
+    }
     const size_t target = (size_t)8 << 20;
     int64_t bc = (int64_t)((target + in_per_b - 1) / in_per_b);
     if (bc < 1) bc = 1;
@@ -128,12 +150,24 @@ hyena_status_t hyena_forward_host(hyena_plan_t plan, int64_t batch, const void *
     void *fwd_ws = s.fwd_ws ? base + 2 * (size_t)(N + 2) * s.tensor : nullptr;
     const char *vh = static_cast<const char *>(v_host);
     char *yh = static_cast<char *>(y_host);
-    const int64_t nstage = (batch + s.bc - 1) / s.bc;
+    const bool split = s.dc < plan->D;
+    const int64_t nsplit = split ? (plan->D + s.dc - 1) / s.dc : 1;   // channel ranges per batch element
+    const int64_t nstage = split ? batch * nsplit : (batch + s.bc - 1) / s.bc;
     for (int64_t c = 0; c < nstage && status == HYENA_OK; ++c) {
         const int k = (int)(c & 1);
-        const int64_t b0 = c * s.bc;
-        const int64_t nb = (batch - b0) < s.bc ? (batch - b0) : s.bc;
-        const size_t bytes = (size_t)nb * (size_t)s.per_b * s.io, off = (size_t)b0 * (size_t)s.per_b * s.io;
+        int64_t b0, nb, d0 = 0, dcount = plan->D;
+        if (split) {
+            b0 = c / nsplit;
+            nb = 1;
+            d0 = (c % nsplit) * s.dc;
+            dcount = (plan->D - d0) < s.dc ? (plan->D - d0) : s.dc;
+        } else {
+            b0 = c * s.bc;
+            nb = (batch - b0) < s.bc ? (batch - b0) : s.bc;
+        }
+        const size_t row_elems = (size_t)(s.per_b / plan->D);   // L (1D) or H W (2D)
+        const size_t bytes = (size_t)nb * (size_t)dcount * row_elems * s.io;
+        const size_t off = ((size_t)b0 * (size_t)plan->D + (size_t)d0) * row_elems * s.io;
         // stage buffer k: v, x^1..x^N, y
         char *buf = base + (size_t)k * (size_t)(N + 2) * s.tensor;
         const void *gdev[HYENA_MAX_ORDER];
@@ -154,7 +188,8 @@ hyena_status_t hyena_forward_host(hyena_plan_t plan, int64_t batch, const void *
             status = HYENA_ERR_CUDA;
             break;
         }
-        status = hyena_forward(plan, nb, buf, gdev, H, Dskip, ydev, fwd_ws, s.fwd_ws, st);
+        status = split ? hyena::forward_channels_1d(plan, d0, dcount, buf, gdev, H, Dskip, ydev, fwd_ws, s.fwd_ws, st)
+                       : hyena_forward(plan, nb, buf, gdev, H, Dskip, ydev, fwd_ws, s.fwd_ws, st);
         if (status != HYENA_OK) break;
         e = cudaEventRecord(ev_comp[k], st);
         // copy-out

@@ -128,6 +128,7 @@ extern "C" hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batc
     a.rows = batch * plan->D;
     a.L = plan->L;
     a.D = plan->D;
+    a.hD = plan->D;
     a.B = batch;
     a.order = plan->order;
     a.es = plan->layout == HYENA_LAYOUT_BLD ? plan->D : 1;

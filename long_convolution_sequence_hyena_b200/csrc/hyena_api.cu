@@ -417,10 +417,13 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
 namespace {
 
 // The forward of both entry points: k == nullptr is the plain operator, else
-// the gate sandwich (z^0 = v SiLU(k), SiLU of every gate).
+// the gate sandwich (z^0 = v SiLU(k), SiLU of every gate). A 1D call may cover
+// the channel range [d0, d0 + dc) of one batch element: v, the gates and y then
+// hold those dc rows, while H and Dskip keep the whole plan's layout.
 hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, const void *k, const void *const *gates,
                             const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
-                            void *stream) {
+                            void *stream, int64_t d0 = 0, int64_t dc = -1) {
+    if (dc < 0) dc = plan->D;
     if (!v || !gates || !H || !y) return HYENA_ERR_INVALID_ARG;
     if (k && !aligned16(k)) return HYENA_ERR_ALIGNMENT;
     for (int n = 0; n < plan->order; ++n)
@@ -428,7 +431,7 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
     if (!aligned16(v) || !aligned16(H) || !aligned16(y) || (Dskip && !aligned4(Dskip))) return HYENA_ERR_ALIGNMENT;
     for (int n = 0; n < plan->order; ++n)
         if (!aligned16(gates[n])) return HYENA_ERR_ALIGNMENT;
-    const size_t ws_need = hyena_workspace_bytes(plan, batch);
+    const size_t ws_need = dc == plan->D ? hyena_workspace_bytes(plan, batch) : hyena::workspace_bytes_1d(plan, batch * dc);
     if (ws_need && (!workspace || ws_bytes < ws_need)) return HYENA_ERR_WORKSPACE;
     if (ws_need && !aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
     hyena_status_t s = check_device(plan);
@@ -483,13 +486,14 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
     std::memset(&a, 0, sizeof(a));
     a.v = v;
     for (int n = 0; n < plan->order; ++n) a.gates[n] = gates[n];
-    a.H = reinterpret_cast<const c32 *>(H);
-    a.dskip = Dskip;
+    a.H = reinterpret_cast<const c32 *>(H) + d0 * plan->spectrum_elems;
+    a.dskip = Dskip ? Dskip + d0 : nullptr;
     a.y = y;
     a.tw = reinterpret_cast<const c32 *>(plan->tw);
-    a.rows = batch * plan->D;
+    a.rows = batch * dc;
     a.L = plan->L;
-    a.D = plan->D;
+    a.D = dc;
+    a.hD = plan->D;
     a.B = batch;
     a.order = plan->order;
     a.es = plan->layout == HYENA_LAYOUT_BLD ? plan->D : 1;
@@ -512,6 +516,23 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
 }
 
 }  // namespace
+
+namespace hyena {
+
+size_t workspace_bytes_1d(hyena_plan_t plan, int64_t rows) {
+    if (plan->ndim != 1 || plan->path != HYENA_PATH_STAGED) return 0;
+    return (size_t)staged_workspace_rows(plan->MC, rows) * (size_t)plan->MC * sizeof(float2);
+}
+
+hyena_status_t forward_channels_1d(hyena_plan_t plan, int64_t d0, int64_t dc, const void *v, const void *const *gates,
+                                   const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
+                                   void *stream) {
+    if (plan->ndim != 1 || plan->layout != HYENA_LAYOUT_BDL || d0 < 0 || dc <= 0 || d0 + dc > plan->D)
+        return HYENA_ERR_INVALID_ARG;
+    return forward_impl(plan, 1, v, nullptr, gates, H, Dskip, y, workspace, ws_bytes, stream, d0, dc);
+}
+
+}  // namespace hyena
 
 extern "C" {
 

@@ -11,8 +11,8 @@ namespace hyena {
 struct Fwd1dArgs {
     const void *v;
     const void *gates[HYENA_MAX_ORDER];
-    const c32 *H;         // [N, D, MC + 1]
-    const float *dskip;   // [N, D] or nullptr
+    const c32 *H;         // row (n, d) at H + (n hD + d) (MC + 1)
+    const float *dskip;   // Dskip^n_d at dskip[n hD + d], or nullptr
     void *y;
     const c32 *tw;        // W_M^m, m in [0, M)
     int64_t rows;         // B * D
@@ -20,6 +20,10 @@ struct Fwd1dArgs {
     int64_t D;
     int64_t B;
     int order;
+    // channels between consecutive orders' rows of H and entries of dskip: D, or
+    // the plan's channel count when a call covers a sub-range of the channels
+    // (H and dskip then point at the range's first channel)
+    int64_t hD;
     // activation layout: es = 1 for [B, D, L] (a channel row is contiguous);
     // es = D for channels-last [B, L, D] (consecutive positions of a row are D
     // elements apart, and channel d of batch element b starts at b L D + d)
@@ -279,8 +283,8 @@ __global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
 #pragma unroll
         for (int q = 0; q < E / 2; ++q)
             g[q] = active ? load_pair_raw_s<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L, a.es) : io<IO>::zero();
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
         if constexpr (HS) {  // stage the spectrum row while the forward FFT runs
             for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);
             cp_async_commit();

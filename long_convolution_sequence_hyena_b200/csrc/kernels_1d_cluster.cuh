@@ -270,8 +270,8 @@ __global__ void __launch_bounds__(G::THREADS, G::MINB) hyena_fwd_1d_cluster(cons
             }
             cp_async_commit();
         }
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
 
         cx.template forward<true>(v, a.tw);
         cx.publish(v);

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(MR3<P>::THREADS, MR3<P>::MINB) hyena_fwd_1d_mr
             pim[k] = v[q].y;
         }
         __syncthreads();
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int k = s + 3 * (t + q * T);

@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
                 gb[q] = active ? load_pair_raw<IO, EVEN>(g1, pos, L) : io<IO>::zero();
             }
         }
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.D + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.D + d) * (MC + 1);
+        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
+        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
         for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);   // staged while the FFT runs
         cp_async_commit();
 

@@ -237,10 +237,10 @@ __global__ void __launch_bounds__(G::RT, G::RMINB) hyena_staged_rows_x2(const St
     // E-q when t2 = 0), so each thread takes q < E/2 and returns the mirror result
     // conj(Ye - i Yo) to its owner; bin (0, M2/2) is its own mirror;
     // the unpacking is written without its factors 1/2, folded into the gain
-    const float dsk0 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.D + d0) : 0.f;
-    const float dsk1 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.D + d1) : 0.f;
-    const c32 *H0 = a.f.H + ((int64_t)a.n * a.f.D + d0) * (MC + 1);
-    const c32 *H1 = a.f.H + ((int64_t)a.n * a.f.D + d1) * (MC + 1);
+    const float dsk0 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.hD + d0) : 0.f;
+    const float dsk1 = a.f.dskip ? __ldg(a.f.dskip + a.n * a.f.hD + d1) : 0.f;
+    const c32 *H0 = a.f.H + ((int64_t)a.n * a.f.hD + d0) * (MC + 1);
+    const c32 *H1 = a.f.H + ((int64_t)a.n * a.f.hD + d1) * (MC + 1);
     const c32 wb = ldg_c(a.f.tw + k1 + M1 * t2);     // W_M^{k1 + M1 t2}
     constexpr float s = 0.25f / (float)MC;
     const int z0 = opaque_zero();

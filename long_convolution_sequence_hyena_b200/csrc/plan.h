@@ -44,3 +44,18 @@ struct hyena_plan_s {
     // device error word (owned): set by a kernel whose bounded wait timed out
     int *dev_err = nullptr;
 };
+
+namespace hyena {
+
+// Rows of a staged 1D chunk (one lane's workspace slot) at packed length MC.
+int64_t staged_chunk_rows(int64_t MC);
+// Scratch a 1D forward over `rows` channel rows needs (0 off the staged path).
+size_t workspace_bytes_1d(hyena_plan_t plan, int64_t rows);
+// The 1D forward over channels [d0, d0 + dc) of one batch element of a
+// [B, D, L] plan: v, the gates and y hold those dc rows; H and Dskip are the
+// plan's whole tensors. Same kernels, so each row equals hyena_forward's.
+hyena_status_t forward_channels_1d(hyena_plan_t plan, int64_t d0, int64_t dc, const void *v, const void *const *gates,
+                                   const void *H, const float *Dskip, void *y, void *workspace, size_t ws_bytes,
+                                   void *stream);
+
+}  // namespace hyena

@@ -55,6 +55,41 @@ def test_forward_host_matches_device_forward(shape, B, D, N, dtype, stages):
     plan.close()
 
 
+@pytest.mark.parametrize("L,B,D,N,dtype,chunk", [
+    (65536, 1, 72, 3, torch.bfloat16, 32),   # channel stages of 32, 32 and 8 rows
+    (65536, 2, 40, 2, torch.float32, 32),    # two batch elements of stages of 32 and 8
+    (100000, 1, 48, 1, torch.bfloat16, 16),  # M = 262144: chunks of 16 rows, stages of 32 and 16
+])
+def test_forward_host_channel_stages(L, B, D, N, dtype, chunk):
+    """Long 1D rows: a batch element over 16 MiB of input is cut into channel
+    ranges of whole staged chunks, each an independent forward; the result
+    still equals hyena_forward's bit for bit."""
+    from long_convolution_sequence_hyena_b200 import api
+
+    plan = api.Plan((L,), D, N, dtype)
+    io = 4 if dtype == torch.float32 else 2
+    per_ch = (N + 1) * L * io
+    assert per_ch * D > 16 << 20
+    dc = max(chunk, (16 << 20) // per_ch // chunk * chunk)
+    assert dc < D
+    v, gates, h, dskip = _inputs(plan, (L,), B, D, N, dtype, seed=L + D)
+    H = plan.filter_spectrum(h=h)
+    y_dev = plan.forward(v, gates, H, dskip)
+    vh = v.cpu().pin_memory()
+    gh = [x.cpu().pin_memory() for x in gates]
+    yh = torch.full_like(vh, float("nan")).pin_memory()
+    plan.forward_host(vh, gh, H, dskip, out=yh)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.cpu())
+    # no Dskip: the channel ranges index the spectrum only
+    y0 = plan.forward(v, gates, H, None)
+    yh0 = torch.full_like(vh, float("nan")).pin_memory()
+    plan.forward_host(vh, gh, H, None, out=yh0)
+    torch.cuda.synchronize()
+    assert torch.equal(yh0, y0.cpu())
+    plan.close()
+
+
 def test_forward_host_sampled_rows_match_oracle():
     import oracle
     from long_convolution_sequence_hyena_b200 import api
