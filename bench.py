@@ -499,11 +499,11 @@ def summarize(w, r, world):
     if r["e2e_ms"] is not None:
         e2e = {"value": w.elements * world / (r["e2e_ms"] * 1e-3), "unit": "elems/s", "ms_per_step": r["e2e_ms"],
                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-               # copy-bound context: the step's input bytes over this box's measured pinned H2D rate;
-               # the copies of both directions share the host link on these boxes, so the
-               # step cannot beat (in + out bytes) at that rate
+               # copy-bound context: the step's input bytes over this box's measured pinned H2D
+               # rate (the floor), and its input and output bytes at that rate (the time if the
+               # two directions did not overlap at all)
                "h2d_gbs_measured": r["h2d"] / (r["h2d_ms"] * 1e-3) / 1e9, "h2d_ms_measured": r["h2d_ms"],
-               "copy_bound_ms": (r["h2d"] + r["d2h"]) / r["h2d"] * r["h2d_ms"]}
+               "copies_serial_ms": (r["h2d"] + r["d2h"]) / r["h2d"] * r["h2d_ms"]}
     out = {"ms_per_step": r["ms"], "value": job_throughput(w.elements, world, r["ms"]), "unit": "elems/s",
            "roofline": roof, "e2e": e2e, "gpu_launches_per_step": r["launches"]}
     if r["filt_ms"] > 0:

@@ -157,6 +157,33 @@ __device__ __forceinline__ void load_b_tile(TcSmem &S, const float *__restrict__
     }
 }
 
+// The head's B tile in two steps, so that the global loads of the next slice
+// overlap the current one: fetch_w3 reads rows [o0, o0 + NT) of W3 (zero past
+// oend) into registers, store_w3 writes them split into the B tile.
+constexpr int B_PER_THREAD = NT * (KW / 4) / THREADS;   // float4 per thread
+__device__ __forceinline__ void fetch_w3(const float *__restrict__ Wm, int64_t o0, int64_t oend, int tid,
+                                         float4 (&w)[B_PER_THREAD]) {
+#pragma unroll
+    for (int j = 0; j < B_PER_THREAD; ++j) {
+        const int i = tid + j * THREADS, o = i % NT, kc = i / NT;
+        const int64_t og = o0 + o;
+        w[j] = og < oend ? __ldg(reinterpret_cast<const float4 *>(Wm + og * KW) + kc) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+__device__ __forceinline__ void store_w3(TcSmem &S, const float4 (&w)[B_PER_THREAD], int tid) {
+    unsigned char *bhi = reinterpret_cast<unsigned char *>(S.b[0]);
+    unsigned char *blo = reinterpret_cast<unsigned char *>(S.b[1]);
+#pragma unroll
+    for (int j = 0; j < B_PER_THREAD; ++j) {
+        const int i = tid + j * THREADS, o = i % NT, kc = i / NT;
+        const float4 h4 = make_float4(tf32_hi(w[j].x), tf32_hi(w[j].y), tf32_hi(w[j].z), tf32_hi(w[j].w));
+        const int off = kc * (NT / 8) * SBO + (o >> 3) * SBO + (o & 7) * 16;
+        *reinterpret_cast<float4 *>(bhi + off) = h4;
+        *reinterpret_cast<float4 *>(blo + off) =
+            make_float4(w[j].x - h4.x, w[j].y - h4.y, w[j].z - h4.z, w[j].w - h4.w);
+    }
+}
+
 // 32 consecutive accumulator columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     uint32_t u[32];
@@ -222,32 +249,8 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
         float a1[KW / PARTS];
 #pragma unroll
         for (int j = 0; j < KW / PARTS; ++j) a1[j] = 0.f;
-#pragma unroll 1
-        for (int f = 0; f < fin; ++f) {
-            float fv = 0.f;
-            if (in) {
-                if (a.ndim == 1) {
-                    if (f == 0) {
-                        fv = (float)((double)pos / (double)a.L);
-                    } else {
-                        const int64_t k = (f + 1) / 2;
-                        const int64_t r = (k * pos) % a.L;   // angle 2 pi k t / L, reduced exactly first
-                        float sv, cv;
-                        sincospif((float)(2.0 * (double)r / (double)a.L), &sv, &cv);
-                        fv = (f & 1) ? cv : sv;
-                    }
-                } else if (a.ndim == 2) {
-                    const int64_t iy = pos / (2 * a.W), ix = pos - iy * (2 * a.W);
-                    fv = f == 0 ? (float)((double)(iy - a.H) / (double)a.H) : (float)((double)(ix - a.W) / (double)a.W);
-                } else {   // 3D: (oz / Dz, oy / H, ox / W) on the offset grid [2Dz][2H][2W]
-                    const int64_t hw = 4 * a.H * a.W;
-                    const int64_t iz = pos / hw, rem = pos - iz * hw;
-                    const int64_t iy = rem / (2 * a.W), ix = rem - iy * (2 * a.W);
-                    fv = f == 0 ? (float)((double)(iz - a.Dz) / (double)a.Dz)
-                                : (f == 1 ? (float)((double)(iy - a.H) / (double)a.H)
-                                          : (float)((double)(ix - a.W) / (double)a.W));
-                }
-            }
+        // adds feature f (value fv) times its first-layer weights to this thread's units
+        auto add_feature = [&](int f, float fv) __attribute__((always_inline)) {
             const float4 *wrow = reinterpret_cast<const float4 *>(S.w1t[0] + f * KW + (KW / PARTS) * part);
 #pragma unroll
             for (int j4 = 0; j4 < KW / PARTS / 4; ++j4) {
@@ -256,6 +259,42 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
                 a1[4 * j4 + 1] = fmaf(w.y, fv, a1[4 * j4 + 1]);
                 a1[4 * j4 + 2] = fmaf(w.z, fv, a1[4 * j4 + 2]);
                 a1[4 * j4 + 3] = fmaf(w.w, fv, a1[4 * j4 + 3]);
+            }
+        };
+        if (a.ndim == 1) {
+            // [t/L, cos(2 pi k t/L), sin(2 pi k t/L) for k = 1..K]: the angle's turns
+            // (k t mod L) / L advance by t per frequency, kept exact in integers
+            // (t < L <= 2^19, so k t fits in 32 bits)
+            const int Li = (int)a.L, t = in ? (int)pos : 0;
+            add_feature(0, in ? __fdiv_rn((float)t, (float)Li) : 0.f);
+            int rk = 0;
+#pragma unroll 1
+            for (int k = 1; 2 * k < fin; ++k) {
+                rk += t;
+                if (rk >= Li) rk -= Li;
+                float sv = 0.f, cv = 0.f;
+                if (in) sincospif(__fdiv_rn((float)(2 * rk), (float)Li), &sv, &cv);
+                add_feature(2 * k - 1, cv);
+                add_feature(2 * k, sv);
+            }
+        } else {
+#pragma unroll 1
+            for (int f = 0; f < fin; ++f) {
+                float fv = 0.f;
+                if (in) {   // offsets on grids of at most 2^21 points: 32-bit index arithmetic
+                    const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, pi = (int)pos;
+                    if (a.ndim == 2) {
+                        const int iy = pi / W2, ix = pi - iy * W2;
+                        fv = f == 0 ? __fdiv_rn((float)(iy - Hi), (float)Hi) : __fdiv_rn((float)(ix - Wi), (float)Wi);
+                    } else {   // 3D: (oz / Dz, oy / H, ox / W) on the offset grid [2Dz][2H][2W]
+                        const int hw = 2 * Hi * W2, Dzi = (int)a.Dz;
+                        const int iz = pi / hw, rem = pi - iz * hw;
+                        const int iy = rem / W2, ix = rem - iy * W2;
+                        fv = f == 0 ? __fdiv_rn((float)(iz - Dzi), (float)Dzi)
+                                    : (f == 1 ? __fdiv_rn((float)(iy - Hi), (float)Hi) : __fdiv_rn((float)(ix - Wi), (float)Wi));
+                    }
+                }
+                add_feature(f, fv);
             }
         }
 #pragma unroll
@@ -319,16 +358,18 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
     if (a.ndim == 1) {
         we = (float)ppos;
     } else if (a.ndim == 2 && ppos < a.npos) {
-        const int64_t iy = ppos / (2 * a.W), ix = ppos - iy * (2 * a.W);
-        const float py = (float)((double)(iy - a.H) / (double)a.H), px = (float)((double)(ix - a.W) / (double)a.W);
+        const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, pi = (int)ppos;
+        const int iy = pi / W2, ix = pi - iy * W2;
+        const float py = __fdiv_rn((float)(iy - Hi), (float)Hi), px = __fdiv_rn((float)(ix - Wi), (float)Wi);
         we = py * py + px * px;
-        poff = iy * a.out_row_stride + ix;
+        poff = (int64_t)iy * a.out_row_stride + ix;
     } else if (a.ndim == 3 && ppos < a.npos) {   // output [2Dz][2H][2W] contiguous per channel
-        const int64_t hw = 4 * a.H * a.W;
-        const int64_t iz = ppos / hw, rem = ppos - iz * hw;
-        const int64_t iy = rem / (2 * a.W), ix = rem - iy * (2 * a.W);
-        const float pz = (float)((double)(iz - a.Dz) / (double)a.Dz);
-        const float py = (float)((double)(iy - a.H) / (double)a.H), px = (float)((double)(ix - a.W) / (double)a.W);
+        const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, Dzi = (int)a.Dz, pi = (int)ppos;
+        const int hw = 2 * Hi * W2;
+        const int iz = pi / hw, rem = pi - iz * hw;
+        const int iy = rem / W2, ix = rem - iy * W2;
+        const float pz = __fdiv_rn((float)(iz - Dzi), (float)Dzi);
+        const float py = __fdiv_rn((float)(iy - Hi), (float)Hi), px = __fdiv_rn((float)(ix - Wi), (float)Wi);
         we = pz * pz + py * py + px * px;
     }
     static_assert(NT / (THREADS / 128) == 32, "each warp reads 32 accumulator columns");
@@ -346,12 +387,19 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
             dst += a.out_stride;
         }
     };
+    // The B tile is free: the second layer's MMAs have completed. Slice s's W3
+    // rows are fetched while slice s - 1's MMAs and slice s - 2's epilogue run,
+    // and written into the B tile once slice s - 1's MMAs are done.
+    float4 wb[B_PER_THREAD];
+    if (nslices > 0) {
+        fetch_w3(a.p.W3, o_begin, o_end, tid, wb);
+        store_w3(S, wb, tid);
+    }
 #pragma unroll 1
     for (int s = 0; s < nslices; ++s) {
-        // W3 rows of slice s as the B tile; their window scales and biases. The
-        // epilogue of slice s - 1 still reads S.oc: it runs after the barrier below.
+        // slice s's window scales and biases; the epilogue of slice s - 1 still
+        // reads S.oc: they are written after the barrier below
         const int64_t os = o_begin + (int64_t)s * NT;
-        load_b_tile(S, a.p.W3, os, NT, o_end, tid);
         float2 oc_new = make_float2(0.f, 0.f);
         if (tid < NT && os + tid < o_end) {
             const float wp = __ldg(a.p.window + os + tid);
@@ -367,11 +415,13 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
             mma_split_k64(tmem + (uint32_t)((s & 1) * NT), sah, sal, sbh, sbl, (NT / 8) * SBO, idesc_n(NT));
             mma_commit(&S.mbar);
         }
+        if (s + 1 < nslices) fetch_w3(a.p.W3, os + NT, o_end, tid, wb);   // in flight during the epilogue
         if (s > 0) epilogue(s - 1);   // overlaps the MMAs of slice s
         __syncthreads();              // every read of S.oc for slice s - 1 done
         if (tid < NT) S.oc[tid] = oc_new;
-        wait_mma();
-        __syncthreads();              // slice s complete (or abandoned) and S.oc updated
+        wait_mma();                   // slice s complete (or abandoned): the B tile is free
+        if (s + 1 < nslices) store_w3(S, wb, tid);
+        __syncthreads();              // S.oc updated (the next iteration fences the B tile)
     }
     if (nslices > 0 && ok) epilogue(nslices - 1);
     tc_fence_before();

@@ -331,10 +331,17 @@ __global__ void __launch_bounds__(rows_per_cta(MC, E) * (MC / E))
     float *sim = sre + MC;
     c32 v[E];
     const float *hrow = h + (active ? o : 0) * h_stride;
+    // tap pairs as one 8-byte load where every row starts 8-byte aligned
+    const bool pairs = ((reinterpret_cast<uintptr_t>(h) | (uintptr_t)(h_stride * 4)) & 7) == 0;
 #pragma unroll
     for (int q = 0; q < E / 2; ++q) {
         const int64_t pos = 2 * (int64_t)(t + q * T);
-        v[q] = mk(active && pos < L ? hrow[pos] : 0.f, active && pos + 1 < L ? hrow[pos + 1] : 0.f);
+        if (pairs && active && pos + 1 < L) {
+            const float2 x = *reinterpret_cast<const float2 *>(hrow + pos);   // plain load: the row may be transformed in place
+            v[q] = mk(x.x, x.y);
+        } else {
+            v[q] = mk(active && pos < L ? hrow[pos] : 0.f, active && pos + 1 < L ? hrow[pos + 1] : 0.f);
+        }
     }
 #pragma unroll
     for (int q = E / 2; q < E; ++q) v[q] = mk(0.f, 0.f);

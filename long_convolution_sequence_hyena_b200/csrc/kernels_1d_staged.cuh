@@ -37,9 +37,11 @@ struct StagedGeom {
     static constexpr int TWS = 1024;                 // sub-transform twiddle table W_1024
     static constexpr size_t CSMEM = (size_t)NCOL * M1 * 8 * ROWS;
     static constexpr size_t RSMEM = (size_t)NROW * M2 * 8 * ROWS;
-    // resident CTAs per SM the register budget is sized for (128-thread CTAs: 3
-    // column / 4 row CTAs; larger CTAs: 128 registers per thread)
-    static constexpr int CMINB = CT <= 128 ? 3 : 512 / CT;
+    // resident CTAs per SM the register budget is sized for (128-thread CTAs: 4,
+    // at 128 registers, a few bytes of spills in some column instances, which
+    // measured faster than 3 CTAs at up to 168 registers; larger CTAs: 128
+    // registers per thread)
+    static constexpr int CMINB = CT <= 128 ? 4 : 512 / CT;
     static constexpr int RMINB = RT <= 128 ? 4 : 512 / RT;
     static_assert(M2 % NCOL == 0 && M1 % NROW == 0 && NROW % 2 == 0, "groups must tile the row");
     static_assert((ROWS == 1 && NCOL >= 16 && NROW >= 16) || (ROWS == 2 && NCOL >= 8 && NROW >= 8),
