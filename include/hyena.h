@@ -152,6 +152,11 @@ HYENA_API hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout);
  * HYENA_ERR_CUDA if an error was recorded, HYENA_OK otherwise.
  */
 HYENA_API hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags, int clear);
+/* Bits of the device error word: a bounded wait ran out; an index check of
+ * the HYENA_CHECK_BOUNDS debug build (libhyena_checked.so) failed and the
+ * access was skipped. */
+#define HYENA_DEVERR_WAIT_TIMEOUT 1
+#define HYENA_DEVERR_BOUNDS 4
 
 /*
  * The number of kernels this library has enqueued in the calling process
@@ -161,6 +166,19 @@ HYENA_API hyena_status_t hyena_plan_device_errors(hyena_plan_t plan, int *flags,
  * touches the device. *count must not be NULL (HYENA_ERR_INVALID_ARG).
  */
 HYENA_API hyena_status_t hyena_launch_count(int64_t *count);
+
+/*
+ * Test hooks for the failure paths of plan creation (no effect on results).
+ * hyena_debug_fail_allocation(n): the n-th resource that plan creation
+ * creates from now on (device buffer, stream or host object, counted over all
+ * threads) fails as if the device or host were out of memory; the plan call
+ * then releases what it had created and returns HYENA_ERR_NOMEM (a stream:
+ * HYENA_ERR_CUDA). n = 0 disarms it; n < 0 is HYENA_ERR_INVALID_ARG.
+ * hyena_debug_plan_resources(&n): the number of such resources all live
+ * plans hold; *count must not be NULL.
+ */
+HYENA_API hyena_status_t hyena_debug_fail_allocation(int nth);
+HYENA_API hyena_status_t hyena_debug_plan_resources(int64_t *count);
 
 /*
  * hyena_plan_create with options. flags is 0 (the same plan as

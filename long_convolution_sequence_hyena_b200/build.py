@@ -1,4 +1,7 @@
-"""Build the CUDA library ``libhyena.so`` in-tree for sm_100a with nvcc."""
+"""Build the CUDA library ``libhyena.so`` in-tree for sm_100a with nvcc, and its
+debug twin ``libhyena_checked.so`` (the same sources with HYENA_CHECK_BOUNDS:
+index checks that record a device error bit instead of accessing out of
+range)."""
 from __future__ import annotations
 
 import glob
@@ -11,6 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libhyena.so")
+LIB_CHECKED = os.path.join(PKG, "libhyena_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -29,10 +33,10 @@ def _deps():
         sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
@@ -51,14 +55,17 @@ def _object_stale(obj: str, dep: str, src: str, flags_file: str, flags: str) -> 
     return any(not os.path.exists(d) or os.path.getmtime(d) > t for d in deps + [src])
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), checked: bool = False) -> str:
     """Compile csrc/*.cu (in parallel, one object each; only the objects whose source or
     included headers changed) and link one shared library. Skipped when the library is
-    newer than every source."""
-    if not force and not needs_build():
-        return LIB
+    newer than every source. checked=True builds the HYENA_CHECK_BOUNDS library."""
+    lib = LIB_CHECKED if checked else LIB
+    if checked:
+        extra_flags = [*extra_flags, "-DHYENA_CHECK_BOUNDS"]
+    if not force and not needs_build(lib):
+        return lib
     nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
-    objdir = os.path.join(PKG, "_build")
+    objdir = os.path.join(PKG, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
     procs = []
     objs = []
@@ -84,13 +91,13 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
                 f.write(flags)
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs, "-lcudart"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def source_hash() -> str:
@@ -105,6 +112,5 @@ def source_hash() -> str:
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True,
+                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [], checked="--checked" in sys.argv))

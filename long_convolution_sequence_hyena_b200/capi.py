@@ -11,7 +11,9 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libhyena.so")
+# HYENA_LIBRARY=checked loads the index-checking debug build (libhyena_checked.so)
+LIB_PATH = os.path.join(_PKG, "libhyena_checked.so" if os.environ.get("HYENA_LIBRARY") == "checked"
+                        else "libhyena.so")
 
 HYENA_MAX_ORDER = 8
 HYENA_F32, HYENA_BF16 = 0, 1
@@ -34,7 +36,7 @@ EXPORTED = (
     "hyena_implicit_filter", "hyena_filter_spectrum", "hyena_forward", "hyena_status_string",
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
     "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors", "hyena_plan_create_ex",
-    "hyena_launch_count",
+    "hyena_launch_count", "hyena_debug_fail_allocation", "hyena_debug_plan_resources",
 )
 
 
@@ -72,6 +74,8 @@ def _load():
         "hyena_plan_device_errors": ([p, ctypes.POINTER(i32), i32], i32),
         "hyena_plan_create_ex": ([ctypes.POINTER(p), i32, ctypes.POINTER(i64), i64, i32, i32, i32, i32], i32),
         "hyena_launch_count": ([ctypes.POINTER(i64)], i32),
+        "hyena_debug_fail_allocation": ([i32], i32),
+        "hyena_debug_plan_resources": ([ctypes.POINTER(i64)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -124,6 +128,15 @@ def hyena_launch_count() -> int:
     st = lib.hyena_launch_count(ctypes.byref(n))
     if st != HYENA_OK:
         raise RuntimeError("hyena_launch_count: %d" % st)
+    return n.value
+
+
+def hyena_debug_plan_resources() -> int:
+    """Device buffers, streams and host objects all live plans hold (test hook)."""
+    n = ctypes.c_int64()
+    st = lib.hyena_debug_plan_resources(ctypes.byref(n))
+    if st != HYENA_OK:
+        raise RuntimeError("hyena_debug_plan_resources: %d" % st)
     return n.value
 
 

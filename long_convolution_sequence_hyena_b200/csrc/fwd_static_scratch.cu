@@ -132,6 +132,7 @@ extern "C" hyena_status_t hyena_forward_no_alloc(hyena_plan_t plan, int64_t batc
     a.B = batch;
     a.order = plan->order;
     a.es = plan->layout == HYENA_LAYOUT_BLD ? plan->D : 1;
+    a.err = plan->dev_err;
     const int64_t chunk = (int64_t)(kScratchBytes / row_bytes) & ~(int64_t)1;   // whole row pairs
     cudaStream_t st = (cudaStream_t)stream;
     const cudaError_t e =

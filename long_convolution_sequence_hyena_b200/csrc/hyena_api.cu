@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "hyena.h"
@@ -41,14 +42,85 @@ std::vector<float2> twiddle_table(int64_t M) {
 }
 
 // Destroy the staged path's streams (those that were created).
+// Resources a plan holds (device buffers, streams, host objects) are created
+// and released through these helpers, which count them (the test hook
+// hyena_debug_plan_resources reads the count) and can be made to fail
+// (hyena_debug_fail_allocation), so that tests reach every unwind path of
+// plan creation.
+std::atomic<int64_t> g_plan_resources{0};
+std::atomic<int> g_fail_countdown{0};   // the nth creation from now fails; 0: none
+
+bool injected_failure() {
+    int n = g_fail_countdown.load();
+    while (n > 0)
+        if (g_fail_countdown.compare_exchange_weak(n, n - 1)) return n == 1;
+    return false;
+}
+bool res_dev_alloc(void **p, size_t bytes) {
+    if (injected_failure()) return false;
+    if (cudaMalloc(p, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return false;
+    }
+    ++g_plan_resources;
+    return true;
+}
+bool res_dev_free(void *p) {
+    if (!p) return true;
+    --g_plan_resources;
+    return cudaFree(p) == cudaSuccess;
+}
+bool res_stream_create(cudaStream_t *s) {
+    if (injected_failure()) return false;
+    if (cudaStreamCreateWithFlags(s, cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        *s = nullptr;
+        return false;
+    }
+    ++g_plan_resources;
+    return true;
+}
+template <typename T, typename... A>
+T *res_new(A &&...args) {
+    if (injected_failure()) return nullptr;
+    T *o = new (std::nothrow) T(std::forward<A>(args)...);
+    if (o) ++g_plan_resources;
+    return o;
+}
+template <typename T>
+void res_delete(T *o) {
+    if (!o) return;
+    --g_plan_resources;
+    delete o;
+}
+
 bool release_lanes(hyena_plan_s *p) {
     if (!p->has_lanes) return true;
     bool ok = true;
     for (int i = 0; i < HYENA_STAGED_LANES; ++i) {
-        if (p->lane[i] && cudaStreamDestroy(p->lane[i]) != cudaSuccess) ok = false;
+        if (p->lane[i]) {
+            --g_plan_resources;
+            if (cudaStreamDestroy(p->lane[i]) != cudaSuccess) ok = false;
+        }
         p->lane[i] = nullptr;
     }
     p->has_lanes = false;
+    return ok;
+}
+
+// Everything a plan (or a plan under construction) holds, except the plan
+// object itself; false if a CUDA release failed.
+bool release_plan_resources(hyena_plan_s *p) {
+    bool ok = release_lanes(p);
+    ok = res_dev_free(p->spec_ws) && ok;
+    ok = res_dev_free(p->dev_err) && ok;
+    ok = res_dev_free(p->tw) && ok;
+    res_delete(p->spec_mu);
+    p->spec_ws = nullptr;
+    p->dev_err = nullptr;
+    p->tw = nullptr;
+    p->spec_mu = nullptr;
     return ok;
 }
 
@@ -218,78 +290,49 @@ hyena_status_t hyena_plan_create_ex(hyena_plan_t *out, int ndim, const int64_t *
         std::vector<float2> sub = twiddle_table(HYENA_SUB_TWIDDLES);
         tw.insert(tw.end(), sub.begin(), sub.end());
     }
-    if (cudaMalloc(&p.tw, sizeof(float2) * tw.size()) != cudaSuccess) {
-        cudaGetLastError();
-        return HYENA_ERR_NOMEM;
-    }
-    if (cudaMemcpy(p.tw, tw.data(), sizeof(float2) * tw.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
-        cudaFree(p.tw);
-        return HYENA_ERR_CUDA;
-    }
-    if (cudaMalloc(&p.dev_err, 4 * sizeof(int)) != cudaSuccess) {
-        cudaGetLastError();
-        cudaFree(p.tw);
-        return HYENA_ERR_NOMEM;
-    }
-    if (cudaMemset(p.dev_err, 0, 4 * sizeof(int)) != cudaSuccess) {
-        cudaFree(p.dev_err);
-        cudaFree(p.tw);
-        return HYENA_ERR_CUDA;
-    }
+    // every failure below releases what was created before it (release_plan_resources)
+    auto fail = [&](hyena_status_t st) {
+        release_plan_resources(&p);
+        return st;
+    };
+    if (!res_dev_alloc(reinterpret_cast<void **>(&p.tw), sizeof(float2) * tw.size())) return fail(HYENA_ERR_NOMEM);
+    if (cudaMemcpy(p.tw, tw.data(), sizeof(float2) * tw.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+        return fail(HYENA_ERR_CUDA);
+    if (!res_dev_alloc(reinterpret_cast<void **>(&p.dev_err), 4 * sizeof(int))) return fail(HYENA_ERR_NOMEM);
+    if (cudaMemset(p.dev_err, 0, 4 * sizeof(int)) != cudaSuccess) return fail(HYENA_ERR_CUDA);
     if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
-        bool ok = true;
-        for (int i = 0; i < HYENA_STAGED_LANES && ok; ++i)
-            ok = cudaStreamCreateWithFlags(&p.lane[i], cudaStreamNonBlocking) == cudaSuccess;
         p.has_lanes = true;
-        if (!ok) {
-            release_lanes(&p);
-            cudaFree(p.dev_err);
-            cudaFree(p.tw);
-            return HYENA_ERR_CUDA;
-        }
-    }
-    if (p.path == HYENA_PATH_STAGED || (p.path == HYENA_PATH_2D && staged2d_supported(p.Ww))) {
+        for (int i = 0; i < HYENA_STAGED_LANES; ++i)
+            if (!res_stream_create(&p.lane[i])) return fail(HYENA_ERR_CUDA);
         const size_t sb = p.path == HYENA_PATH_STAGED ? staged_spec_scratch_bytes(p.MC)
                                                       : staged2d_spec_scratch_bytes(p.Ww);
-        if (cudaMalloc(&p.spec_ws, sb) != cudaSuccess) {
-            cudaGetLastError();
-            release_lanes(&p);
-            cudaFree(p.dev_err);
-            cudaFree(p.tw);
-            return HYENA_ERR_NOMEM;
-        }
-        p.spec_mu = new (std::nothrow) std::mutex;
-        if (!p.spec_mu) {
-            cudaFree(p.spec_ws);
-            release_lanes(&p);
-            cudaFree(p.dev_err);
-            cudaFree(p.tw);
-            return HYENA_ERR_NOMEM;
-        }
+        if (!res_dev_alloc(reinterpret_cast<void **>(&p.spec_ws), sb)) return fail(HYENA_ERR_NOMEM);
+        p.spec_mu = res_new<std::mutex>();
+        if (!p.spec_mu) return fail(HYENA_ERR_NOMEM);
     }
-    hyena_plan_s *heap = new (std::nothrow) hyena_plan_s(p);
-    if (!heap) {
-        release_lanes(&p);
-        if (p.spec_ws) cudaFree(p.spec_ws);
-        delete p.spec_mu;
-        cudaFree(p.dev_err);
-        cudaFree(p.tw);
-        return HYENA_ERR_NOMEM;
-    }
+    hyena_plan_s *heap = res_new<hyena_plan_s>(p);
+    if (!heap) return fail(HYENA_ERR_NOMEM);
     *out = heap;
     return HYENA_OK;
 }
 
 hyena_status_t hyena_plan_destroy(hyena_plan_t plan) {
     if (!plan) return HYENA_OK;
-    hyena_status_t st = HYENA_OK;
-    if (plan->tw && cudaFree(plan->tw) != cudaSuccess) st = HYENA_ERR_CUDA;
-    if (!release_lanes(plan)) st = HYENA_ERR_CUDA;
-    if (plan->spec_ws && cudaFree(plan->spec_ws) != cudaSuccess) st = HYENA_ERR_CUDA;
-    if (plan->dev_err && cudaFree(plan->dev_err) != cudaSuccess) st = HYENA_ERR_CUDA;
-    delete plan->spec_mu;
-    delete plan;
-    return st;
+    const bool ok = release_plan_resources(plan);
+    res_delete(plan);
+    return ok ? HYENA_OK : HYENA_ERR_CUDA;
+}
+
+hyena_status_t hyena_debug_fail_allocation(int nth) {
+    if (nth < 0) return HYENA_ERR_INVALID_ARG;
+    g_fail_countdown.store(nth);
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_debug_plan_resources(int64_t *count) {
+    if (!count) return HYENA_ERR_INVALID_ARG;
+    *count = g_plan_resources.load();
+    return HYENA_OK;
 }
 
 hyena_status_t hyena_plan_set_layout(hyena_plan_t plan, int layout) {
@@ -471,6 +514,7 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
         a.C = plan->D;
         a.B = batch;
         a.order = plan->order;
+        a.err = plan->dev_err;
         cudaError_t e2;
         if (staged2d_supported(plan->Ww)) {
             CallLanes cl(plan);
@@ -497,6 +541,7 @@ hyena_status_t forward_impl(hyena_plan_t plan, int64_t batch, const void *v, con
     a.B = batch;
     a.order = plan->order;
     a.es = plan->layout == HYENA_LAYOUT_BLD ? plan->D : 1;
+    a.err = plan->dev_err;
     const bool even = (plan->L % 2) == 0;
     cudaError_t e;
     if (plan->path == HYENA_PATH_STAGED) {

@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
     auto wait_mma = [&]() {
         if (ok && !mbar_wait(&S.mbar, phase)) {
             ok = false;
-            atomicExch(err, 1);
+            atomicOr(err, HYENA_DEVERR_WAIT_TIMEOUT);
         }
         phase ^= 1;
         tc_fence_after();

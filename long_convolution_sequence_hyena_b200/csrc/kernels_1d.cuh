@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "check.cuh"
 #include "cta_fft.cuh"
 #include "hyena.h"
 
@@ -24,6 +25,7 @@ struct Fwd1dArgs {
     // the plan's channel count when a call covers a sub-range of the channels
     // (H and dskip then point at the range's first channel)
     int64_t hD;
+    int *err;             // the plan's device error word (index checks of the debug build)
     // activation layout: es = 1 for [B, D, L] (a channel row is contiguous);
     // es = D for channels-last [B, L, D] (consecutive positions of a row are D
     // elements apart, and channel d of batch element b starts at b L D + d)
@@ -257,10 +259,11 @@ __global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
     const int lrow = threadIdx.x / T;
     const int t = threadIdx.x - lrow * T;
     const int64_t ord = (int64_t)blockIdx.x * RPC + lrow;
-    const bool active = ord < a.rows;
-    const int64_t d = active ? ord / a.B : 0;
-    const int64_t b = active ? ord - d * a.B : 0;
+    const bool in_grid = ord < a.rows;
+    const int64_t d = in_grid ? ord / a.B : 0;
+    const int64_t b = in_grid ? ord - d * a.B : 0;
     const int64_t row = b * a.D + d;
+    const bool active = in_grid && check_index(a.err, row, a.rows) && check_index(a.err, d, a.D);
     float *sre = smem + lrow * fwd_smem_floats_per_row(MC);
     float *sim = sre + MC;
     c32 *Hs = HS ? reinterpret_cast<c32 *>(sim + MC) : nullptr;
@@ -283,8 +286,9 @@ __global__ void __launch_bounds__(fwd_threads(MC, E), fwd_min_blocks(MC, E))
 #pragma unroll
         for (int q = 0; q < E / 2; ++q)
             g[q] = active ? load_pair_raw_s<IO, EVEN>(grow, 2 * (int64_t)(t + q * T), L, a.es) : io<IO>::zero();
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
+        const int64_t hrow = check_index(a.err, (int64_t)n * a.hD + d, (int64_t)a.order * a.hD) ? n * a.hD + d : 0;
+        const float dsk = a.dskip ? __ldg(a.dskip + hrow) : 0.f;
+        const c32 *Hrow = a.H + hrow * (MC + 1);
         if constexpr (HS) {  // stage the spectrum row while the forward FFT runs
             for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);
             cp_async_commit();

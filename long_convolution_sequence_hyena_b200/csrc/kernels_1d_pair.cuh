@@ -190,11 +190,13 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
     const int t = threadIdx.x - lp * T;
     const int64_t npairs = a.rows / 2;
     const int64_t pidx = (int64_t)blockIdx.x * PPC + lp;
-    const bool active = pidx < npairs;
+    const bool in_grid = pidx < npairs;
     const int64_t hb = a.B / 2;
-    const int64_t d = active ? pidx / hb : 0;
-    const int64_t b0 = active ? 2 * (pidx - d * hb) : 0;
+    const int64_t d = in_grid ? pidx / hb : 0;
+    const int64_t b0 = in_grid ? 2 * (pidx - d * hb) : 0;
     const int64_t row0 = b0 * a.D + d, row1 = row0 + a.D;
+    const bool active = in_grid && check_index(a.err, row0, a.rows) && check_index(a.err, row1, a.rows) &&
+                        check_index(a.err, d, a.D);
     unsigned char *base = reinterpret_cast<unsigned char *>(smem4) + lp * pair_smem_bytes_per_pair(MC);
     float2 *sre = reinterpret_cast<float2 *>(base);
     float2 *sim = sre + MC;
@@ -248,8 +250,9 @@ __global__ void __launch_bounds__(pair_threads(MC, E), pair_min_blocks(MC, E))
                 gb[q] = active ? load_pair_raw<IO, EVEN>(g1, pos, L) : io<IO>::zero();
             }
         }
-        const float dsk = a.dskip ? __ldg(a.dskip + n * a.hD + d) : 0.f;
-        const c32 *Hrow = a.H + ((int64_t)n * a.hD + d) * (MC + 1);
+        const int64_t hrow = check_index(a.err, (int64_t)n * a.hD + d, (int64_t)a.order * a.hD) ? n * a.hD + d : 0;
+        const float dsk = a.dskip ? __ldg(a.dskip + hrow) : 0.f;
+        const c32 *Hrow = a.H + hrow * (MC + 1);
         for (int i = t; i <= MC; i += T) cp_async8(Hs + i, Hrow + i);   // staged while the FFT runs
         cp_async_commit();
 

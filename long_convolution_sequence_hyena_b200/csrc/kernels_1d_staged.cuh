@@ -116,6 +116,10 @@ __global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_cols_x2(const St
     int64_t d0, d1;
     const int64_t row0 = visit_row(a.f, a.o0 + 2 * lp, d0);
     const int64_t row1 = visit_row(a.f, a.o0 + 2 * lp + (has1 ? 1 : 0), d1);
+    // debug build: the CTA's rows exist (uniform over the CTA, so it may leave as a whole)
+    if (!(check_index(a.f.err, row0, a.f.rows) && check_index(a.f.err, row1, a.f.rows) &&
+          check_index(a.f.err, 2 * lp + (has1 ? 1 : 0), nr)))
+        return;
     const int64_t L = a.f.L;
     float2 *w0 = a.ws + (2 * lp) * MC;
     float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
@@ -147,6 +151,10 @@ __global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_cols_x2(const St
 #pragma unroll
         for (int q = 0; q < E; ++q) {
             const int ad = (t1 + q * T1) * M2 + n2;     // k1 = t1 + q T1
+            if (!check_index(a.f.err, ad, MC)) {
+                v[q] = c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
+                continue;
+            }
             const float2 f0 = ld_pol(w0 + ad, pol), f1 = ld_pol(w1 + ad, pol);
             v[q] = c32x2{f2(f0.x, f1.x), f2(f0.y, f1.y)};
         }
@@ -181,6 +189,7 @@ __global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_cols_x2(const St
         for (int q = 0; q < E; ++q) {
             const c32x2 r = mul(v[q], base);
             const int ad = (t1 + q * T1) * M2 + n2;
+            if (!check_index(a.f.err, ad, MC)) continue;
             st_pol(w0 + ad, make_float2(r.re.x, r.im.x), keep);
             if (has1) st_pol(w1 + ad, make_float2(r.re.y, r.im.y), keep);
         }
@@ -203,15 +212,23 @@ __global__ void __launch_bounds__(G::RT, G::RMINB) hyena_staged_rows_x2(const St
     int64_t d0, d1;
     (void)visit_row(a.f, a.o0 + 2 * lp, d0);
     (void)visit_row(a.f, a.o0 + 2 * lp + (has1 ? 1 : 0), d1);
+    // debug build: the CTA's rows and their spectrum rows exist (uniform over the CTA)
+    const int64_t hrows = (int64_t)a.f.order * a.f.hD;
+    if (!(check_index(a.f.err, 2 * lp + (has1 ? 1 : 0), nr) && check_index(a.f.err, d0, a.f.D) &&
+          check_index(a.f.err, d1, a.f.D) && check_index(a.f.err, (int64_t)a.n * a.f.hD + d1, hrows)))
+        return;
     float2 *w0 = a.ws + (2 * lp) * MC;
     float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * MC;
     const c32 *tws = a.f.tw + M;
-    // shared element (re a, re b, im a, im b)
+    // shared element (re a, re b, im a, im b); the debug build checks the slot index
     auto ld = [&](int ad) -> c32x2 {
+        if (!check_index(a.f.err, ad, NROW * M2)) return c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
         const float4 f = rowb[ad];
         return c32x2{f2(f.x, f.y), f2(f.z, f.w)};
     };
-    auto st = [&](int ad, c32x2 x) { rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y); };
+    auto st = [&](int ad, c32x2 x) {
+        if (check_index(a.f.err, ad, NROW * M2)) rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y);
+    };
 
     // the group's rows of both lanes, coalesced, into the sequence-major buffer
     const uint64_t keep = l2_keep(), stream = l2_stream();

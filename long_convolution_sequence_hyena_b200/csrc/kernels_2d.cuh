@@ -30,6 +30,7 @@ struct Fwd2dArgs {
     int64_t C;
     int64_t B;
     int order;
+    int *err;             // the plan's device error word (index checks of the debug build)
 };
 
 // Fused order-N 2D forward (planes visited c-major, b-minor). GATED: the

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dAr
     const int xc = cgp * G::NCOL + j;                // data column x' < XW
     int64_t c;
     const int64_t plane = visit_plane(a.f, a.o0 + lp, c);
+    // debug build: the plane exists (uniform over the CTA, so it may leave as a whole)
+    if (!(check_index(a.f.err, plane, a.f.planes) && check_index(a.f.err, c, a.f.C))) return;
     float2 *wp = a.ws + lp * G::PLANE;
     const c32 *tws = a.f.tw + 2 * G::M2;             // W_1024 after the W_{2W} table
     const int64_t plane_elems = (int64_t)Hh * Ww;
@@ -138,14 +140,22 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged2d_rows_x2(const Staged2
     int64_t c0, c1;
     (void)visit_plane(a.f, a.o0 + 2 * lp, c0);
     (void)visit_plane(a.f, a.o0 + 2 * lp + (has1 ? 1 : 0), c1);
+    // debug build: the planes and their kernel spectra exist (uniform over the CTA)
+    if (!(check_index(a.f.err, 2 * lp + (has1 ? 1 : 0), np) && check_index(a.f.err, c0, a.f.C) &&
+          check_index(a.f.err, c1, a.f.C) && check_index(a.f.err, a.n, a.f.order)))
+        return;
     float2 *w0 = a.ws + (2 * lp) * G::PLANE;
     float2 *w1 = a.ws + (2 * lp + (has1 ? 1 : 0)) * G::PLANE;
     const c32 *tws = a.f.tw + 2 * M2;
+    // the debug build checks the slot index of every shared access
     auto ld = [&](int ad) -> c32x2 {
+        if (!check_index(a.f.err, ad, NROW * M2)) return c32x2{f2(0.f, 0.f), f2(0.f, 0.f)};
         const float4 f = rowb[ad];
         return c32x2{f2(f.x, f.y), f2(f.z, f.w)};
     };
-    auto st = [&](int ad, c32x2 x) { rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y); };
+    auto st = [&](int ad, c32x2 x) {
+        if (check_index(a.f.err, ad, NROW * M2)) rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y);
+    };
 
     // the group's rows of both planes (data columns x' < XW), coalesced
     const uint64_t keep = l2_keep();

@@ -127,3 +127,11 @@ def test_launch_count_without_a_gpu(capi):
     assert capi.hyena_forward(None, 1, 16, [16], 16, None, 16) == capi.HYENA_ERR_INVALID_ARG
     assert capi.hyena_launch_count() == n0
     assert capi.lib.hyena_launch_count(None) == capi.HYENA_ERR_INVALID_ARG
+
+
+def test_debug_hooks_reject_bad_arguments(capi):
+    """The plan-failure test hooks check their arguments without a GPU."""
+    assert capi.lib.hyena_debug_fail_allocation(-1) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.lib.hyena_debug_fail_allocation(0) == capi.HYENA_OK
+    assert capi.lib.hyena_debug_plan_resources(None) == capi.HYENA_ERR_INVALID_ARG
+    assert capi.hyena_debug_plan_resources() >= 0
