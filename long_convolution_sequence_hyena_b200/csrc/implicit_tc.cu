@@ -137,6 +137,19 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *mbar, uint32_t par
     return false;
 }
 
+// sin x for the sine layers: Cody and Waite's reduction x = 2 pi k + r, with
+// 2 pi split into 6.28125 (8 significant bits, so k * 6.28125 is exact for
+// the k that occur) and 2 pi - 6.28125, then the hardware sine __sinf on
+// r in [-pi, pi], where its absolute error is below 2^-21.4. Arguments of
+// magnitude 8192 and more, far outside what the layers produce, go to sinf.
+__device__ __forceinline__ float sin_layer(float x) {
+    if (fabsf(x) >= 8192.f) return sinf(x);
+    const float k = rintf(x * 0.159154943091895336f);   // x / (2 pi)
+    float r = fmaf(-k, 6.28125f, x);
+    r = fmaf(-k, 1.93530717958647692e-3f, r);
+    return __sinf(r);
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -303,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
             float hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float v = in ? sinf(a.p.omega0 * (a1[4 * c + u] + S.b1[4 * kc + u])) : 0.f;
+                const float v = in ? sin_layer(a.p.omega0 * (a1[4 * c + u] + S.b1[4 * kc + u])) : 0.f;
                 hi[u] = tf32_hi(v);
                 lo[u] = v - hi[u];
             }
@@ -336,7 +349,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
             float hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float v = in ? sinf(a.p.omega_hidden * (r[4 * c + u] + S.b2[4 * kc + u])) : 0.f;
+                const float v = in ? sin_layer(a.p.omega_hidden * (r[4 * c + u] + S.b2[4 * kc + u])) : 0.f;
                 hi[u] = tf32_hi(v);
                 lo[u] = v - hi[u];
             }
