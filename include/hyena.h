@@ -249,10 +249,27 @@ HYENA_API hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_im
  * transform the filters in chunks through a device buffer that the plan
  * allocates at creation and owns. Those chunks run on the plan's own two
  * streams, forked from `stream` and joined back to it, so calls on one such
- * plan (from any stream or thread) run one after another on the GPU.
+ * plan (from any stream or thread) run one after another on the GPU;
+ * hyena_filter_spectrum_ws, with a workspace per caller, lets them overlap.
  */
 HYENA_API hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
                                      void *H_out, void *stream);
+
+/*
+ * hyena_filter_spectrum with the transforms' scratch supplied by the caller:
+ * workspace (device, 16-byte aligned) of at least
+ * hyena_filter_spectrum_workspace_bytes(plan) bytes, or NULL for the plan's
+ * own (then the same as hyena_filter_spectrum). With a workspace of its own
+ * each call is independent of the others on the plan: calls from several
+ * threads with separate workspaces overlap on the GPU (the plan's streams
+ * carry them, each call with its own fork and join events). A workspace that
+ * is too small is HYENA_ERR_WORKSPACE. Plans whose spectra need no scratch
+ * (hyena_filter_spectrum_workspace_bytes = 0) ignore it.
+ */
+HYENA_API hyena_status_t hyena_filter_spectrum_ws(hyena_plan_t plan, const float *h,
+                                                  const hyena_implicit_params_t *params, void *H_out,
+                                                  void *workspace, size_t ws_bytes, void *stream);
+HYENA_API size_t hyena_filter_spectrum_workspace_bytes(hyena_plan_t plan);
 
 /*
  * The fused forward pass: all N orders in one launch per row, each row read

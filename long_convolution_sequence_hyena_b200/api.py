@@ -104,16 +104,26 @@ class Plan:
         _check(capi.hyena_implicit_filter(self.handle, c, out.data_ptr(), _stream(stream)), "hyena_implicit_filter")
         return out
 
-    def filter_spectrum(self, h=None, implicit: dict | None = None, out=None, stream=None):
-        """Spectra as a complex64 tensor of ``spectrum_shape``."""
+    def filter_spectrum(self, h=None, implicit: dict | None = None, out=None, stream=None, workspace=None):
+        """Spectra as a complex64 tensor of ``spectrum_shape``. ``workspace``: a uint8 device tensor
+        of at least ``spectrum_workspace_bytes()`` for the transforms, so that calls on one plan
+        from several threads overlap (None: the plan's own scratch, one call at a time)."""
         if out is None:
             out = torch.empty(self.spectrum_shape, dtype=torch.complex64, device="cuda")
         c = implicit_params(implicit) if implicit is not None else None
         if h is not None:
             h = h.contiguous()
-        _check(capi.hyena_filter_spectrum(self.handle, _ptr(h), c, out.data_ptr(), _stream(stream)),
-               "hyena_filter_spectrum")
+        if workspace is None:
+            _check(capi.hyena_filter_spectrum(self.handle, _ptr(h), c, out.data_ptr(), _stream(stream)),
+                   "hyena_filter_spectrum")
+        else:
+            _check(capi.hyena_filter_spectrum_ws(self.handle, _ptr(h), c, out.data_ptr(), workspace.data_ptr(),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+                   "hyena_filter_spectrum_ws")
         return out
+
+    def spectrum_workspace_bytes(self) -> int:
+        return capi.lib.hyena_filter_spectrum_workspace_bytes(self.handle)
 
     def forward(self, v, gates, H, dskip=None, out=None, workspace=None, stream=None):
         if out is None:

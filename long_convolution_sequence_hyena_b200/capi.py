@@ -37,6 +37,7 @@ EXPORTED = (
     "hyena_forward_no_alloc", "hyena_forward_host_workspace_bytes", "hyena_forward_host",
     "hyena_forward_gated", "hyena_plan_set_layout", "hyena_plan_device_errors", "hyena_plan_create_ex",
     "hyena_launch_count", "hyena_debug_fail_allocation", "hyena_debug_plan_resources",
+    "hyena_filter_spectrum_ws", "hyena_filter_spectrum_workspace_bytes",
 )
 
 
@@ -76,6 +77,8 @@ def _load():
         "hyena_launch_count": ([ctypes.POINTER(i64)], i32),
         "hyena_debug_fail_allocation": ([i32], i32),
         "hyena_debug_plan_resources": ([ctypes.POINTER(i64)], i32),
+        "hyena_filter_spectrum_ws": ([p, p, ctypes.POINTER(hyena_implicit_params_t), p, p, sz, p], i32),
+        "hyena_filter_spectrum_workspace_bytes": ([p], sz),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -157,6 +160,11 @@ def hyena_implicit_filter(plan, params, h_out: int, stream: int = 0) -> int:
 
 def hyena_filter_spectrum(plan, h, params, H_out: int, stream: int = 0) -> int:
     return lib.hyena_filter_spectrum(plan, h, ctypes.byref(params) if params is not None else None, H_out, stream)
+
+
+def hyena_filter_spectrum_ws(plan, h, params, H_out: int, workspace, ws_bytes: int, stream: int = 0) -> int:
+    return lib.hyena_filter_spectrum_ws(plan, h, ctypes.byref(params) if params is not None else None, H_out,
+                                        workspace, ws_bytes, stream)
 
 
 def hyena_forward(plan, batch: int, v: int, gates, H: int, Dskip, y: int, workspace=None, ws_bytes: int = 0,

@@ -393,9 +393,27 @@ hyena_status_t hyena_implicit_filter(hyena_plan_t plan, const hyena_implicit_par
     return launch_implicit(a, plan->dev_err, (cudaStream_t)stream) == cudaSuccess ? HYENA_OK : HYENA_ERR_CUDA;
 }
 
+size_t hyena_filter_spectrum_workspace_bytes(hyena_plan_t plan) {
+    if (!plan) return 0;
+    if (plan->ndim == 1 && plan->path == HYENA_PATH_STAGED) return staged_spec_scratch_bytes(plan->MC);
+    if (plan->ndim == 2 && staged2d_supported(plan->Ww)) return staged2d_spec_scratch_bytes(plan->Ww);
+    return 0;
+}
+
 hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
                                      void *H_out, void *stream) {
+    return hyena_filter_spectrum_ws(plan, h, params, H_out, nullptr, 0, stream);
+}
+
+hyena_status_t hyena_filter_spectrum_ws(hyena_plan_t plan, const float *h, const hyena_implicit_params_t *params,
+                                        void *H_out, void *workspace, size_t ws_bytes, void *stream) {
     if (!plan || !H_out || (!h && !params)) return HYENA_ERR_INVALID_ARG;
+    // the transforms' scratch: the caller's workspace, or (none given) the plan's,
+    // whose lock then keeps each call's launch sequence together
+    const size_t ws_need = hyena_filter_spectrum_workspace_bytes(plan);
+    if (workspace && ws_bytes < ws_need) return HYENA_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
+    float2 *scratch = workspace ? reinterpret_cast<float2 *>(workspace) : plan->spec_ws;
     if (!aligned16(H_out) || (h && !aligned16(h))) return HYENA_ERR_ALIGNMENT;
     hyena_status_t s;
     if (!h && (s = check_implicit(plan, params)) != HYENA_OK) return s;
@@ -425,8 +443,9 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
         if (plan->path == HYENA_PATH_STAGED) {
             CallLanes cl(plan);
             if (!cl.ok) return HYENA_ERR_CUDA;
-            std::lock_guard<std::mutex> hold(*plan->spec_mu);
-            e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, plan->spec_ws, st, cl.l);
+            std::unique_lock<std::mutex> hold(*plan->spec_mu, std::defer_lock);
+            if (!workspace) hold.lock();
+            e = launch_spec_1d_staged(src, src_stride, plan->L, Hc, nrows, plan->MC, tw, scratch, st, cl.l);
         } else {
             e = plan->P3 ? launch_spec_1d_mr3(src, src_stride, plan->L, Hc, nrows, plan->P3, tw, st)
                 : plan->path == HYENA_PATH_CTA
@@ -446,8 +465,9 @@ hyena_status_t hyena_filter_spectrum(hyena_plan_t plan, const float *h, const hy
         if (plan->spec_ws) {
             CallLanes cl(plan);
             if (!cl.ok) return HYENA_ERR_CUDA;
-            std::lock_guard<std::mutex> hold(*plan->spec_mu);
-            e = launch_spec_2d_staged(src, rs, cs, Hc, nrows, plan->Ww, tw, plan->spec_ws, st, cl.l);
+            std::unique_lock<std::mutex> hold(*plan->spec_mu, std::defer_lock);
+            if (!workspace) hold.lock();
+            e = launch_spec_2d_staged(src, rs, cs, Hc, nrows, plan->Ww, tw, scratch, st, cl.l);
         } else {
             e = launch_spec_2d(src, rs, cs, Hc, nrows, plan->Ww, tw, st);
         }

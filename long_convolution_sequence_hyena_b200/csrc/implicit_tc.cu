@@ -142,8 +142,9 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *mbar, uint32_t par
 // the k that occur) and 2 pi - 6.28125, then the hardware sine __sinf on
 // r in [-pi, pi], where its absolute error is below 2^-21.4. Arguments of
 // magnitude 8192 and more, far outside what the layers produce, go to sinf.
+__device__ __noinline__ float sin_large(float x) { return sinf(x); }   // kept out of the hot code
 __device__ __forceinline__ float sin_layer(float x) {
-    if (fabsf(x) >= 8192.f) return sinf(x);
+    if (fabsf(x) >= 8192.f) return sin_large(x);
     const float k = rintf(x * 0.159154943091895336f);   // x / (2 pi)
     float r = fmaf(-k, 6.28125f, x);
     r = fmaf(-k, 1.93530717958647692e-3f, r);
@@ -213,11 +214,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
+// NDIM: the grid's dimension (1, 2 or 3), fixed per instance so that each holds
+// only its own feature and window code.
+template <int NDIM>
 __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const ImplicitArgs a, int *err) {
     extern __shared__ float4 tc_smem4[];
     TcSmem &S = *reinterpret_cast<TcSmem *>(tc_smem4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int fin = a.ndim == 1 ? 1 + 2 * a.p.num_freqs : a.ndim;
+    const int fin = NDIM == 1 ? 1 + 2 * a.p.num_freqs : NDIM;
     const int64_t p0 = (int64_t)blockIdx.x * TP;
 
     // first-layer weights and biases, W2 as the B tile, the barrier and tensor memory
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
                 a1[4 * j4 + 3] = fmaf(w.w, fv, a1[4 * j4 + 3]);
             }
         };
-        if (a.ndim == 1) {
+        if constexpr (NDIM == 1) {
             // [t/L, cos(2 pi k t/L), sin(2 pi k t/L) for k = 1..K]: the angle's turns
             // (k t mod L) / L advance by t per frequency, kept exact in integers
             // (t < L <= 2^19, so k t fits in 32 bits)
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
                 float fv = 0.f;
                 if (in) {   // offsets on grids of at most 2^21 points: 32-bit index arithmetic
                     const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, pi = (int)pos;
-                    if (a.ndim == 2) {
+                    if constexpr (NDIM == 2) {
                         const int iy = pi / W2, ix = pi - iy * W2;
                         fv = f == 0 ? __fdiv_rn((float)(iy - Hi), (float)Hi) : __fdiv_rn((float)(ix - Wi), (float)Wi);
                     } else {   // 3D: (oz / Dz, oy / H, ox / W) on the offset grid [2Dz][2H][2W]
@@ -368,15 +372,17 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
     const int64_t ppos = p0 + prow;
     float we = 0.f;                                    // window exponent argument: t (1D) or |p|^2 (2D, 3D)
     int64_t poff = ppos;
-    if (a.ndim == 1) {
+    if constexpr (NDIM == 1) {
         we = (float)ppos;
-    } else if (a.ndim == 2 && ppos < a.npos) {
+    } else if (NDIM == 2) {
+        if (ppos < a.npos) {
         const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, pi = (int)ppos;
         const int iy = pi / W2, ix = pi - iy * W2;
         const float py = __fdiv_rn((float)(iy - Hi), (float)Hi), px = __fdiv_rn((float)(ix - Wi), (float)Wi);
         we = py * py + px * px;
         poff = (int64_t)iy * a.out_row_stride + ix;
-    } else if (a.ndim == 3 && ppos < a.npos) {   // output [2Dz][2H][2W] contiguous per channel
+        }
+    } else if (ppos < a.npos) {   // 3D: output [2Dz][2H][2W] contiguous per channel
         const int W2 = 2 * (int)a.W, Hi = (int)a.H, Wi = (int)a.W, Dzi = (int)a.Dz, pi = (int)ppos;
         const int hw = 2 * Hi * W2;
         const int iz = pi / hw, rem = pi - iz * hw;
@@ -417,7 +423,7 @@ __global__ void __launch_bounds__(THREADS, 2) hyena_implicit_tc_kernel(const Imp
         if (tid < NT && os + tid < o_end) {
             const float wp = __ldg(a.p.window + os + tid);
             // exp(-alpha t) (1D) or exp(-|p|^2 / (2 sigma^2)) (2D, 3D), as 2^(scale * arg)
-            const float esc = a.ndim == 1 ? -wp : -1.f / (2.f * wp * wp);
+            const float esc = NDIM == 1 ? -wp : -1.f / (2.f * wp * wp);
             oc_new = make_float2(esc * 1.4426950408889634f, __ldg(a.p.b3 + os + tid));
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -450,10 +456,12 @@ size_t implicit_tc_smem_bytes(int fin) { return sizeof(TcSmem) + (size_t)(fin - 
 
 cudaError_t launch_implicit_tc(const ImplicitArgs &a, int *err, cudaStream_t st) {
     const int sm = (int)implicit_tc_smem_bytes(a.ndim == 1 ? 1 + 2 * a.p.num_freqs : a.ndim);
-    cudaError_t e = cudaFuncSetAttribute(hyena_implicit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    auto kern = a.ndim == 1 ? hyena_implicit_tc_kernel<1> : (a.ndim == 2 ? hyena_implicit_tc_kernel<2>
+                                                                          : hyena_implicit_tc_kernel<3>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.npos + TP - 1) / TP), (unsigned)((a.nout + SLICE_OUT - 1) / SLICE_OUT));
-    hyena_implicit_tc_kernel<<<grid, THREADS, sm, st>>>(a, err);
+    kern<<<grid, THREADS, sm, st>>>(a, err);
     return launched();
 }
 

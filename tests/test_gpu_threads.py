@@ -13,8 +13,11 @@ import torch
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("own_ws", [False, True])
 @pytest.mark.parametrize("shape,B,D,N", [((32768,), 2, 80, 2), ((256, 256), 1, 70, 1)])
-def test_concurrent_calls_on_one_plan(shape, B, D, N):
+def test_concurrent_calls_on_one_plan(shape, B, D, N, own_ws):
+    """own_ws: each thread's spectrum calls bring their own scratch
+    (hyena_filter_spectrum_ws), so they need not wait for each other."""
     from long_convolution_sequence_hyena_b200 import api
 
     plan = api.Plan(shape, D, N, torch.bfloat16)
@@ -36,6 +39,8 @@ def test_concurrent_calls_on_one_plan(shape, B, D, N):
         sets.append(dict(v=v, gates=gates, dskip=dskip, h=h, H_ref=H_ref, y_ref=y_ref,
                          H=torch.empty_like(H_ref), y=torch.empty_like(y_ref),
                          ws=torch.empty(max(1, plan.workspace_bytes(B)), dtype=torch.uint8, device="cuda"),
+                         sws=(torch.empty(max(1, plan.spectrum_workspace_bytes()), dtype=torch.uint8, device="cuda")
+                              if own_ws else None),
                          stream=torch.cuda.Stream()))
     torch.cuda.synchronize()
     errors = []
@@ -44,7 +49,7 @@ def test_concurrent_calls_on_one_plan(shape, B, D, N):
         try:
             torch.cuda.set_device(0)
             for it in range(12):
-                plan.filter_spectrum(h=s["h"], out=s["H"], stream=s["stream"])
+                plan.filter_spectrum(h=s["h"], out=s["H"], stream=s["stream"], workspace=s["sws"])
                 plan.forward(s["v"], s["gates"], s["H"], s["dskip"], out=s["y"], workspace=s["ws"],
                              stream=s["stream"])
                 s["stream"].synchronize()
@@ -62,3 +67,24 @@ def test_concurrent_calls_on_one_plan(shape, B, D, N):
     assert not any(t.is_alive() for t in threads)
     assert not errors, errors
     plan.close()
+
+
+def test_spectrum_workspace_checks():
+    from long_convolution_sequence_hyena_b200 import api, capi
+    plan = api.Plan((65536,), 4, 1, torch.float32)
+    need = plan.spectrum_workspace_bytes()
+    assert need > 0
+    h = torch.randn(1, 4, 65536, device="cuda")
+    H = torch.empty(plan.spectrum_shape, dtype=torch.complex64, device="cuda")
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    assert capi.hyena_filter_spectrum_ws(plan.handle, h.data_ptr(), None, H.data_ptr(), small.data_ptr(),
+                                         small.numel(), 0) == capi.HYENA_ERR_WORKSPACE
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    H1 = plan.filter_spectrum(h=h, workspace=ws)
+    H2 = plan.filter_spectrum(h=h)
+    torch.cuda.synchronize()
+    assert torch.equal(H1, H2)
+    plan2 = api.Plan((2048,), 4, 1, torch.float32)   # spectra without scratch
+    assert plan2.spectrum_workspace_bytes() == 0
+    plan.close()
+    plan2.close()
