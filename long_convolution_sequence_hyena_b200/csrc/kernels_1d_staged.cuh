@@ -126,6 +126,23 @@ __global__ void __launch_bounds__(G::CT, G::CMINB) hyena_staged_cols_x2(const St
     const c32 *tws = a.f.tw + M;                     // W_1024
     auto pos_of = [&](int q) -> int64_t { return 2 * ((int64_t)M2 * (t1 + q * T1) + n2); };
 
+    // The columns read their input (v, or this order's gate) in sectors 1 KB and
+    // more apart, which DRAM serves poorly. The chunk's rows are contiguous, so
+    // each CTA first brings its share of its two rows (1/CGROUPS of each) into
+    // L2 in one bulk prefetch per row; the column loads then meet L2.
+    if (a.f.es == 1 && threadIdx.x < 2 && (threadIdx.x == 0 || has1)) {
+        const IO *in = MODE == 0 ? reinterpret_cast<const IO *>(a.f.v)
+                                 : reinterpret_cast<const IO *>(a.f.gates[a.n]);
+        const uintptr_t row_start = reinterpret_cast<uintptr_t>(in + (threadIdx.x ? row1 : row0) * L);
+        const int64_t row_bytes = L * (int64_t)sizeof(IO);
+        const int64_t piece = ((row_bytes + G::CGROUPS - 1) / G::CGROUPS + 15) & ~(int64_t)15;
+        const int64_t off = (int64_t)cgp * piece;
+        int64_t len = row_bytes - off < piece ? row_bytes - off : piece;
+        len &= ~(int64_t)15;   // whole 16-byte blocks inside the row
+        if ((row_start & 15) == 0 && len > 0)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row_start + off), "r"((uint32_t)len)
+                         : "memory");
+    }
     c32x2 v[E];
     if constexpr (MODE == 0) {
         const IO *r0 = reinterpret_cast<const IO *>(a.f.v) + act_row_off(a.f, row0);
@@ -230,6 +247,21 @@ __global__ void __launch_bounds__(G::RT, G::RMINB) hyena_staged_rows_x2(const St
         if (check_index(a.f.err, ad, NROW * M2)) rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y);
     };
 
+    // The spectrum bins of a row group lie 2 KB apart in the channel's spectrum
+    // row, which DRAM serves poorly. The RGROUPS CTAs of a row pair cover both
+    // rows' spectra, so each first brings 1/RGROUPS of them (a contiguous run
+    // of 16-byte blocks inside the row) into L2 with one bulk prefetch per row.
+    if (threadIdx.x < 2 && (threadIdx.x == 0 || d1 != d0)) {
+        const uintptr_t rs =
+            reinterpret_cast<uintptr_t>(a.f.H + ((int64_t)a.n * a.f.hD + (threadIdx.x ? d1 : d0)) * (MC + 1));
+        const uintptr_t re = rs + (uintptr_t)(MC + 1) * 8;
+        const uintptr_t piece = (((uintptr_t)(MC + 1) * 8 + G::RGROUPS - 1) / G::RGROUPS + 15) & ~(uintptr_t)15;
+        const uintptr_t b = (rs + (uintptr_t)g * piece + 15) & ~(uintptr_t)15;
+        uintptr_t e = rs + (uintptr_t)(g + 1) * piece;
+        e = (e < re ? e : re) & ~(uintptr_t)15;
+        if (e > b)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(b), "r"((uint32_t)(e - b)) : "memory");
+    }
     // the group's rows of both lanes, coalesced, into the sequence-major buffer
     const uint64_t keep = l2_keep(), stream = l2_stream();
 #pragma unroll
