@@ -76,6 +76,23 @@ __global__ void __launch_bounds__(G::CT, 3) hyena_staged2d_cols(const Staged2dAr
     // register q holds row y = t1 + q T1 of column x'; rows y < H (q < E/2) carry data
     auto pos_of = [&](int q) -> int64_t { return (int64_t)(t1 + q * T1) * Ww + 2 * xc; };
 
+    // The columns read their plane in sectors a row (2W bytes and more) apart,
+    // which DRAM serves poorly. The CGROUPS CTAs of a plane cover all of it, so
+    // each first brings 1/CGROUPS of the plane's input (v and, for the gate
+    // sandwich, k; or this order's gate) into L2 with one bulk prefetch each.
+    if (threadIdx.x < (MODE == 0 && GATED ? 2 : 1)) {
+        const IO *in = MODE != 0 ? reinterpret_cast<const IO *>(a.f.gates[a.n])
+                                 : reinterpret_cast<const IO *>(threadIdx.x ? a.f.k : a.f.v);
+        const uintptr_t ps = reinterpret_cast<uintptr_t>(in + plane * plane_elems);
+        const int64_t plane_bytes = plane_elems * (int64_t)sizeof(IO);
+        const int64_t piece = ((plane_bytes + G::CGROUPS - 1) / G::CGROUPS + 15) & ~(int64_t)15;
+        const int64_t off = (int64_t)cgp * piece;
+        int64_t len = plane_bytes - off < piece ? plane_bytes - off : piece;
+        len &= ~(int64_t)15;
+        if ((ps & 15) == 0 && len > 0)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ps + off), "r"((uint32_t)len)
+                         : "memory");
+    }
     c32 v[E];
     if constexpr (MODE == 0) {
         const IO *vp = reinterpret_cast<const IO *>(a.f.v) + plane * plane_elems;
@@ -157,6 +174,22 @@ __global__ void __launch_bounds__(G::RT, 3) hyena_staged2d_rows_x2(const Staged2
         if (check_index(a.f.err, ad, NROW * M2)) rowb[ad] = make_float4(x.re.x, x.re.y, x.im.x, x.im.y);
     };
 
+    // The kernel-spectrum bins of a row group lie 2H bins apart, which DRAM
+    // serves poorly. The RGROUPS CTAs of a plane pair cover both planes'
+    // spectra, so each first brings 1/RGROUPS of them (a contiguous run of
+    // 16-byte blocks inside the channel's spectrum) into L2, one bulk prefetch
+    // per channel.
+    if (threadIdx.x < 2 && (threadIdx.x == 0 || c1 != c0)) {
+        const uintptr_t ks = reinterpret_cast<uintptr_t>(
+            a.f.K + ((int64_t)a.n * a.f.C + (threadIdx.x ? c1 : c0)) * (int64_t)(M1 * (M2 + 1)));
+        const uintptr_t ke = ks + (uintptr_t)(M1 * (M2 + 1)) * 8;
+        const uintptr_t piece = (((uintptr_t)(M1 * (M2 + 1)) * 8 + G::RGROUPS - 1) / G::RGROUPS + 15) & ~(uintptr_t)15;
+        const uintptr_t b = (ks + (uintptr_t)g * piece + 15) & ~(uintptr_t)15;
+        uintptr_t e = ks + (uintptr_t)(g + 1) * piece;
+        e = (e < ke ? e : ke) & ~(uintptr_t)15;
+        if (e > b)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(b), "r"((uint32_t)(e - b)) : "memory");
+    }
     // the group's rows of both planes (data columns x' < XW), coalesced
     const uint64_t keep = l2_keep();
 #pragma unroll
