@@ -91,6 +91,15 @@ int main(void) {
     int64_t launches = -1;
     if (hyena_launch_count(NULL) != HYENA_ERR_INVALID_ARG) bad = 9;
     if (hyena_launch_count(&launches) != HYENA_OK || launches != 0) bad = 10;
+    if (hyena_filter_spectrum_ws(NULL, NULL, NULL, NULL, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG) bad = 11;
+    if (hyena_filter_spectrum_workspace_bytes(NULL) != 0) bad = 12;
+    if (hyena_debug_fail_allocation(-1) != HYENA_ERR_INVALID_ARG) bad = 13;
+    if (hyena_debug_fail_allocation(0) != HYENA_OK) bad = 14;
+    if (hyena_debug_plan_resources(NULL) != HYENA_ERR_INVALID_ARG) bad = 15;
+    if (hyena_plan_device_errors(NULL, NULL, 0) != HYENA_ERR_INVALID_ARG) bad = 16;
+    if (hyena_plan_set_layout(NULL, HYENA_LAYOUT_BLD) != HYENA_ERR_INVALID_ARG) bad = 17;
+    if (hyena_forward_gated(NULL, 1, NULL, NULL, gates, NULL, NULL, NULL, NULL, 0, NULL) != HYENA_ERR_INVALID_ARG)
+        bad = 18;
     printf("%s\n", bad ? "FAIL" : "OK");
     return bad;
 }
