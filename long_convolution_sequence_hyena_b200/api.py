@@ -45,7 +45,7 @@ def implicit_params(p: dict) -> capi.hyena_implicit_params_t:
 
 
 class Plan:
-    """A plan for one geometry: shape (L,) or (H, W), channels, order, io dtype, and the
+    """A plan for one geometry: shape (L,), (H, W) or (Dz, H, W), channels, order, io dtype, and the
     activation layout of 1D plans: "bdl" ([B, D, L], the default) or "bld" ([B, L, D],
     channels-last, read and written in place). radix3: a 1D plan may pad to M = 6 * 2^j
     when that is below the power of two."""
