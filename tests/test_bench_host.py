@@ -52,3 +52,36 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1, out.stdout
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0
+
+
+def test_cost_model_of_the_default_workload():
+    """The roofline convention, worked by hand for order 3, bf16, B 1, D 768, L 65536
+    (M = 131072): v, three gates and y at 2 bytes per element, every spectrum row
+    (M/2 + 1 complex64 bins) and Dskip once; two 5 M log2 M transforms per row and order."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_convolution_sequence_hyena_b200.workloads import WORKLOADS
+    c = bench.cost_model(WORKLOADS["order3_bf16_b1_d768_l65536"])
+    assert c["M"] == 131072
+    act = 5 * 768 * 65536 * 2
+    spec = 3 * 768 * 65537 * 8
+    assert c["bytes"] == act + spec + 3 * 768 * 4 == 1711303680
+    assert c["flops"] == 2 * 3 * 768 * 5.0 * 131072 * 17
+    g = bench.cost_model(WORKLOADS["gated_order1_bf16_2d_b2_c256_256x256"])
+    # q, k, one gate and y over B C H W, the kernel spectra [C, W + 1, 2H], Dskip
+    assert g["bytes"] == 4 * 2 * 256 * 256 * 256 * 2 + 256 * 257 * 512 * 8 + 256 * 4
+
+
+def test_traffic_record_is_tied_to_the_sources(monkeypatch):
+    """A committed DRAM-traffic record is reported only for the source version it was
+    taken at."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_convolution_sequence_hyena_b200 import build
+    from long_convolution_sequence_hyena_b200.workloads import WORKLOADS
+    w = WORKLOADS["order3_bf16_b1_d768_l65536"]
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic_%s.json" % w.name)))
+    monkeypatch.setattr(build, "source_hash", lambda: rec["source_hash"])
+    assert bench.traffic_record(w) == rec["dram_bytes_per_launch"]
+    monkeypatch.setattr(build, "source_hash", lambda: "0" * 16)
+    assert bench.traffic_record(w) is None
